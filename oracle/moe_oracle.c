@@ -1,0 +1,383 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU oracle for MoE
+ * expert-parallel dispatch and combine with their layout metadata.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file.  Only the test suite, the package smoke check and the
+ * CPU-baseline leg of the benchmark use it.  It shares no code, header,
+ * table or helper with the CUDA library; the two meet only through the
+ * seeded input generator.
+ *
+ * What it computes, and where the pages say so:
+ *
+ *  - Expert -> rank partition.  "[None][feat] support non-divisible EP in MoE
+ *    alltoall and slurm benchmark" (TensorRT-LLM PR #13888), PR description
+ *    ("ceil/floor contiguous partitioning") and the commit that adds the
+ *    divisible fast path (base = E / R, remainder = E mod R, example 256
+ *    experts on 7 ranks -> base 36, remainder 4).  Reading taken: ranks are
+ *    filled in order with contiguous experts and the first `remainder` ranks
+ *    hold one extra expert.  Here that is a plain loop over ranks, not the
+ *    closed form.
+ *  - E < R is refused up front.  Same PR, review thread on num_experts <
+ *    ep_size (a clear error instead of ranks with no experts).
+ *  - Layout ("segment descriptors").  FUSCO article (aigc.bar), section
+ *    "FUSCO 的核心创新": gather-send reads scattered rows by segment
+ *    descriptor, scatter-recv writes each row straight into its final
+ *    position.  The descriptor contents are not given; the reading taken is
+ *    an expert-major receive buffer of exactly T*k rows, ordered inside each
+ *    expert by ascending token index, with per-expert counts/offsets,
+ *    per-rank offsets and a per-(token, slot) destination row.
+ *  - Dispatch.  INC-MoE abstract (dispatch moves each token to the devices
+ *    hosting its selected experts) and the FUSCO article section above: one
+ *    copy of x[t] lands in every destination row of token t.
+ *  - Two-level dispatch.  FUSCO article, section "负载均衡与跨节点去重":
+ *    a token bound for several GPUs of one node crosses nodes once, to a
+ *    forwarding GPU that fans it out inside the node.  Here: one staging row
+ *    per (token, node touched), node-major then token order, then expansion
+ *    from staging to the expert rows of that node.
+ *  - Combine.  INC-MoE abstract (combine returns expert outputs to each
+ *    token's owner) with the reduction by gate weight.  The pages fix no
+ *    order or precision; the reading taken is fp32 accumulation with one
+ *    fused multiply-add per selected expert in top-k column order j = 0..k-1,
+ *    starting from +0.0f, and one round-to-nearest-even store to bf16.
+ *
+ * Build: cc -std=c99 -O2 -ffp-contract=off -shared -fPIC (so that the only
+ * fused multiply-add is the explicit fmaf call).
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+
+/* Status codes.  Their meaning mirrors the library's public status enum by
+ * convention (same numbers, same meaning); they are defined here on their
+ * own so the oracle needs no header of the library. */
+enum {
+    ORC_OK = 0,
+    ORC_INVALID_ARG = 1,
+    ORC_EMPTY_RANK = 2,
+    ORC_BAD_NODES = 3,
+    ORC_EXPERT_OOB = 4,
+    ORC_DUP_EXPERT = 5
+};
+
+/* ------------------------------------------------------------------ */
+/* bf16 <-> fp32, from the IEEE-754 binary32 layout                    */
+/* ------------------------------------------------------------------ */
+
+/* bf16 is the upper half of a binary32: widening is a 16-bit shift. */
+float oracle_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Narrowing with round-to-nearest, ties-to-even, written from the
+ * definition: keep the upper 16 bits, look at the 16 discarded bits, round
+ * up when they exceed one half, or equal one half and the kept part is odd.
+ * A carry out of the mantissa moves into the exponent, which is the correct
+ * result (up to and including overflow to infinity).  NaN stays NaN: the
+ * sign and upper payload are kept and the quiet bit is forced so that the
+ * truncated payload can never read as infinity. */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t exp_bits = (u >> 23) & 0xFFu;
+    uint32_t man_bits = u & 0x7FFFFFu;
+    if (exp_bits == 0xFFu && man_bits != 0u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t kept = u >> 16;
+    uint32_t dropped = u & 0xFFFFu;
+    int round_up = 0;
+    if (dropped > 0x8000u)
+        round_up = 1;
+    else if (dropped == 0x8000u && (kept & 1u))
+        round_up = 1;
+    return (uint16_t)(kept + (uint32_t)round_up);
+}
+
+void oracle_f32_to_bf16_array(const float *src, uint16_t *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = oracle_f32_to_bf16(src[i]);
+}
+
+void oracle_bf16_to_f32_array(const uint16_t *src, float *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = oracle_bf16_to_f32(src[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* Partition                                                           */
+/* ------------------------------------------------------------------ */
+
+/* Fill rank_first_expert[0..R] by walking the ranks in order and giving each
+ * one base experts, plus one more while the remainder lasts. */
+int oracle_partition(int32_t E, int32_t R, int32_t *rank_first_expert)
+{
+    if (E < 1 || R < 1 || rank_first_expert == NULL)
+        return ORC_INVALID_ARG;
+    if (E < R)
+        return ORC_EMPTY_RANK;
+    int32_t base = E / R;
+    int32_t extra_left = E - base * R;
+    int32_t next = 0;
+    for (int32_t r = 0; r < R; ++r) {
+        rank_first_expert[r] = next;
+        int32_t size = base;
+        if (extra_left > 0) {
+            size += 1;
+            extra_left -= 1;
+        }
+        next += size;
+    }
+    rank_first_expert[R] = next;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Validation                                                          */
+/* ------------------------------------------------------------------ */
+
+int oracle_validate_config(int64_t T, int32_t H, int32_t E, int32_t k,
+                           int32_t R, int32_t N)
+{
+    if (T < 0 || H < 1 || E < 1 || R < 1 || N < 1 || k < 1)
+        return ORC_INVALID_ARG;
+    if (k > E)
+        return ORC_INVALID_ARG;
+    if (E < R)
+        return ORC_EMPTY_RANK;
+    if (N > R || (R % N) != 0)
+        return ORC_BAD_NODES;
+    return ORC_OK;
+}
+
+/* Every index lies in [0, E) and no token names one expert twice.  An
+ * out-of-range index is reported before a repeat when both occur. */
+int oracle_validate_topk(int64_t T, int32_t k, int32_t E, const int32_t *topk)
+{
+    int any_dup = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t e = topk[t * k + j];
+            if (e < 0 || e >= E)
+                return ORC_EXPERT_OOB;
+            for (int32_t i = 0; i < j; ++i)
+                if (topk[t * k + i] == e)
+                    any_dup = 1;
+        }
+    }
+    return any_dup ? ORC_DUP_EXPERT : ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Layout                                                              */
+/* ------------------------------------------------------------------ */
+
+/* topk:            int32 [T][k] row-major
+ * expert_counts:   int32 [E]
+ * expert_offsets:  int32 [E+1]   exclusive prefix of counts
+ * rank_offsets:    int32 [R+1]   first receive row of each rank
+ * slot:            int32 [T][k]  destination row of (t, j)
+ * node_counts:     int32 [N]     tokens touching node n   (optional)
+ * node_offsets:    int32 [N+1]   exclusive prefix         (optional)
+ * node_slot:       int32 [T][N]  rank of t among tokens touching n, or -1
+ *                                                         (optional)
+ * The three node arrays are either all NULL or all given. */
+int oracle_layout(int64_t T, int32_t k, int32_t E, int32_t R, int32_t N,
+                  const int32_t *topk,
+                  int32_t *expert_counts, int32_t *expert_offsets,
+                  int32_t *rank_offsets, int32_t *slot,
+                  int32_t *node_counts, int32_t *node_offsets,
+                  int32_t *node_slot)
+{
+    int st = oracle_validate_config(T, 1, E, k, R, N);
+    if (st != ORC_OK)
+        return st;
+    st = oracle_validate_topk(T, k, E, topk);
+    if (st != ORC_OK)
+        return st;
+
+    /* counts, then offsets as an exclusive prefix sum over experts */
+    for (int32_t e = 0; e < E; ++e)
+        expert_counts[e] = 0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j)
+            expert_counts[topk[t * k + j]] += 1;
+    int64_t run = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        expert_offsets[e] = (int32_t)run;
+        run += expert_counts[e];
+    }
+    expert_offsets[E] = (int32_t)run;
+
+    int32_t *first = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R + 1));
+    if (first == NULL)
+        return ORC_INVALID_ARG;
+    oracle_partition(E, R, first);
+    for (int32_t r = 0; r <= R; ++r)
+        rank_offsets[r] = expert_offsets[first[r]];
+
+    /* slots: one cursor per expert, walked in token order */
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (cursor == NULL) {
+        free(first);
+        return ORC_INVALID_ARG;
+    }
+    for (int32_t e = 0; e < E; ++e)
+        cursor[e] = expert_offsets[e];
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int32_t e = topk[t * k + j];
+            slot[t * k + j] = cursor[e];
+            cursor[e] += 1;
+        }
+    free(cursor);
+
+    if (node_counts != NULL && node_offsets != NULL && node_slot != NULL) {
+        int32_t ranks_per_node = R / N;
+        int32_t *node_of_expert = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+        int32_t *ncursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+        if (node_of_expert == NULL || ncursor == NULL) {
+            free(node_of_expert);
+            free(ncursor);
+            free(first);
+            return ORC_INVALID_ARG;
+        }
+        for (int32_t r = 0; r < R; ++r)
+            for (int32_t e = first[r]; e < first[r + 1]; ++e)
+                node_of_expert[e] = r / ranks_per_node;
+        for (int32_t n = 0; n < N; ++n)
+            ncursor[n] = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            for (int32_t n = 0; n < N; ++n) {
+                int touched = 0;
+                for (int32_t j = 0; j < k; ++j)
+                    if (node_of_expert[topk[t * k + j]] == n)
+                        touched = 1;
+                if (touched) {
+                    node_slot[t * N + n] = ncursor[n];
+                    ncursor[n] += 1;
+                } else {
+                    node_slot[t * N + n] = -1;
+                }
+            }
+        }
+        int64_t nrun = 0;
+        for (int32_t n = 0; n < N; ++n) {
+            node_counts[n] = ncursor[n];
+            node_offsets[n] = (int32_t)nrun;
+            nrun += ncursor[n];
+        }
+        node_offsets[N] = (int32_t)nrun;
+        free(node_of_expert);
+        free(ncursor);
+    }
+    free(first);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dispatch                                                            */
+/* ------------------------------------------------------------------ */
+
+/* recv[slot[t][j]] = x[t] for every (t, j).  Rows are H bf16 values. */
+void oracle_dispatch_flat(int64_t T, int32_t H, int32_t k,
+                          const int32_t *slot, const uint16_t *x,
+                          uint16_t *recv)
+{
+    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int64_t dst = slot[t * k + j];
+            memcpy(recv + dst * H, x + t * H, row_bytes);
+        }
+}
+
+/* Two-level dispatch.  Phase 1: x[t] goes once into the staging region of
+ * every node it touches (row node_offsets[n] + node_slot[t][n]).  Phase 2:
+ * for each node, in node order, each staging row is copied from staging to
+ * every expert row of its token that lies on that node.  A row lies on node
+ * n when its receive row falls in node n's rank range
+ * [rank_offsets[n*R/N], rank_offsets[(n+1)*R/N]). */
+void oracle_dispatch_two_level(int64_t T, int32_t H, int32_t k, int32_t R,
+                               int32_t N, const int32_t *slot,
+                               const int32_t *rank_offsets,
+                               const int32_t *node_offsets,
+                               const int32_t *node_slot,
+                               const uint16_t *x, uint16_t *staging,
+                               uint16_t *recv)
+{
+    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+    int32_t ranks_per_node = R / N;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t n = 0; n < N; ++n) {
+            int32_t ns = node_slot[t * N + n];
+            if (ns >= 0) {
+                int64_t row = (int64_t)node_offsets[n] + ns;
+                memcpy(staging + row * H, x + t * H, row_bytes);
+            }
+        }
+    for (int32_t n = 0; n < N; ++n) {
+        int32_t lo = rank_offsets[n * ranks_per_node];
+        int32_t hi = rank_offsets[(n + 1) * ranks_per_node];
+        for (int64_t t = 0; t < T; ++t) {
+            int32_t ns = node_slot[t * N + n];
+            if (ns < 0)
+                continue;
+            int64_t srow = (int64_t)node_offsets[n] + ns;
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t dst = slot[t * k + j];
+                if (dst >= lo && dst < hi)
+                    memcpy(recv + (int64_t)dst * H, staging + srow * H, row_bytes);
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Combine                                                             */
+/* ------------------------------------------------------------------ */
+
+/* y[t][h] = bf16_rne( fma(w[t][k-1], eo[slot[t][k-1]][h], ...
+ *                      fma(w[t][0], eo[slot[t][0]][h], +0.0f)) ) */
+void oracle_combine(int64_t T, int32_t H, int32_t k, const int32_t *slot,
+                    const float *w, const uint16_t *eo, uint16_t *y)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                int64_t row = slot[t * k + j];
+                float v = oracle_bf16_to_f32(eo[row * H + h]);
+                acc = fmaf(w[t * k + j], v, acc);
+            }
+            y[t * H + h] = oracle_f32_to_bf16(acc);
+        }
+}
+
+/* Same sum for a chosen list of tokens only; y_rows is [n_tokens][H].  Used
+ * to check large workloads on sampled tokens. */
+void oracle_combine_tokens(int64_t n_tokens, const int64_t *tokens,
+                           int32_t H, int32_t k, const int32_t *slot,
+                           const float *w, const uint16_t *eo,
+                           uint16_t *y_rows)
+{
+    for (int64_t i = 0; i < n_tokens; ++i) {
+        int64_t t = tokens[i];
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                int64_t row = slot[t * k + j];
+                float v = oracle_bf16_to_f32(eo[row * H + h]);
+                acc = fmaf(w[t * k + j], v, acc);
+            }
+            y_rows[i * H + h] = oracle_f32_to_bf16(acc);
+        }
+    }
+}
