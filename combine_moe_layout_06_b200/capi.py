@@ -1,0 +1,199 @@
+"""Python binding of libmoe_layout.so (include/moe_layout.h).
+
+Argument marshalling only: every entry point forwards to the C function of
+the same name, and all device work runs in the library's CUDA kernels.
+Tensors (anything with ``data_ptr()``) or raw integer addresses may be passed
+where the C ABI takes a pointer; ``stream`` may be a ``torch.cuda.Stream``,
+a raw ``cudaStream_t`` integer, or ``None`` for torch's current stream.
+
+If the shared library has not been built this module raises on first use;
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_layout.so")
+
+MOE_MAX_EXPERTS = 1024
+MOE_MAX_TOPK = 32
+MOE_MAX_NODES = 32
+
+MOE_FLAG_TWO_LEVEL = 0x1
+MOE_FLAG_COPY_VECTOR = 0x2
+MOE_FLAG_COPY_BULK = 0x4
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_EMPTY_RANK = 2
+MOE_ERR_BAD_NODES = 3
+MOE_ERR_EXPERT_OOB = 4
+MOE_ERR_DUP_EXPERT = 5
+MOE_ERR_TIMEOUT = 6
+MOE_ERR_CUDA = 7
+MOE_ERR_BAD_LAYOUT = 8
+
+STATUS_NAMES = {
+    MOE_OK: "OK", MOE_ERR_INVALID_ARG: "INVALID_ARG", MOE_ERR_EMPTY_RANK: "EMPTY_RANK",
+    MOE_ERR_BAD_NODES: "BAD_NODES", MOE_ERR_EXPERT_OOB: "EXPERT_OOB",
+    MOE_ERR_DUP_EXPERT: "DUP_EXPERT", MOE_ERR_TIMEOUT: "TIMEOUT", MOE_ERR_CUDA: "CUDA",
+    MOE_ERR_BAD_LAYOUT: "BAD_LAYOUT",
+}
+
+# Every entry point the header declares, in declaration order.
+ENTRY_POINTS = (
+    "moe_status_string", "moe_check_config", "moe_expert_partition",
+    "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
+    "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
+)
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("num_tokens", ctypes.c_int64), ("hidden", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("num_ranks", ctypes.c_int32), ("num_nodes", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+class MoeLayout(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "expert_counts", "expert_offsets", "rank_offsets", "slot", "node_counts",
+        "node_offsets", "node_slot", "error_word", "workspace")]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{where}: {moe_status_string(status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library.  Raises if it was never built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m combine_moe_layout_06_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, C, S = ctypes.c_void_p, ctypes.POINTER(MoeConfig), ctypes.c_int
+    L.moe_status_string.argtypes = [S]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_check_config.argtypes = [C]
+    L.moe_expert_partition.argtypes = [ctypes.c_int32, ctypes.c_int32, P]
+    L.moe_layout_workspace_bytes.argtypes = [C, ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_node_staging_rows.argtypes = [C, ctypes.POINTER(ctypes.c_int64)]
+    LP = ctypes.POINTER(MoeLayout)
+    L.moe_layout.argtypes = [C, P, LP, P]
+    L.moe_dispatch.argtypes = [C, LP, P, P, P, P]
+    L.moe_combine.argtypes = [C, LP, P, P, P, P]
+    L.moe_get_error.argtypes = [LP, P]
+    L.moe_dispatch_decoupled.argtypes = [C, LP, P, P, P, P, P]
+    L.moe_combine_decoupled.argtypes = [C, LP, P, P, P, P, P, P]
+    for name in ENTRY_POINTS[1:]:
+        getattr(L, name).restype = S
+    _lib = L
+    return L
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr() or None
+    return int(x)
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream or None
+    if hasattr(stream, "cuda_stream"):
+        return stream.cuda_stream or None
+    return int(stream) or None
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def config(T, H, E, k, R, N=1, flags=0) -> MoeConfig:
+    return MoeConfig(int(T), int(H), int(E), int(k), int(R), int(N), int(flags))
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_check_config(cfg: MoeConfig) -> int:
+    return lib().moe_check_config(ctypes.byref(cfg))
+
+
+def moe_expert_partition(num_experts: int, num_ranks: int) -> list:
+    out = (ctypes.c_int32 * (max(num_ranks, 0) + 1))()
+    _check(lib().moe_expert_partition(num_experts, num_ranks, out), "moe_expert_partition")
+    return list(out)
+
+
+def moe_layout_workspace_bytes(cfg: MoeConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_layout_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n)),
+           "moe_layout_workspace_bytes")
+    return n.value
+
+
+def moe_node_staging_rows(cfg: MoeConfig) -> int:
+    n = ctypes.c_int64(0)
+    _check(lib().moe_node_staging_rows(ctypes.byref(cfg), ctypes.byref(n)), "moe_node_staging_rows")
+    return n.value
+
+
+def layout_struct(expert_counts, expert_offsets, rank_offsets, slot, error_word, workspace,
+                  node_counts=None, node_offsets=None, node_slot=None) -> MoeLayout:
+    return MoeLayout(_ptr(expert_counts), _ptr(expert_offsets), _ptr(rank_offsets), _ptr(slot),
+                     _ptr(node_counts), _ptr(node_offsets), _ptr(node_slot), _ptr(error_word),
+                     _ptr(workspace))
+
+
+def moe_layout(cfg: MoeConfig, topk_idx, layout: MoeLayout, stream=None) -> None:
+    _check(lib().moe_layout(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(layout),
+                            _stream(stream)), "moe_layout")
+
+
+def moe_dispatch(cfg: MoeConfig, layout: MoeLayout, x, recv, node_staging=None,
+                 stream=None) -> None:
+    _check(lib().moe_dispatch(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x), _ptr(recv),
+                              _ptr(node_staging), _stream(stream)), "moe_dispatch")
+
+
+def moe_combine(cfg: MoeConfig, layout: MoeLayout, expert_out, topk_weights, y,
+                stream=None) -> None:
+    _check(lib().moe_combine(ctypes.byref(cfg), ctypes.byref(layout), _ptr(expert_out),
+                             _ptr(topk_weights), _ptr(y), _stream(stream)), "moe_combine")
+
+
+def moe_get_error(layout: MoeLayout, stream=None) -> int:
+    """Status recorded on the device since the last call (waits for stream)."""
+    return lib().moe_get_error(ctypes.byref(layout), _stream(stream))
+
+
+def moe_dispatch_decoupled(cfg: MoeConfig, layout: MoeLayout, x, send, xfer, recv,
+                           stream=None) -> None:
+    _check(lib().moe_dispatch_decoupled(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x),
+                                        _ptr(send), _ptr(xfer), _ptr(recv), _stream(stream)),
+           "moe_dispatch_decoupled")
+
+
+def moe_combine_decoupled(cfg: MoeConfig, layout: MoeLayout, expert_out, topk_weights, send,
+                          xfer, y, stream=None) -> None:
+    _check(lib().moe_combine_decoupled(ctypes.byref(cfg), ctypes.byref(layout), _ptr(expert_out),
+                                       _ptr(topk_weights), _ptr(send), _ptr(xfer), _ptr(y),
+                                       _stream(stream)), "moe_combine_decoupled")

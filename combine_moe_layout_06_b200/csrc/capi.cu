@@ -1,0 +1,251 @@
+// capi.cu -- the C ABI of libmoe_layout.so (declared in include/moe_layout.h):
+// host-side validation, then the kernel launchers.  No entry point
+// allocates device memory.
+#include "moe_layout.h"
+#include "moe_kernels.h"
+
+namespace {
+
+using moe::CopyEngine;
+
+constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK;
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+CopyEngine engine_of(uint32_t flags) {
+    if (flags & MOE_FLAG_COPY_VECTOR) return CopyEngine::kVector;
+    if (flags & MOE_FLAG_COPY_BULK) return CopyEngine::kBulk;
+    return CopyEngine::kAuto;
+}
+
+bool two_level(const moe_config_t* c) { return (c->flags & MOE_FLAG_TWO_LEVEL) != 0; }
+
+moe_status_t check_layout_ptrs(const moe_config_t* c, const moe_layout_t* L) {
+    // Per-token arrays may be NULL only when there are no tokens.
+    const bool tokens = c->num_tokens > 0;
+    if (L == nullptr || L->expert_counts == nullptr || L->expert_offsets == nullptr ||
+        L->rank_offsets == nullptr || (tokens && L->slot == nullptr) || L->error_word == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (two_level(c) && (L->node_counts == nullptr || L->node_offsets == nullptr ||
+                         (tokens && L->node_slot == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+int64_t staging_rows(const moe_config_t* c) {
+    const int32_t m = c->num_nodes < c->top_k ? c->num_nodes : c->top_k;
+    return c->num_tokens * (int64_t)m;
+}
+
+moe::RowMoveParams move_params(const moe_config_t* c, const moe_layout_t* L) {
+    moe::RowMoveParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.N = c->num_nodes;
+    p.ranks_per_node = c->num_ranks / c->num_nodes;
+    p.row_bytes = (size_t)c->hidden * 2;
+    p.slot = L->slot;
+    p.node_slot = L->node_slot;
+    p.node_offsets = L->node_offsets;
+    p.rank_offsets = L->rank_offsets;
+    p.err = L->error_word;
+    p.engine = engine_of(c->flags);
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+        case MOE_ERR_EMPTY_RANK:
+            return "MOE_ERR_EMPTY_RANK: num_experts < num_ranks leaves a rank with no expert";
+        case MOE_ERR_BAD_NODES:
+            return "MOE_ERR_BAD_NODES: num_nodes must divide num_ranks (and be <= MOE_MAX_NODES "
+                   "for node staging)";
+        case MOE_ERR_EXPERT_OOB: return "MOE_ERR_EXPERT_OOB: expert index outside [0, num_experts)";
+        case MOE_ERR_DUP_EXPERT: return "MOE_ERR_DUP_EXPERT: a token names the same expert twice";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait gave up";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+        case MOE_ERR_BAD_LAYOUT: return "MOE_ERR_BAD_LAYOUT: a slot outside the receive buffer";
+    }
+    return "unknown moe_status_t";
+}
+
+moe_status_t moe_check_config(const moe_config_t* c) {
+    if (c == nullptr) return MOE_ERR_INVALID_ARG;
+    if (c->num_tokens < 0 || c->hidden < 1 || c->num_experts < 1 || c->num_ranks < 1 ||
+        c->num_nodes < 1 || c->top_k < 1)
+        return MOE_ERR_INVALID_ARG;
+    if (c->top_k > c->num_experts || c->top_k > MOE_MAX_TOPK) return MOE_ERR_INVALID_ARG;
+    if (c->num_experts > MOE_MAX_EXPERTS) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & ~kKnownFlags) != 0) return MOE_ERR_INVALID_ARG;
+    if ((c->flags & MOE_FLAG_COPY_VECTOR) && (c->flags & MOE_FLAG_COPY_BULK))
+        return MOE_ERR_INVALID_ARG;
+    if (c->num_tokens * (int64_t)c->top_k >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+    if (c->num_experts < c->num_ranks) return MOE_ERR_EMPTY_RANK;
+    if (c->num_nodes > c->num_ranks || c->num_ranks % c->num_nodes != 0) return MOE_ERR_BAD_NODES;
+    if (two_level(c) && c->num_nodes > MOE_MAX_NODES) return MOE_ERR_BAD_NODES;
+    return MOE_OK;
+}
+
+moe_status_t moe_expert_partition(int32_t num_experts, int32_t num_ranks,
+                                  int32_t* rank_first_expert) {
+    if (num_experts < 1 || num_ranks < 1 || rank_first_expert == nullptr) return MOE_ERR_INVALID_ARG;
+    if (num_experts < num_ranks) return MOE_ERR_EMPTY_RANK;
+    const moe::Partition p = moe::Partition::make(num_experts, num_ranks, 1);
+    for (int32_t r = 0; r <= num_ranks; ++r) rank_first_expert[r] = p.first_expert(r);
+    return MOE_OK;
+}
+
+moe_status_t moe_layout_workspace_bytes(const moe_config_t* c, size_t* bytes) {
+    const moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (bytes == nullptr) return MOE_ERR_INVALID_ARG;
+    *bytes = moe::layout_workspace_bytes(c->num_tokens, c->num_experts, c->num_nodes, two_level(c));
+    return MOE_OK;
+}
+
+moe_status_t moe_node_staging_rows(const moe_config_t* c, int64_t* rows) {
+    const moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (rows == nullptr) return MOE_ERR_INVALID_ARG;
+    *rows = staging_rows(c);
+    return MOE_OK;
+}
+
+moe_status_t moe_layout(const moe_config_t* c, const int32_t* topk_idx, const moe_layout_t* L,
+                        void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (L->workspace == nullptr || (c->num_tokens > 0 && topk_idx == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    moe::LayoutParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.E = c->num_experts;
+    p.R = c->num_ranks;
+    p.N = c->num_nodes;
+    p.nodes = two_level(c);
+    p.topk = topk_idx;
+    p.expert_counts = L->expert_counts;
+    p.expert_offsets = L->expert_offsets;
+    p.rank_offsets = L->rank_offsets;
+    p.slot = L->slot;
+    p.node_counts = L->node_counts;
+    p.node_offsets = L->node_offsets;
+    p.node_slot = L->node_slot;
+    p.err = L->error_word;
+    p.workspace = L->workspace;
+    return cuda_status(moe::launch_layout(p, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch(const moe_config_t* c, const moe_layout_t* L, const void* x, void* recv,
+                          void* node_staging, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || recv == nullptr) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe::RowMoveParams p = move_params(c, L);
+    if (!two_level(c)) return cuda_status(moe::launch_dispatch_flat(p, x, recv, s));
+    if (node_staging == nullptr) return MOE_ERR_INVALID_ARG;
+    const int64_t rows = staging_rows(c);
+    cudaError_t e = moe::launch_node_pack(p, x, node_staging, rows, s);
+    if (e == cudaSuccess) e = moe::launch_node_expand(p, node_staging, rows, recv, s);
+    return cuda_status(e);
+}
+
+moe_status_t moe_combine(const moe_config_t* c, const moe_layout_t* L, const void* expert_out,
+                         const float* topk_weights, void* y, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (expert_out == nullptr || topk_weights == nullptr || y == nullptr) return MOE_ERR_INVALID_ARG;
+    moe::CombineParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.row_bytes = (size_t)c->hidden * 2;
+    p.slot = L->slot;
+    p.w = topk_weights;
+    p.err = L->error_word;
+    p.engine = engine_of(c->flags);
+    return cuda_status(moe::launch_combine(p, expert_out, y, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_error(const moe_layout_t* L, void* stream) {
+    if (L == nullptr || L->error_word == nullptr) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t bits = 0;
+    cudaError_t e = cudaMemcpyAsync(&bits, L->error_word, sizeof bits, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L->error_word, 0, sizeof bits, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (bits & moe::kErrExpertOob) return MOE_ERR_EXPERT_OOB;
+    if (bits & moe::kErrDupExpert) return MOE_ERR_DUP_EXPERT;
+    if (bits & moe::kErrBadLayout) return MOE_ERR_BAD_LAYOUT;
+    if (bits & moe::kErrTimeout) return MOE_ERR_TIMEOUT;
+    return MOE_OK;
+}
+
+moe_status_t moe_dispatch_decoupled(const moe_config_t* c, const moe_layout_t* L, const void* x,
+                                    void* send, void* xfer, void* recv, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (!two_level(c) || c->num_nodes != c->num_ranks) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || send == nullptr || xfer == nullptr || recv == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe::RowMoveParams p = move_params(c, L);
+    const int64_t rows = staging_rows(c);
+    cudaError_t e = moe::launch_node_pack(p, x, send, rows, s);
+    if (e == cudaSuccess)
+        e = moe::launch_copy_rows(send, xfer, L->node_offsets + c->num_nodes, rows, p.row_bytes, s);
+    if (e == cudaSuccess) e = moe::launch_node_expand(p, xfer, rows, recv, s);
+    return cuda_status(e);
+}
+
+moe_status_t moe_combine_decoupled(const moe_config_t* c, const moe_layout_t* L,
+                                   const void* expert_out, const float* topk_weights, void* send,
+                                   void* xfer, void* y, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (expert_out == nullptr || topk_weights == nullptr || send == nullptr || xfer == nullptr ||
+        y == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe::RowMoveParams p = move_params(c, L);
+    const int64_t rows = c->num_tokens * (int64_t)c->top_k;
+    cudaError_t e = moe::launch_gather_rows(p, expert_out, send, s);
+    if (e == cudaSuccess) e = moe::launch_copy_rows(send, xfer, nullptr, rows, p.row_bytes, s);
+    if (e == cudaSuccess) {
+        moe::CombineParams cp;
+        cp.T = c->num_tokens;
+        cp.k = c->top_k;
+        cp.row_bytes = p.row_bytes;
+        cp.slot = nullptr;
+        cp.w = topk_weights;
+        cp.err = L->error_word;
+        cp.engine = engine_of(c->flags);
+        e = moe::launch_combine(cp, xfer, y, s);
+    }
+    return cuda_status(e);
+}
+
+}  // extern "C"

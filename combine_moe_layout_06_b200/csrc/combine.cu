@@ -1,0 +1,147 @@
+// combine.cu -- fused combine.
+//
+// INC-MoE abstract: combine returns the expert outputs of each token to the
+// token's owner, where they are reduced by gate weight.  Here the k expert
+// rows of token t are gathered straight from the expert-major buffer (the
+// scatter-recv layout of the FUSCO article, section "FUSCO 的核心创新") and
+// summed in fp32 registers before one bf16 store; no unpack pass runs.
+//
+// Arithmetic, fixed so that results are reproducible bit for bit: acc starts
+// at +0.0f and, for j = 0 .. k-1 in top-k column order, acc = fma(w[t][j],
+// float(eo[slot[t][j]][h]), acc) with a single rounding per step; the store
+// rounds to nearest even.
+//
+// One warp per token.  Lanes hold the k slots and weights; each pass covers
+// 32*VPL vectors of the row, and rows are fetched four at a time so that
+// 4*VPL streaming loads per lane are in flight before their FMAs.
+#include "moe_kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+constexpr int kThreads = kWarpsPerCta * 32;
+constexpr int kRowsInFlight = 4;
+
+struct CombArgs {
+    const void* eo;
+    const float* w;
+    const int* slot;   // nullptr: row of (t, j) is t*k + j
+    void* y;
+    int64_t T;
+    int k;
+    int64_t rv;        // vectors per row
+    int64_t eo_rows;
+    int* err;
+};
+
+template <typename V, int VPL>
+__global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
+    constexpr int EPV = VecInfo<V>::kElems;
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    const V* eo = static_cast<const V*>(a.eo);
+    V* y = static_cast<V*>(a.y);
+    int errbits = 0;
+    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < a.T; t += nwarps) {
+        int s = -1;
+        float wl = 0.f;
+        if (lane < a.k) {
+            s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
+            wl = __ldg(a.w + t * a.k + lane);
+            if (s < 0 || s >= a.eo_rows) {
+                if (s != -1) errbits |= kErrBadLayout;
+                s = -1;
+            }
+        }
+        for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
+            float acc[VPL][EPV];
+#pragma unroll
+            for (int i = 0; i < VPL; ++i)
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) acc[i][e] = 0.f;
+            for (int j0 = 0; j0 < a.k; j0 += kRowsInFlight) {
+                V v[kRowsInFlight][VPL];
+                float wq[kRowsInFlight];
+                bool ok[kRowsInFlight];
+#pragma unroll
+                for (int q = 0; q < kRowsInFlight; ++q) {
+                    const int j = j0 + q;
+                    const int sj = __shfl_sync(kFullMask, s, j & 31);
+                    wq[q] = __shfl_sync(kFullMask, wl, j & 31);
+                    ok[q] = j < a.k && sj >= 0;
+                    if (ok[q]) {
+                        const V* row = eo + (int64_t)sj * a.rv;
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i) {
+                            const int64_t idx = base + i * 32 + lane;
+                            if (idx < a.rv) v[q][i] = ld_stream(row + idx);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kRowsInFlight; ++q) {
+                    if (!ok[q]) continue;
+#pragma unroll
+                    for (int i = 0; i < VPL; ++i) {
+                        const int64_t idx = base + i * 32 + lane;
+                        if (idx < a.rv) {
+                            float f[EPV];
+                            unpack_bf16<V>(v[q][i], f);
+#pragma unroll
+                            for (int e = 0; e < EPV; ++e) acc[i][e] = __fmaf_rn(wq[q], f[e], acc[i][e]);
+                        }
+                    }
+                }
+            }
+            V* yrow = y + t * a.rv;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int64_t idx = base + i * 32 + lane;
+                if (idx < a.rv) yrow[idx] = pack_bf16<V>(acc[i]);
+            }
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+inline int vec_bytes(size_t row_bytes, const void* a, const void* b) {
+    const uintptr_t bits = row_bytes | reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b);
+    if (bits % 16 == 0) return 16;
+    if (bits % 4 == 0) return 4;
+    return 2;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void* y,
+                           cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    CombArgs a;
+    a.eo = expert_out;
+    a.w = p.w;
+    a.slot = p.slot;
+    a.y = y;
+    a.T = p.T;
+    a.k = p.k;
+    a.eo_rows = p.T * p.k;
+    a.err = p.err;
+    int64_t g = (p.T + kWarpsPerCta - 1) / kWarpsPerCta;
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    const int grid = (int)(g > cap ? cap : g);
+    switch (vec_bytes(p.row_bytes, expert_out, y)) {
+        case 16:
+            a.rv = (int64_t)(p.row_bytes / 16);
+            return launch_pdl(combine_kernel<uint4, 2>, dim3(grid), dim3(kThreads), 0, stream, a);
+        case 4:
+            a.rv = (int64_t)(p.row_bytes / 4);
+            return launch_pdl(combine_kernel<uint32_t, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+        default:
+            a.rv = (int64_t)(p.row_bytes / 2);
+            return launch_pdl(combine_kernel<uint16_t, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,317 @@
+// dispatch.cu -- fused dispatch and the row-movement kernels around it.
+//
+// Fused dispatch is the gather-send / scatter-recv of the FUSCO article
+// (aigc.bar), section "FUSCO 的核心创新": each token row is read once
+// straight from x and written straight into every destination row the
+// layout names, so no pack or unpack pass runs.  Two-level dispatch follows
+// section "负载均衡与跨节点去重": a row goes once to each node it touches
+// (a node staging region, node-major then token order) and is then expanded
+// inside the node to that node's expert rows.  The same two kernels with
+// one "node" per rank, plus a contiguous copy, form the decoupled
+// pack -> copy -> unpack path that section "传统 MoE 通信的痛点" describes.
+//
+// Register engine: one warp moves one source row.  Lanes hold the
+// destination rows (k <= 32 slots, or N <= 32 nodes); the row is loaded in
+// passes of 32*VPL vectors with streaming loads and stored to every
+// destination with evict-first stores.  The bulk engine lives in bulk.cu.
+#include <initializer_list>
+
+#include "moe_kernels.h"
+
+namespace moe {
+
+int device_sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+constexpr int kThreads = kWarpsPerCta * 32;
+
+enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2 };
+
+struct FanArgs {
+    const void* src;
+    void* dst;
+    const int* slot;
+    const int* node_slot;
+    const int* node_offsets;
+    const int* rank_offsets;
+    int64_t T;
+    int k, N, ranks_per_node;
+    int64_t rv;        // vectors per row
+    int64_t src_rows;  // rows in src (bounds check)
+    int64_t dst_rows;  // rows in dst (bounds check)
+    int* err;
+};
+
+// One warp per work item.  Flat and node-pack items are tokens; node-expand
+// items are (node, token) pairs, node-major, so each node's forwarder work
+// is one contiguous run of items.
+template <int MODE, typename V, int VPL>
+__global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t items = MODE == kNodeExpand ? a.T * a.N : a.T;
+    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    int errbits = 0;
+    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
+         item += nwarps) {
+        int64_t src_row;
+        int64_t dst = -1;
+        if (MODE == kFlat) {
+            src_row = item;
+            if (lane < a.k) {
+                const int s = __ldg(a.slot + item * a.k + lane);
+                if (s >= 0 && s < a.dst_rows) dst = s;
+                else if (s != -1) errbits |= kErrBadLayout;
+            }
+        } else if (MODE == kNodePack) {
+            src_row = item;
+            if (lane < a.N) {
+                const int ns = __ldg(a.node_slot + item * a.N + lane);
+                if (ns >= 0) {
+                    const int64_t d = (int64_t)__ldg(a.node_offsets + lane) + ns;
+                    if (d >= 0 && d < a.dst_rows) dst = d;
+                    else errbits |= kErrBadLayout;
+                }
+            }
+        } else {
+            const int n = (int)(item / a.T);
+            const int64_t t = item - (int64_t)n * a.T;
+            const int ns = __ldg(a.node_slot + t * a.N + n);  // same for all lanes
+            if (ns < 0) continue;
+            src_row = (int64_t)__ldg(a.node_offsets + n) + ns;
+            if (src_row < 0 || src_row >= a.src_rows) {
+                errbits |= kErrBadLayout;
+                continue;
+            }
+            const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
+            const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
+            if (lane < a.k) {
+                const int s = __ldg(a.slot + t * a.k + lane);
+                if (s >= lo && s < hi && s < a.dst_rows) dst = s;
+            }
+        }
+        const unsigned dmask = __ballot_sync(kFullMask, dst >= 0);
+        const V* srow = static_cast<const V*>(a.src) + src_row * a.rv;
+        V* dbase = static_cast<V*>(a.dst);
+        for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
+            V v[VPL];
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const int64_t idx = base + i * 32 + lane;
+                if (idx < a.rv) v[i] = ld_stream(srow + idx);
+            }
+            unsigned m = dmask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int64_t d = __shfl_sync(kFullMask, dst, j);
+                V* drow = dbase + d * a.rv;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int64_t idx = base + i * 32 + lane;
+                    if (idx < a.rv) st_stream(drow + idx, v[i]);
+                }
+            }
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+// dst[t*k + j] = src[slot[t][j]] (decoupled combine's pack).  One warp per
+// token, one source row at a time.
+template <typename V, int VPL>
+__global__ void __launch_bounds__(kThreads) gather_kernel(FanArgs a) {
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    int errbits = 0;
+    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < a.T; t += nwarps) {
+        int s = -1;
+        if (lane < a.k) {
+            s = __ldg(a.slot + t * a.k + lane);
+            if (s < 0 || s >= a.src_rows) {
+                if (s != -1) errbits |= kErrBadLayout;
+                s = -1;
+            }
+        }
+        for (int j = 0; j < a.k; ++j) {
+            const int sj = __shfl_sync(kFullMask, s, j);
+            if (sj < 0) continue;
+            const V* srow = static_cast<const V*>(a.src) + (int64_t)sj * a.rv;
+            V* drow = static_cast<V*>(a.dst) + (t * a.k + j) * a.rv;
+            for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
+                V v[VPL];
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int64_t idx = base + i * 32 + lane;
+                    if (idx < a.rv) v[i] = ld_stream(srow + idx);
+                }
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int64_t idx = base + i * 32 + lane;
+                    if (idx < a.rv) st_stream(drow + idx, v[i]);
+                }
+            }
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+// Contiguous copy of `rows` rows; the row count may live in device memory
+// (the decoupled path's transfer size is known only on the device).
+template <typename V>
+__global__ void __launch_bounds__(kThreads) copy_kernel(const V* __restrict__ src, V* __restrict__ dst,
+                                                        const int* rows_dev, int64_t max_rows,
+                                                        int64_t rv) {
+    pdl_wait();
+    pdl_trigger();
+    int64_t rows = max_rows;
+    if (rows_dev != nullptr) {
+        const int64_t r = *rows_dev;
+        rows = r < 0 ? 0 : (r < max_rows ? r : max_rows);
+    }
+    const int64_t n = rows * rv;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n; i += 4 * stride) {
+        V v0 = ld_stream(src + i), v1 = ld_stream(src + i + stride);
+        V v2 = ld_stream(src + i + 2 * stride), v3 = ld_stream(src + i + 3 * stride);
+        st_stream(dst + i, v0);
+        st_stream(dst + i + stride, v1);
+        st_stream(dst + i + 2 * stride, v2);
+        st_stream(dst + i + 3 * stride, v3);
+    }
+    for (; i < n; i += stride) st_stream(dst + i, ld_stream(src + i));
+}
+
+// Widest vector that divides the row and every base address.
+inline int vec_bytes(size_t row_bytes, std::initializer_list<const void*> ptrs) {
+    uintptr_t bits = row_bytes;
+    for (const void* p : ptrs) bits |= reinterpret_cast<uintptr_t>(p);
+    if (bits % 16 == 0) return 16;
+    if (bits % 4 == 0) return 4;
+    return 2;
+}
+
+inline int grid_for(int64_t warp_items) {
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    int64_t g = (warp_items + kWarpsPerCta - 1) / kWarpsPerCta;
+    if (g > cap) g = cap;
+    return (int)(g < 1 ? 1 : g);
+}
+
+template <int MODE, typename V>
+cudaError_t launch_fan_v(FanArgs a, int64_t items, cudaStream_t stream) {
+    a.rv /= sizeof(V);
+    const int grid = grid_for(items);
+    if (sizeof(V) == 16 && a.rv % (32 * 7) == 0 && a.rv % (32 * 8) != 0)
+        return launch_pdl(fanout_kernel<MODE, V, 7>, dim3(grid), dim3(kThreads), 0, stream, a);
+    if (a.rv >= 32 * 8)
+        return launch_pdl(fanout_kernel<MODE, V, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
+    return launch_pdl(fanout_kernel<MODE, V, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
+template <int MODE>
+cudaError_t launch_fan(FanArgs a, int64_t items, cudaStream_t stream) {
+    if (items <= 0) return cudaSuccess;
+    switch (vec_bytes((size_t)a.rv, {a.src, a.dst})) {
+        case 16: return launch_fan_v<MODE, uint4>(a, items, stream);
+        case 4: return launch_fan_v<MODE, uint32_t>(a, items, stream);
+        default: return launch_fan_v<MODE, uint16_t>(a, items, stream);
+    }
+}
+
+FanArgs fan_args(const RowMoveParams& p, const void* src, void* dst, int64_t src_rows,
+                 int64_t dst_rows) {
+    FanArgs a;
+    a.src = src;
+    a.dst = dst;
+    a.slot = p.slot;
+    a.node_slot = p.node_slot;
+    a.node_offsets = p.node_offsets;
+    a.rank_offsets = p.rank_offsets;
+    a.T = p.T;
+    a.k = p.k;
+    a.N = p.N;
+    a.ranks_per_node = p.ranks_per_node;
+    a.rv = (int64_t)p.row_bytes;  // bytes until the vector width is chosen
+    a.src_rows = src_rows;
+    a.dst_rows = dst_rows;
+    a.err = p.err;
+    return a;
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch_flat(const RowMoveParams& p, const void* x, void* recv,
+                                        cudaStream_t stream) {
+    FanArgs a = fan_args(p, x, recv, p.T, p.T * p.k);
+    return launch_fan<kFlat>(a, p.T, stream);
+}
+
+cudaError_t launch_node_pack(const RowMoveParams& p, const void* x, void* staging,
+                             int64_t staging_rows, cudaStream_t stream) {
+    FanArgs a = fan_args(p, x, staging, p.T, staging_rows);
+    return launch_fan<kNodePack>(a, p.T, stream);
+}
+
+cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging, int64_t staging_rows,
+                               void* recv, cudaStream_t stream) {
+    FanArgs a = fan_args(p, staging, recv, staging_rows, p.T * p.k);
+    return launch_fan<kNodeExpand>(a, p.T * p.N, stream);
+}
+
+cudaError_t launch_gather_rows(const RowMoveParams& p, const void* src, void* dst,
+                               cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    FanArgs a = fan_args(p, src, dst, p.T * p.k, p.T * p.k);
+    const int grid = grid_for(p.T);
+    switch (vec_bytes(p.row_bytes, {src, dst})) {
+        case 16:
+            a.rv /= 16;
+            return launch_pdl(gather_kernel<uint4, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+        case 4:
+            a.rv /= 4;
+            return launch_pdl(gather_kernel<uint32_t, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
+        default:
+            a.rv /= 2;
+            return launch_pdl(gather_kernel<uint16_t, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
+    }
+}
+
+cudaError_t launch_copy_rows(const void* src, void* dst, const int* rows_dev, int64_t max_rows,
+                             size_t row_bytes, cudaStream_t stream) {
+    if (max_rows <= 0) return cudaSuccess;
+    const int grid = device_sm_count() * 8;
+    switch (vec_bytes(row_bytes, {src, dst})) {
+        case 16:
+            return launch_pdl(copy_kernel<uint4>, dim3(grid), dim3(kThreads), 0, stream,
+                              static_cast<const uint4*>(src), static_cast<uint4*>(dst), rows_dev,
+                              max_rows, (int64_t)(row_bytes / 16));
+        case 4:
+            return launch_pdl(copy_kernel<uint32_t>, dim3(grid), dim3(kThreads), 0, stream,
+                              static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst),
+                              rows_dev, max_rows, (int64_t)(row_bytes / 4));
+        default:
+            return launch_pdl(copy_kernel<uint16_t>, dim3(grid), dim3(kThreads), 0, stream,
+                              static_cast<const uint16_t*>(src), static_cast<uint16_t*>(dst),
+                              rows_dev, max_rows, (int64_t)(row_bytes / 2));
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,205 @@
+// moe_common.cuh -- shared device helpers of the B200 MoE dispatch/combine
+// kernels: error bits, the ceil/floor expert partition, cache-hinted vector
+// loads/stores, bf16 packing and the launch wrapper.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device error-word bits (moe_layout_t.error_word).
+constexpr int kErrExpertOob = 1 << 0;
+constexpr int kErrDupExpert = 1 << 1;
+constexpr int kErrBadLayout = 1 << 2;
+constexpr int kErrTimeout = 1 << 3;
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// Ceil/floor contiguous expert partition (TensorRT-LLM PR #13888, PR
+// description and the divisible-fast-path commit): base = E / R and rem =
+// E % R are computed once; ranks below rem hold base + 1 experts.  When rem
+// is zero the rank is a single division.
+struct Partition {
+    int E, R, base, rem, ranks_per_node;
+
+    __host__ __device__ static Partition make(int E, int R, int N) {
+        Partition p;
+        p.E = E;
+        p.R = R;
+        p.base = E / R;
+        p.rem = E % R;
+        p.ranks_per_node = R / N;
+        return p;
+    }
+    __host__ __device__ __forceinline__ int rank_of(int e) const {
+        if (rem == 0) return e / base;
+        const int big = rem * (base + 1);
+        return e < big ? e / (base + 1) : rem + (e - big) / base;
+    }
+    __host__ __device__ __forceinline__ int first_expert(int r) const {
+        return r * base + (r < rem ? r : rem);
+    }
+    __host__ __device__ __forceinline__ int node_of(int e) const {
+        return rank_of(e) / ranks_per_node;
+    }
+};
+
+// ---- programmatic dependent launch -------------------------------------
+// Every kernel waits for its predecessor grid before touching memory and
+// lets its dependent grid launch early, so launch latency overlaps the
+// previous kernel's tail.
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- cache-hinted global access -----------------------------------------
+// Streaming loads of rows read exactly once (no L1 allocation) and
+// evict-first stores of rows written once.
+template <typename V>
+__device__ __forceinline__ V ld_stream(const V* p);
+template <>
+__device__ __forceinline__ uint4 ld_stream<uint4>(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+template <>
+__device__ __forceinline__ uint32_t ld_stream<uint32_t>(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+template <>
+__device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+template <typename V>
+__device__ __forceinline__ void st_stream(V* p, const V& v);
+template <>
+__device__ __forceinline__ void st_stream<uint4>(uint4* p, const uint4& v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+template <>
+__device__ __forceinline__ void st_stream<uint32_t>(uint32_t* p, const uint32_t& v) {
+    asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+template <>
+__device__ __forceinline__ void st_stream<uint16_t>(uint16_t* p, const uint16_t& v) {
+    asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
+}
+
+// ---- bf16 <-> fp32 over vector words -------------------------------------
+// A bf16 value is the upper half of a binary32, so widening is a shift.
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two fp32 -> two bf16 (round to nearest even, one cvt instruction).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+// Number of bf16 values in one vector word.
+template <typename V>
+struct VecInfo;
+template <>
+struct VecInfo<uint4> {
+    static constexpr int kElems = 8;
+};
+template <>
+struct VecInfo<uint32_t> {
+    static constexpr int kElems = 2;
+};
+template <>
+struct VecInfo<uint16_t> {
+    static constexpr int kElems = 1;
+};
+
+template <typename V>
+__device__ __forceinline__ void unpack_bf16(const V& v, float (&f)[VecInfo<V>::kElems]);
+template <>
+__device__ __forceinline__ void unpack_bf16<uint4>(const uint4& v, float (&f)[8]) {
+    f[0] = bf16lo_to_f32(v.x);
+    f[1] = bf16hi_to_f32(v.x);
+    f[2] = bf16lo_to_f32(v.y);
+    f[3] = bf16hi_to_f32(v.y);
+    f[4] = bf16lo_to_f32(v.z);
+    f[5] = bf16hi_to_f32(v.z);
+    f[6] = bf16lo_to_f32(v.w);
+    f[7] = bf16hi_to_f32(v.w);
+}
+template <>
+__device__ __forceinline__ void unpack_bf16<uint32_t>(const uint32_t& v, float (&f)[2]) {
+    f[0] = bf16lo_to_f32(v);
+    f[1] = bf16hi_to_f32(v);
+}
+template <>
+__device__ __forceinline__ void unpack_bf16<uint16_t>(const uint16_t& v, float (&f)[1]) {
+    f[0] = __uint_as_float(((uint32_t)v) << 16);
+}
+
+template <typename V>
+__device__ __forceinline__ V pack_bf16(const float (&f)[VecInfo<V>::kElems]);
+template <>
+__device__ __forceinline__ uint4 pack_bf16<uint4>(const float (&f)[8]) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+template <>
+__device__ __forceinline__ uint32_t pack_bf16<uint32_t>(const float (&f)[2]) {
+    return pack_bf16x2(f[0], f[1]);
+}
+template <>
+__device__ __forceinline__ uint16_t pack_bf16<uint16_t>(const float (&f)[1]) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f[0]);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Record error bits once per warp.
+__device__ __forceinline__ void warp_report(int* err_word, int bits) {
+    const int any = __reduce_or_sync(kFullMask, bits);
+    if (any && (threadIdx.x & 31) == 0 && err_word != nullptr) atomicOr(err_word, any);
+}
+
+// ---- launching ------------------------------------------------------------
+// Launch with programmatic stream serialization allowed, so the kernel may
+// start while its predecessor drains; each kernel calls pdl_wait() before
+// it reads anything a predecessor wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,80 @@
+// moe_kernels.h -- host launchers of the MoE dispatch/combine kernels
+// (internal to libmoe_layout.so; the public C ABI is include/moe_layout.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe_common.cuh"
+
+namespace moe {
+
+// Which row-copy engine moves bf16 rows.
+enum class CopyEngine { kAuto = 0, kVector = 1, kBulk = 2 };
+
+// ---- layout ----------------------------------------------------------------
+struct LayoutParams {
+    int64_t T;
+    int k, E, R, N;
+    bool nodes;             // also build node staging maps
+    const int* topk;        // [T*k]
+    int* expert_counts;     // [E]
+    int* expert_offsets;    // [E+1]
+    int* rank_offsets;      // [R+1]
+    int* slot;              // [T*k]
+    int* node_counts;       // [N]    (nodes)
+    int* node_offsets;      // [N+1]  (nodes)
+    int* node_slot;         // [T*N]  (nodes)
+    int* err;               // [1]
+    void* workspace;        // layout_workspace_bytes()
+};
+size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes);
+cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
+
+// ---- row movement ------------------------------------------------------------
+// Geometry shared by the dispatch-side kernels.  Row sizes are in bytes;
+// every row of x / recv / staging is row_bytes long and rows are packed.
+struct RowMoveParams {
+    int64_t T;
+    int k, N, ranks_per_node;
+    size_t row_bytes;
+    const int* slot;          // [T*k]
+    const int* node_slot;     // [T*N]
+    const int* node_offsets;  // [N+1]
+    const int* rank_offsets;  // [R+1]
+    int* err;
+    CopyEngine engine;
+};
+
+// recv[slot[t][j]] = x[t]
+cudaError_t launch_dispatch_flat(const RowMoveParams& p, const void* x, void* recv,
+                                 cudaStream_t stream);
+// staging[node_offsets[n] + node_slot[t][n]] = x[t] for every node touched
+cudaError_t launch_node_pack(const RowMoveParams& p, const void* x, void* staging,
+                             int64_t staging_rows, cudaStream_t stream);
+// recv[slot[t][j]] = staging[node row of (t, n)] for the j whose row lies on n
+cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging,
+                               int64_t staging_rows, void* recv, cudaStream_t stream);
+// dst[0 .. rows) = src[0 .. rows); rows = *rows_dev (clamped to max_rows)
+// when rows_dev is given, else max_rows.
+cudaError_t launch_copy_rows(const void* src, void* dst, const int* rows_dev, int64_t max_rows,
+                             size_t row_bytes, cudaStream_t stream);
+// dst[t*k + j] = src[slot[t][j]]
+cudaError_t launch_gather_rows(const RowMoveParams& p, const void* src, void* dst,
+                               cudaStream_t stream);
+
+// ---- combine -----------------------------------------------------------------
+struct CombineParams {
+    int64_t T;
+    int k;
+    size_t row_bytes;
+    const int* slot;   // [T*k]; nullptr = rows t*k + j (contiguous source order)
+    const float* w;    // [T*k]
+    int* err;
+    CopyEngine engine;
+};
+cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void* y,
+                           cudaStream_t stream);
+
+}  // namespace moe

@@ -178,3 +178,16 @@ def random_bf16(shape, seed: int, scale: float = 1.0) -> np.ndarray:
     """N(0, scale^2) values as bf16 bit patterns (e.g. stand-in expert outputs)."""
     rng = _rng(seed)
     return x_bf16_bits(scale * rng.standard_normal(shape, dtype=np.float32))
+
+
+def random_bf16_bits(shape, seed: int) -> np.ndarray:
+    """Fast stand-in expert outputs: bf16 bit patterns with a random sign, a
+    biased exponent in [120, 130] (magnitudes 2^-7 .. 2^4) and a uniform
+    7-bit mantissa.  16-bit integer draws only, so multi-GB buffers are
+    cheap."""
+    rng = _rng(seed)
+    r = rng.integers(0, 1 << 16, size=int(np.prod(shape)), dtype=np.uint16)
+    out = (r & np.uint16(1)) << np.uint16(15)
+    out |= (np.uint16(120) + (r >> np.uint16(1)) % np.uint16(11)) << np.uint16(7)
+    out |= (r >> np.uint16(8)) & np.uint16(0x7F)
+    return out.reshape(shape)

@@ -1,0 +1,230 @@
+/*
+ * moe_layout.h -- C ABI of the B200 MoE dispatch / combine library
+ * (libmoe_layout.so).
+ *
+ * The library moves token rows between a batch of activations and an
+ * expert-major receive buffer, the data shuffle of expert-parallel MoE, with
+ * the layout transformation fused into the data movement.  Sources:
+ *
+ *  - FUSCO article (aigc.bar, "超DeepEP两倍！无问芯穹FUSCO如何以「空中变阵」
+ *    突破MoE通信瓶颈"), section "传统 MoE 通信的痛点": decoupled designs pack
+ *    scattered tokens into contiguous blocks before sending and unpack them
+ *    after receiving; section "FUSCO 的核心创新": gather-send reads rows
+ *    straight from their scattered locations by segment descriptor and
+ *    scatter-recv writes them straight into the final layout; section
+ *    "负载均衡与跨节点去重": one copy per destination node, fanned out
+ *    inside the node by a forwarding GPU.
+ *  - INC-MoE abstract: dispatch moves tokens to the holders of their
+ *    selected experts, combine returns expert outputs to the token's owner.
+ *  - TensorRT-LLM PR #13888 ("support non-divisible EP in MoE alltoall and
+ *    slurm benchmark"): ceil/floor contiguous expert partitioning across
+ *    ranks, a divisible fast path, and a clear error when num_experts <
+ *    ep_size.
+ *
+ * Everything runs on one GPU.  Expert-parallel ranks and nodes are virtual:
+ * rank r owns a contiguous range of receive rows, node n a contiguous range
+ * of ranks.
+ *
+ * Conventions for every entry point
+ *  - Pointers named "device" point to CUDA device memory of the current
+ *    device; the caller allocates and owns all of it.  Nothing here
+ *    allocates device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Device work is enqueued on it asynchronously.
+ *  - Argument and shape errors are detected on the host and returned before
+ *    anything is enqueued.  Errors that depend on device data (an expert
+ *    index out of range, a token naming one expert twice, a slot outside the
+ *    receive buffer) are recorded in the layout's device error word and read
+ *    back by moe_get_error(); kernels never trap.  When one is recorded the
+ *    outputs of that call are unspecified, but every access stays inside the
+ *    buffers described here.
+ *  - A failed CUDA launch returns MOE_ERR_CUDA.
+ *  - bf16 tensors are row-major [rows][hidden] 16-bit brain-float values.
+ *    Rows whose byte size and base address are multiples of 16 take the
+ *    vectorised kernels; other shapes are supported by narrower kernels.
+ *  - The library keeps no state between calls other than per-device
+ *    launch attributes; calls on different streams may run concurrently if
+ *    their buffers do not overlap.
+ */
+#ifndef MOE_LAYOUT_H
+#define MOE_LAYOUT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Size limits. */
+#define MOE_MAX_EXPERTS 1024 /* experts per layer */
+#define MOE_MAX_TOPK 32      /* experts per token */
+#define MOE_MAX_NODES 32     /* virtual nodes when node staging is used */
+
+/* moe_config_t.flags */
+#define MOE_FLAG_TWO_LEVEL 0x1u  /* layout also builds node staging maps;
+                                    dispatch goes through node staging */
+#define MOE_FLAG_COPY_VECTOR 0x2u /* force the register (16-byte vector)
+                                     copy kernels */
+#define MOE_FLAG_COPY_BULK 0x4u   /* force the bulk-copy (TMA) kernels */
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, bad flag */
+    MOE_ERR_EMPTY_RANK = 2,  /* num_experts < num_ranks: some rank would
+                                hold no expert (PR #13888 review thread) */
+    MOE_ERR_BAD_NODES = 3,   /* num_nodes does not divide num_ranks, or too
+                                many nodes for node staging */
+    MOE_ERR_EXPERT_OOB = 4,  /* device data: expert index outside [0, E) */
+    MOE_ERR_DUP_EXPERT = 5,  /* device data: a token names an expert twice */
+    MOE_ERR_TIMEOUT = 6,     /* device: a bounded wait gave up */
+    MOE_ERR_CUDA = 7,        /* a CUDA call failed */
+    MOE_ERR_BAD_LAYOUT = 8   /* device data: a slot outside the receive
+                                buffer was met by dispatch or combine */
+} moe_status_t;
+
+/* Shape of one dispatch/combine problem.
+ *   num_tokens  T >= 0 tokens in the batch (T * top_k < 2^31)
+ *   hidden      H >= 1 bf16 values per token row
+ *   num_experts E, 1 <= E <= MOE_MAX_EXPERTS
+ *   top_k       k experts per token, 1 <= k <= min(E, MOE_MAX_TOPK)
+ *   num_ranks   R virtual expert-parallel ranks, 1 <= R <= E
+ *   num_nodes   N virtual nodes, N divides R (R/N ranks per node)
+ *   flags       MOE_FLAG_* bits */
+typedef struct moe_config {
+    int64_t num_tokens;
+    int32_t hidden;
+    int32_t num_experts;
+    int32_t top_k;
+    int32_t num_ranks;
+    int32_t num_nodes;
+    uint32_t flags;
+} moe_config_t;
+
+/* Layout metadata ("segment descriptors"), all device int32 arrays owned by
+ * the caller.  The receive buffer has exactly T*k rows, expert-major: the
+ * rows of expert e are [expert_offsets[e], expert_offsets[e+1]) in
+ * ascending token order; rank r owns rows [rank_offsets[r],
+ * rank_offsets[r+1]).
+ *   expert_counts  [E]     rows per expert
+ *   expert_offsets [E+1]   exclusive prefix of expert_counts
+ *   rank_offsets   [R+1]   first row of each rank (last = T*k)
+ *   slot           [T*k]   receive row of (token t, column j), row-major
+ *   node_counts    [N]     tokens touching node n          (TWO_LEVEL)
+ *   node_offsets   [N+1]   exclusive prefix of node_counts (TWO_LEVEL)
+ *   node_slot      [T*N]   rank of token t among the tokens touching node n,
+ *                          or -1 when t touches no expert of n (TWO_LEVEL)
+ *   error_word     [1]     device error bits; zero it once before first use,
+ *                          moe_get_error() reads and clears it
+ *   workspace      moe_layout_workspace_bytes() bytes, 16-byte aligned,
+ *                          scratch for moe_layout only
+ * Node arrays may be NULL when MOE_FLAG_TWO_LEVEL is not set. */
+typedef struct moe_layout {
+    int32_t *expert_counts;
+    int32_t *expert_offsets;
+    int32_t *rank_offsets;
+    int32_t *slot;
+    int32_t *node_counts;
+    int32_t *node_offsets;
+    int32_t *node_slot;
+    int32_t *error_word;
+    void *workspace;
+} moe_layout_t;
+
+/* Text of a status code (static storage, never NULL). */
+const char *moe_status_string(moe_status_t status);
+
+/* Host-side check of a configuration (the same check every entry point
+ * runs first).  Order of checks: basic ranges (MOE_ERR_INVALID_ARG), then
+ * E < R (MOE_ERR_EMPTY_RANK), then the node grouping (MOE_ERR_BAD_NODES). */
+moe_status_t moe_check_config(const moe_config_t *cfg);
+
+/* Ceil/floor contiguous expert partition (PR #13888, PR description and
+ * the divisible-fast-path commit): base = E / R, rem = E % R; ranks 0 ..
+ * rem-1 hold base+1 consecutive experts, the others base.  Writes
+ * rank_first_expert[0..R] (host array, R+1 entries, last = E).  Host only.
+ * Errors: MOE_ERR_INVALID_ARG for E < 1, R < 1 or a NULL array;
+ * MOE_ERR_EMPTY_RANK for E < R. */
+moe_status_t moe_expert_partition(int32_t num_experts, int32_t num_ranks,
+                                  int32_t *rank_first_expert);
+
+/* Bytes of moe_layout_t.workspace needed by moe_layout() for cfg. */
+moe_status_t moe_layout_workspace_bytes(const moe_config_t *cfg, size_t *bytes);
+
+/* Rows a node staging buffer must hold for cfg: T * min(N, k). */
+moe_status_t moe_node_staging_rows(const moe_config_t *cfg, int64_t *rows);
+
+/* Layout: per-expert histogram, exclusive scan in expert-major/chunk-minor
+ * order, and stable slot assignment (FUSCO article, "FUSCO 的核心创新":
+ * the segment descriptors that drive gather-send / scatter-recv).
+ *   topk_idx  device int32 [T*k], row-major [T][k], the router's choices
+ *   layout    device arrays as described above (TWO_LEVEL: node arrays too)
+ * Data errors go to layout->error_word. */
+moe_status_t moe_layout(const moe_config_t *cfg, const int32_t *topk_idx,
+                        const moe_layout_t *layout, void *stream);
+
+/* Fused dispatch (gather-send / scatter-recv): recv[slot[t][j]] = x[t] for
+ * every (t, j); each x row is read once and written straight to all its
+ * destination rows, with no pack or unpack pass.
+ *   x             device bf16 [T][H]
+ *   recv          device bf16 [T*k][H]
+ *   node_staging  device bf16 [moe_node_staging_rows()][H] when
+ *                 MOE_FLAG_TWO_LEVEL is set (NULL otherwise): rows are first
+ *                 written once per (token, node touched), node-major then
+ *                 token order (FUSCO article, "负载均衡与跨节点去重"), then
+ *                 expanded from staging to the expert rows of that node.
+ *                 The final recv is identical in both modes. */
+moe_status_t moe_dispatch(const moe_config_t *cfg, const moe_layout_t *layout,
+                          const void *x, void *recv, void *node_staging,
+                          void *stream);
+
+/* Fused combine: y[t] = bf16_rne( sum_{j=0..k-1} w[t][j] * eo[slot[t][j]] ),
+ * accumulated in fp32 with one fused multiply-add per j in column order,
+ * starting from +0 (INC-MoE abstract: combine returns expert outputs to the
+ * token's owner; the order and precision are this library's choice).
+ *   expert_out    device bf16 [T*k][H], receive-buffer layout
+ *   topk_weights  device fp32 [T][k], used as given
+ *   y             device bf16 [T][H] */
+moe_status_t moe_combine(const moe_config_t *cfg, const moe_layout_t *layout,
+                         const void *expert_out, const float *topk_weights,
+                         void *y, void *stream);
+
+/* Waits for `stream`, reads and clears layout->error_word, and returns the
+ * recorded error: MOE_ERR_EXPERT_OOB before MOE_ERR_DUP_EXPERT before
+ * MOE_ERR_BAD_LAYOUT before MOE_ERR_TIMEOUT; MOE_OK when none. */
+moe_status_t moe_get_error(const moe_layout_t *layout, void *stream);
+
+/* ---- decoupled comparison path (pack -> contiguous copy -> unpack) ----
+ * The design the FUSCO article ("传统 MoE 通信的痛点") measures reorder
+ * passes against: rows are first packed into contiguous per-destination
+ * blocks, the blocks are moved by one contiguous copy, and the receiver
+ * unpacks them into the final layout.  Results equal moe_dispatch /
+ * moe_combine bit for bit. */
+
+/* Dispatch, decoupled.  `cfg` must have num_nodes == num_ranks (<=
+ * MOE_MAX_NODES) and MOE_FLAG_TWO_LEVEL, and `layout` must come from
+ * moe_layout() with that cfg, so its node arrays are per-rank blocks.
+ * Pack: x[t] -> send, once per (token, rank touched), rank-major then token
+ * order.  Copy: send -> xfer (node_offsets[R] rows, read on the device).
+ * Unpack: each xfer row -> the token's expert rows on that rank.
+ *   send, xfer  device bf16 [moe_node_staging_rows(cfg)][H] each. */
+moe_status_t moe_dispatch_decoupled(const moe_config_t *cfg,
+                                    const moe_layout_t *layout, const void *x,
+                                    void *send, void *xfer, void *recv,
+                                    void *stream);
+
+/* Combine, decoupled.  Pack: send[t*k + j] = expert_out[slot[t][j]] (source
+ * order).  Copy: send -> xfer (T*k rows).  Unpack: y[t] = the same fp32 sum
+ * as moe_combine, read from the contiguous rows xfer[t*k .. t*k+k-1].
+ *   send, xfer  device bf16 [T*k][H] each. */
+moe_status_t moe_combine_decoupled(const moe_config_t *cfg,
+                                   const moe_layout_t *layout,
+                                   const void *expert_out,
+                                   const float *topk_weights, void *send,
+                                   void *xfer, void *y, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_LAYOUT_H */

@@ -1,0 +1,261 @@
+"""GPU parity: the CUDA path through the C ABI against the oracle.
+
+Layout and dispatch must match bit for bit; combine must be within 1e-2
+relative / 1e-3 absolute of the oracle (and is expected to be bit-exact,
+since both sides use the same fp32 FMA order and one RNE store).  Small
+shapes compare every value; the five named workloads run at full size in the
+launch configuration bench.py times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_testlib as M
+from combine_moe_layout_06_b200 import capi, inputs
+
+pytestmark = pytest.mark.gpu
+
+TWO = capi.MOE_FLAG_TWO_LEVEL
+
+SMALL = [
+    # T, H, E, k, R, N
+    (1, 8, 4, 1, 1, 1),
+    (7, 64, 8, 3, 4, 2),
+    (33, 136, 13, 4, 5, 5),
+    (255, 128, 16, 8, 8, 4),
+    (256, 128, 8, 2, 2, 1),
+    (257, 72, 64, 8, 4, 2),
+    (1000, 256, 60, 4, 7, 7),
+    (513, 9, 20, 6, 10, 5),      # odd row: 18 bytes -> 2-byte vectors
+    (300, 10, 32, 16, 8, 8),     # 20-byte rows -> 4-byte vectors, k > 8
+    (130, 64, 32, 32, 4, 2),     # k = E = 32
+    (600, 16, 1024, 8, 32, 32),  # E at the library maximum
+    (2049, 2048, 64, 8, 4, 1),
+]
+
+
+def _small_inputs(T, H, E, k, seed):
+    d = inputs.make_random(T, H, E, k, seed=seed, zipf_s=0.7)
+    return d["x"], d["topk_idx"], d["topk_w"]
+
+
+@pytest.mark.parametrize("T,H,E,k,R,N", SMALL)
+def test_layout_small(oracle_mod, T, H, E, k, R, N):
+    _, topk, _ = _small_inputs(T, H, E, k, seed=T + E)
+    for flags in (0, TWO):
+        cfg = M.cfg_of(T, H, E, k, R, N, flags)
+        lay, _ = M.gpu_layout(cfg, topk)
+        ref = oracle_mod.layout(topk, E, R, N, nodes=bool(flags))
+        M.assert_layout_equal(lay.host(), ref)
+        assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+@pytest.mark.parametrize("T,H,E,k,R,N", SMALL)
+def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
+    x, topk, w = _small_inputs(T, H, E, k, seed=3 * T + H)
+    ref = oracle_mod.layout(topk, E, R, N, nodes=True)
+    recv_ref = oracle_mod.dispatch_flat(x, ref["slot"])
+    staging_ref, recv2_ref = oracle_mod.dispatch_two_level(x, ref, R, N)
+    assert np.array_equal(recv2_ref, recv_ref)
+    eo = inputs.random_bf16_bits((T * k, H), seed=T * k + H)
+    y_ref = oracle_mod.combine(eo, w, ref["slot"])
+    x_dev = M.to_dev(x)
+    for flags in (0, TWO):
+        cfg = M.cfg_of(T, H, E, k, R, N, flags)
+        lay, _ = M.gpu_layout(cfg, topk)
+        recv, staging = M.gpu_dispatch(cfg, lay, x_dev, fill=0x7F81)
+        assert np.array_equal(M.bits(recv), recv_ref)
+        if flags:
+            U = int(ref["node_offsets"][-1])
+            st = M.bits(staging)
+            assert np.array_equal(st[:U], staging_ref)
+            assert np.all(st[U:] == 0x7F81), "no stray staging writes"
+        y = M.gpu_combine(cfg, lay, M.to_dev(eo), w)
+        M.assert_combine_close(M.bits(y), y_ref)
+        assert np.array_equal(M.bits(y), y_ref), "fixed-order fp32 FMA is bit-exact"
+        assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_empty_batch(oracle_mod):
+    cfg = M.cfg_of(0, 64, 8, 2, 2, 2, TWO)
+    lay, _ = M.gpu_layout(cfg, np.zeros((0, 2), np.int32))
+    h = lay.host()
+    assert not h["expert_offsets"].any() and not h["rank_offsets"].any()
+    assert not h["node_offsets"].any() and not h["expert_counts"].any()
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    capi.moe_dispatch(cfg, lay.struct, x, x, x)
+    capi.moe_combine(cfg, lay.struct, x, torch.empty(0, device="cuda"), x)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_k1_unit_weight_round_trip_is_identity():
+    x, topk, _ = _small_inputs(777, 96, 12, 1, seed=5)
+    cfg = M.cfg_of(777, 96, 12, 1, 3)
+    lay, _ = M.gpu_layout(cfg, topk)
+    x_dev = M.to_dev(x)
+    recv, _ = M.gpu_dispatch(cfg, lay, x_dev)
+    y = M.gpu_combine(cfg, lay, recv, np.ones((777, 1), np.float32))
+    assert torch.equal(y.view(torch.int16), x_dev.view(torch.int16))
+
+
+def test_round_trip_identity_expert_renormalised():
+    x, topk, w = _small_inputs(1500, 512, 32, 6, seed=8)
+    cfg = M.cfg_of(1500, 512, 32, 6, 4)
+    lay, _ = M.gpu_layout(cfg, topk)
+    recv, _ = M.gpu_dispatch(cfg, lay, M.to_dev(x))
+    y = M.gpu_combine(cfg, lay, recv, w)
+    M.assert_combine_close(M.bits(y), x)
+
+
+def test_unaligned_buffers(oracle_mod):
+    """Base addresses off the 16-byte grid take the narrow-vector kernels."""
+    T, H, E, k, R = 300, 64, 16, 4, 4
+    x, topk, w = _small_inputs(T, H, E, k, seed=21)
+    ref = oracle_mod.layout(topk, E, R)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, topk)
+    for shift in (1, 2):   # elements: 2-byte and 4-byte offsets
+        xs = torch.empty(T * H + 8, dtype=torch.bfloat16, device="cuda")
+        xv = xs[shift:shift + T * H].view(T, H)
+        xv.copy_(M.to_dev(x))
+        rs = torch.empty(T * k * H + 8, dtype=torch.bfloat16, device="cuda")
+        rv = rs[shift:shift + T * k * H].view(T * k, H)
+        capi.moe_dispatch(cfg, lay.struct, xv, rv)
+        assert np.array_equal(M.bits(rv), oracle_mod.dispatch_flat(x, ref["slot"]))
+        ys = torch.empty(T * H + 8, dtype=torch.bfloat16, device="cuda")
+        yv = ys[shift:shift + T * H].view(T, H)
+        capi.moe_combine(cfg, lay.struct, rv, torch.from_numpy(w).cuda(), yv)
+        assert np.array_equal(M.bits(yv), oracle_mod.combine(M.bits(rv), w, ref["slot"]))
+
+
+# ---------------------------------------------------------------- workloads
+
+NAMES = ["tiny", "olmoe", "qwen3", "dsv3", "longctx"]
+
+
+def _workload_cfg(wl, two_level):
+    return M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, TWO if two_level else 0)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_workload_layout_dispatch(oracle_mod, name):
+    d = inputs.make(name)
+    wl = d["workload"]
+    x, topk = d["x"], d["topk_idx"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
+    x_dev = M.to_dev(x)
+    modes = [False, True] if wl.two_level or wl.N > 1 else [False]
+    for two in modes:
+        cfg = _workload_cfg(wl, two)
+        lay, _ = M.gpu_layout(cfg, topk)
+        got = lay.host()
+        want = ref if two else {k_: v for k_, v in ref.items() if not k_.startswith("node")}
+        M.assert_layout_equal(got, want)
+        recv, staging = M.gpu_dispatch(cfg, lay, x_dev)
+        # every receive row equals its token's row (full check on the device)
+        slot_dev = torch.from_numpy(ref["slot"].reshape(-1).astype(np.int64)).cuda()
+        tok_dev = torch.arange(wl.T, device="cuda").repeat_interleave(wl.k)
+        assert torch.equal(recv.view(torch.int16)[slot_dev], x_dev.view(torch.int16)[tok_dev])
+        del slot_dev, tok_dev
+        if wl.T * wl.k * wl.H <= 1 << 30:
+            assert np.array_equal(M.bits(recv), oracle_mod.dispatch_flat(x, ref["slot"]))
+        if two:
+            U = int(ref["node_offsets"][-1])
+            node_tok = np.concatenate([np.flatnonzero(ref["node_slot"][:, n] >= 0)
+                                       for n in range(wl.N)])
+            assert node_tok.size == U
+            st = staging[:U].view(torch.int16)
+            assert torch.equal(st, x_dev.view(torch.int16)[torch.from_numpy(node_tok).cuda()])
+        assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+        del recv, staging
+        torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_workload_combine(oracle_mod, name):
+    d = inputs.make(name)
+    wl = d["workload"]
+    topk, w = d["topk_idx"], d["topk_w"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R)
+    eo = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
+    y_ref = oracle_mod.combine(eo, w, ref["slot"])
+    cfg = _workload_cfg(wl, wl.two_level)
+    lay, _ = M.gpu_layout(cfg, topk)
+    y = M.bits(M.gpu_combine(cfg, lay, M.to_dev(eo), w))
+    M.assert_combine_close(y, y_ref)
+    assert np.array_equal(y, y_ref)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+# ---------------------------------------------------------------- decoupled
+
+@pytest.mark.parametrize("name", ["tiny", "olmoe", "longctx"])
+def test_decoupled_equals_fused(oracle_mod, name):
+    d = inputs.make(name)
+    wl = d["workload"]
+    x, topk, w = d["x"], d["topk_idx"], d["topk_w"]
+    x_dev = M.to_dev(x)
+    fused_cfg = _workload_cfg(wl, False)
+    flay, _ = M.gpu_layout(fused_cfg, topk)
+    recv_f, _ = M.gpu_dispatch(fused_cfg, flay, x_dev)
+    y_f = M.gpu_combine(fused_cfg, flay, recv_f, w)
+    dcfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R, TWO)
+    dlay, _ = M.gpu_layout(dcfg, topk)
+    rows = capi.moe_node_staging_rows(dcfg)
+    send = torch.empty((rows, wl.H), dtype=torch.bfloat16, device="cuda")
+    xfer = torch.empty_like(send)
+    recv_d = torch.empty_like(recv_f)
+    capi.moe_dispatch_decoupled(dcfg, dlay.struct, x_dev, send, xfer, recv_d)
+    assert torch.equal(recv_d.view(torch.int16), recv_f.view(torch.int16))
+    send2 = torch.empty_like(recv_f)
+    xfer2 = torch.empty_like(recv_f)
+    y_d = torch.empty_like(y_f)
+    wd = torch.from_numpy(w).cuda()
+    capi.moe_combine_decoupled(dcfg, dlay.struct, recv_d, wd, send2, xfer2, y_d)
+    assert torch.equal(y_d.view(torch.int16), y_f.view(torch.int16))
+    if wl.T <= 4096:
+        ref = oracle_mod.layout(topk, wl.E, wl.R)
+        assert np.array_equal(M.bits(y_d), oracle_mod.combine(M.bits(recv_d), w, ref["slot"]))
+    assert capi.moe_get_error(dlay.struct) == capi.MOE_OK
+
+
+# ---------------------------------------------------------------- errors
+
+def test_device_data_errors_are_reported():
+    T, H, E, k, R = 64, 32, 8, 2, 2
+    _, topk, w = _small_inputs(T, H, E, k, seed=1)
+    bad = topk.copy()
+    bad[5, 1] = E          # out of range
+    cfg = M.cfg_of(T, H, E, k, R, 2, TWO)
+    lay, _ = M.gpu_layout(cfg, bad)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_EXPERT_OOB
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK, "reading clears the word"
+    dup = topk.copy()
+    dup[9, 1] = dup[9, 0]
+    lay, _ = M.gpu_layout(cfg, dup)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_DUP_EXPERT
+    neg = topk.copy()
+    neg[0, 0] = -3
+    neg[1, 1] = neg[1, 0]
+    lay, _ = M.gpu_layout(cfg, neg)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_EXPERT_OOB, "out-of-range wins"
+    # the layout of the valid entries still only names rows inside the buffer
+    h = lay.host()
+    s = h["slot"]
+    assert s[0, 0] == -1 and s[1, 1] == -1
+    valid = s[s >= 0]
+    assert valid.max() < T * k and np.unique(valid).size == valid.size
+
+
+def test_bad_slot_is_reported_and_skipped():
+    T, H, E, k, R = 40, 64, 8, 2, 2
+    x, topk, w = _small_inputs(T, H, E, k, seed=2)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, topk)
+    lay.slot[3] = T * k + 5          # corrupt one slot
+    recv = torch.zeros((T * k, H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_dispatch(cfg, lay.struct, M.to_dev(x), recv)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_BAD_LAYOUT
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_combine(cfg, lay.struct, recv, torch.from_numpy(w).cuda(), y)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_BAD_LAYOUT
