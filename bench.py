@@ -56,6 +56,37 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+KERNEL_SOURCES = {
+    "combine": ["combine.cu", "moe_common.cuh"],
+    "dispatch": ["dispatch.cu", "moe_common.cuh"],
+}
+
+
+def kernel_source_sha(stage):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[stage]:
+        with open(os.path.join(ROOT, "combine_moe_layout_06_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(stage, workload):
+    """DRAM bytes per launch (read + write) from the committed ncu summary of
+    this kernel, or None when there is none or the kernel source changed
+    since it was captured."""
+    import glob
+    import re
+    want = kernel_source_sha(stage)
+    pat = re.compile(r"<!-- roofline-traffic kernel=(\w+) workload=(\w+) bytes=(\d+) sources=(\w+) -->")
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        with open(path) as f:
+            for m in pat.finditer(f.read()):
+                if m.group(1) == stage and m.group(2) == workload and m.group(4) == want:
+                    return int(m.group(3))
+    return None
+
+
 def algorithmic_bytes(wl, tokens=None):
     T = wl.T if tokens is None else tokens
     row = wl.H * 2
@@ -386,7 +417,8 @@ def main():
                            "combine": round(t_combine, 5)},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": None, "peak_kind": f"{peak_src} copy bandwidth"},
+                         "traffic": profiled_traffic(dom, wl.name),
+                         "peak_kind": f"{peak_src} copy bandwidth (burst: kernel timed alone)"},
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

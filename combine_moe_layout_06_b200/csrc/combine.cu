@@ -11,9 +11,11 @@
 // float(eo[slot[t][j]][h]), acc) with a single rounding per step; the store
 // rounds to nearest even.
 //
-// One warp per token.  Lanes hold the k slots and weights; each pass covers
-// 32*VPL vectors of the row, and rows are fetched four at a time so that
-// 4*VPL streaming loads per lane are in flight before their FMAs.
+// Work items are (token, row chunk) pairs, a chunk being 32*VPL vectors of
+// the row, handed out warp by warp over a persistent grid sized to what is
+// resident, so every SM stays busy to the end.  Lanes hold the token's k
+// slots and weights; the chunk of up to KB expert rows is loaded before any
+// FMA, so KB*VPL streaming loads per lane are in flight at once.
 #include "moe_kernels.h"
 
 namespace moe {
@@ -21,7 +23,6 @@ namespace {
 
 constexpr int kWarpsPerCta = 8;
 constexpr int kThreads = kWarpsPerCta * 32;
-constexpr int kRowsInFlight = 4;
 
 struct CombArgs {
     const void* eo;
@@ -35,17 +36,23 @@ struct CombArgs {
     int* err;
 };
 
-template <typename V, int VPL>
+template <typename V, int VPL, int KB>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     constexpr int EPV = VecInfo<V>::kElems;
+    constexpr int CHUNK = 32 * VPL;
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
+    const int64_t items = a.T * cpr;
     const V* eo = static_cast<const V*>(a.eo);
     V* y = static_cast<V*>(a.y);
     int errbits = 0;
-    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < a.T; t += nwarps) {
+    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
+         item += nwarps) {
+        const int64_t t = item / cpr;
+        const int64_t base = (item - t * cpr) * CHUNK;
         int s = -1;
         float wl = 0.f;
         if (lane < a.k) {
@@ -56,55 +63,66 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
                 s = -1;
             }
         }
-        for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
-            float acc[VPL][EPV];
+        float acc[VPL][EPV];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i)
+        for (int i = 0; i < VPL; ++i)
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) acc[i][e] = 0.f;
-            for (int j0 = 0; j0 < a.k; j0 += kRowsInFlight) {
-                V v[kRowsInFlight][VPL];
-                float wq[kRowsInFlight];
-                bool ok[kRowsInFlight];
+            for (int e = 0; e < EPV; ++e) acc[i][e] = 0.f;
+        for (int j0 = 0; j0 < a.k; j0 += KB) {
+            V v[KB][VPL];
+            float wq[KB];
+            bool ok[KB];
 #pragma unroll
-                for (int q = 0; q < kRowsInFlight; ++q) {
-                    const int j = j0 + q;
-                    const int sj = __shfl_sync(kFullMask, s, j & 31);
-                    wq[q] = __shfl_sync(kFullMask, wl, j & 31);
-                    ok[q] = j < a.k && sj >= 0;
-                    if (ok[q]) {
-                        const V* row = eo + (int64_t)sj * a.rv;
-#pragma unroll
-                        for (int i = 0; i < VPL; ++i) {
-                            const int64_t idx = base + i * 32 + lane;
-                            if (idx < a.rv) v[q][i] = ld_stream(row + idx);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < kRowsInFlight; ++q) {
-                    if (!ok[q]) continue;
+            for (int q = 0; q < KB; ++q) {
+                const int j = j0 + q;
+                const int sj = __shfl_sync(kFullMask, s, j & 31);
+                wq[q] = __shfl_sync(kFullMask, wl, j & 31);
+                ok[q] = j < a.k && sj >= 0;
+                if (ok[q]) {
+                    const V* row = eo + (int64_t)sj * a.rv + base;
 #pragma unroll
                     for (int i = 0; i < VPL; ++i) {
                         const int64_t idx = base + i * 32 + lane;
-                        if (idx < a.rv) {
-                            float f[EPV];
-                            unpack_bf16<V>(v[q][i], f);
-#pragma unroll
-                            for (int e = 0; e < EPV; ++e) acc[i][e] = __fmaf_rn(wq[q], f[e], acc[i][e]);
-                        }
+                        if (idx < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
                     }
                 }
             }
-            V* yrow = y + t * a.rv;
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int64_t idx = base + i * 32 + lane;
-                if (idx < a.rv) yrow[idx] = pack_bf16<V>(acc[i]);
+            for (int q = 0; q < KB; ++q) {
+                if (!ok[q]) continue;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int64_t idx = base + i * 32 + lane;
+                    if (idx < a.rv) {
+                        float f[EPV];
+                        unpack_bf16<V>(v[q][i], f);
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) acc[i][e] = __fmaf_rn(wq[q], f[e], acc[i][e]);
+                    }
+                }
             }
+        }
+        V* yrow = y + t * a.rv + base;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int64_t idx = base + i * 32 + lane;
+            if (idx < a.rv) yrow[i * 32 + lane] = pack_bf16<V>(acc[i]);
         }
     }
     warp_report(a.err, errbits);
+}
+
+template <typename V, int VPL, int KB>
+cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
+    constexpr auto kern = combine_kernel<V, VPL, KB>;
+    const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
+    const int grid = persistent_grid<kern>(a.T * cpr, kThreads);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
+template <typename V, int VPL>
+cudaError_t launch_combine_k(CombArgs a, cudaStream_t stream) {
+    return a.k <= 4 ? launch_combine_v<V, VPL, 4>(a, stream) : launch_combine_v<V, VPL, 8>(a, stream);
 }
 
 inline int vec_bytes(size_t row_bytes, const void* a, const void* b) {
@@ -128,19 +146,16 @@ cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void*
     a.k = p.k;
     a.eo_rows = p.T * p.k;
     a.err = p.err;
-    int64_t g = (p.T + kWarpsPerCta - 1) / kWarpsPerCta;
-    const int64_t cap = (int64_t)device_sm_count() * 16;
-    const int grid = (int)(g > cap ? cap : g);
     switch (vec_bytes(p.row_bytes, expert_out, y)) {
         case 16:
             a.rv = (int64_t)(p.row_bytes / 16);
-            return launch_pdl(combine_kernel<uint4, 2>, dim3(grid), dim3(kThreads), 0, stream, a);
+            return launch_combine_k<uint4, 2>(a, stream);
         case 4:
             a.rv = (int64_t)(p.row_bytes / 4);
-            return launch_pdl(combine_kernel<uint32_t, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+            return launch_combine_k<uint32_t, 4>(a, stream);
         default:
             a.rv = (int64_t)(p.row_bytes / 2);
-            return launch_pdl(combine_kernel<uint16_t, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+            return launch_combine_k<uint16_t, 4>(a, stream);
     }
 }
 

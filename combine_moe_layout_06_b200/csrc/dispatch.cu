@@ -10,10 +10,11 @@
 // one "node" per rank, plus a contiguous copy, form the decoupled
 // pack -> copy -> unpack path that section "传统 MoE 通信的痛点" describes.
 //
-// Register engine: one warp moves one source row.  Lanes hold the
-// destination rows (k <= 32 slots, or N <= 32 nodes); the row is loaded in
-// passes of 32*VPL vectors with streaming loads and stored to every
-// destination with evict-first stores.  The bulk engine lives in bulk.cu.
+// Register engine: work items are (source row, row chunk) pairs, a chunk
+// being 32*VPL vectors, handed out warp by warp over a persistent grid sized
+// to what is resident.  Lanes hold the destination rows (k <= 32 slots, or
+// N <= 32 nodes); the chunk is loaded once with streaming loads and stored
+// to every destination with evict-first stores.
 #include <initializer_list>
 
 #include "moe_kernels.h"
@@ -55,32 +56,36 @@ struct FanArgs {
     int* err;
 };
 
-// One warp per work item.  Flat and node-pack items are tokens; node-expand
-// items are (node, token) pairs, node-major, so each node's forwarder work
-// is one contiguous run of items.
+// Flat and node-pack rows are tokens; node-expand rows are (node, token)
+// pairs, node-major, so each node's forwarder work is one contiguous run.
 template <int MODE, typename V, int VPL>
 __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
+    constexpr int CHUNK = 32 * VPL;
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
-    const int64_t items = MODE == kNodeExpand ? a.T * a.N : a.T;
+    const int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
+    const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
+    const int64_t items = rows * cpr;
     const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
     int errbits = 0;
     for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
          item += nwarps) {
+        const int64_t row = item / cpr;
+        const int64_t base = (item - row * cpr) * CHUNK;
         int64_t src_row;
         int64_t dst = -1;
         if (MODE == kFlat) {
-            src_row = item;
+            src_row = row;
             if (lane < a.k) {
-                const int s = __ldg(a.slot + item * a.k + lane);
+                const int s = __ldg(a.slot + row * a.k + lane);
                 if (s >= 0 && s < a.dst_rows) dst = s;
                 else if (s != -1) errbits |= kErrBadLayout;
             }
         } else if (MODE == kNodePack) {
-            src_row = item;
+            src_row = row;
             if (lane < a.N) {
-                const int ns = __ldg(a.node_slot + item * a.N + lane);
+                const int ns = __ldg(a.node_slot + row * a.N + lane);
                 if (ns >= 0) {
                     const int64_t d = (int64_t)__ldg(a.node_offsets + lane) + ns;
                     if (d >= 0 && d < a.dst_rows) dst = d;
@@ -88,8 +93,8 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
                 }
             }
         } else {
-            const int n = (int)(item / a.T);
-            const int64_t t = item - (int64_t)n * a.T;
+            const int n = (int)(row / a.T);
+            const int64_t t = row - (int64_t)n * a.T;
             const int ns = __ldg(a.node_slot + t * a.N + n);  // same for all lanes
             if (ns < 0) continue;
             src_row = (int64_t)__ldg(a.node_offsets + n) + ns;
@@ -105,69 +110,56 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
             }
         }
         const unsigned dmask = __ballot_sync(kFullMask, dst >= 0);
-        const V* srow = static_cast<const V*>(a.src) + src_row * a.rv;
-        V* dbase = static_cast<V*>(a.dst);
-        for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
-            V v[VPL];
+        const V* src = static_cast<const V*>(a.src) + src_row * a.rv + base;
+        V* dbase = static_cast<V*>(a.dst) + base;
+        V v[VPL];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int64_t idx = base + i * 32 + lane;
-                if (idx < a.rv) v[i] = ld_stream(srow + idx);
-            }
-            unsigned m = dmask;
-            while (m) {
-                const int j = __ffs(m) - 1;
-                m &= m - 1;
-                const int64_t d = __shfl_sync(kFullMask, dst, j);
-                V* drow = dbase + d * a.rv;
+        for (int i = 0; i < VPL; ++i)
+            if (base + i * 32 + lane < a.rv) v[i] = ld_stream(src + i * 32 + lane);
+        unsigned m = dmask;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            const int64_t d = __shfl_sync(kFullMask, dst, j);
+            V* drow = dbase + d * a.rv;
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int64_t idx = base + i * 32 + lane;
-                    if (idx < a.rv) st_stream(drow + idx, v[i]);
-                }
-            }
+            for (int i = 0; i < VPL; ++i)
+                if (base + i * 32 + lane < a.rv) st_stream(drow + i * 32 + lane, v[i]);
         }
     }
     warp_report(a.err, errbits);
 }
 
-// dst[t*k + j] = src[slot[t][j]] (decoupled combine's pack).  One warp per
-// token, one source row at a time.
+// dst[t*k + j] = src[slot[t][j]] (decoupled combine's pack).  Items are
+// (destination row, row chunk) pairs.
 template <typename V, int VPL>
 __global__ void __launch_bounds__(kThreads) gather_kernel(FanArgs a) {
+    constexpr int CHUNK = 32 * VPL;
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
+    const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
+    const int64_t items = a.T * a.k * cpr;
     const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
     int errbits = 0;
-    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); t < a.T; t += nwarps) {
-        int s = -1;
-        if (lane < a.k) {
-            s = __ldg(a.slot + t * a.k + lane);
-            if (s < 0 || s >= a.src_rows) {
-                if (s != -1) errbits |= kErrBadLayout;
-                s = -1;
-            }
+    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
+         item += nwarps) {
+        const int64_t drow = item / cpr;
+        const int64_t base = (item - drow * cpr) * CHUNK;
+        const int s = __ldg(a.slot + drow);   // same for all lanes
+        if (s < 0 || s >= a.src_rows) {
+            if (s != -1) errbits |= kErrBadLayout;
+            continue;
         }
-        for (int j = 0; j < a.k; ++j) {
-            const int sj = __shfl_sync(kFullMask, s, j);
-            if (sj < 0) continue;
-            const V* srow = static_cast<const V*>(a.src) + (int64_t)sj * a.rv;
-            V* drow = static_cast<V*>(a.dst) + (t * a.k + j) * a.rv;
-            for (int64_t base = 0; base < a.rv; base += 32 * VPL) {
-                V v[VPL];
+        const V* src = static_cast<const V*>(a.src) + (int64_t)s * a.rv + base;
+        V* dst = static_cast<V*>(a.dst) + drow * a.rv + base;
+        V v[VPL];
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int64_t idx = base + i * 32 + lane;
-                    if (idx < a.rv) v[i] = ld_stream(srow + idx);
-                }
+        for (int i = 0; i < VPL; ++i)
+            if (base + i * 32 + lane < a.rv) v[i] = ld_stream(src + i * 32 + lane);
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int64_t idx = base + i * 32 + lane;
-                    if (idx < a.rv) st_stream(drow + idx, v[i]);
-                }
-            }
-        }
+        for (int i = 0; i < VPL; ++i)
+            if (base + i * 32 + lane < a.rv) st_stream(dst + i * 32 + lane, v[i]);
     }
     warp_report(a.err, errbits);
 }
@@ -208,22 +200,20 @@ inline int vec_bytes(size_t row_bytes, std::initializer_list<const void*> ptrs) 
     return 2;
 }
 
-inline int grid_for(int64_t warp_items) {
-    const int64_t cap = (int64_t)device_sm_count() * 16;
-    int64_t g = (warp_items + kWarpsPerCta - 1) / kWarpsPerCta;
-    if (g > cap) g = cap;
-    return (int)(g < 1 ? 1 : g);
+template <int MODE, typename V, int VPL>
+cudaError_t launch_fan_vpl(FanArgs a, int64_t rows, cudaStream_t stream) {
+    constexpr auto kern = fanout_kernel<MODE, V, VPL>;
+    const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
+    const int grid = persistent_grid<kern>(rows * cpr, kThreads);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
 }
 
 template <int MODE, typename V>
-cudaError_t launch_fan_v(FanArgs a, int64_t items, cudaStream_t stream) {
+cudaError_t launch_fan_v(FanArgs a, int64_t rows, cudaStream_t stream) {
     a.rv /= sizeof(V);
-    const int grid = grid_for(items);
-    if (sizeof(V) == 16 && a.rv % (32 * 7) == 0 && a.rv % (32 * 8) != 0)
-        return launch_pdl(fanout_kernel<MODE, V, 7>, dim3(grid), dim3(kThreads), 0, stream, a);
-    if (a.rv >= 32 * 8)
-        return launch_pdl(fanout_kernel<MODE, V, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
-    return launch_pdl(fanout_kernel<MODE, V, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
+    // chunks that tile the row exactly where possible
+    if (a.rv % (32 * 4) == 0 || a.rv > 32 * 4) return launch_fan_vpl<MODE, V, 4>(a, rows, stream);
+    return launch_fan_vpl<MODE, V, 2>(a, rows, stream);
 }
 
 template <int MODE>
@@ -280,17 +270,26 @@ cudaError_t launch_gather_rows(const RowMoveParams& p, const void* src, void* ds
                                cudaStream_t stream) {
     if (p.T <= 0) return cudaSuccess;
     FanArgs a = fan_args(p, src, dst, p.T * p.k, p.T * p.k);
-    const int grid = grid_for(p.T);
+    const int64_t rows = p.T * p.k;
     switch (vec_bytes(p.row_bytes, {src, dst})) {
-        case 16:
+        case 16: {
             a.rv /= 16;
-            return launch_pdl(gather_kernel<uint4, 4>, dim3(grid), dim3(kThreads), 0, stream, a);
-        case 4:
+            constexpr auto kern = gather_kernel<uint4, 4>;
+            const int grid = persistent_grid<kern>(rows * ((a.rv + 127) / 128), kThreads);
+            return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+        }
+        case 4: {
             a.rv /= 4;
-            return launch_pdl(gather_kernel<uint32_t, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
-        default:
+            constexpr auto kern = gather_kernel<uint32_t, 8>;
+            const int grid = persistent_grid<kern>(rows * ((a.rv + 255) / 256), kThreads);
+            return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+        }
+        default: {
             a.rv /= 2;
-            return launch_pdl(gather_kernel<uint16_t, 8>, dim3(grid), dim3(kThreads), 0, stream, a);
+            constexpr auto kern = gather_kernel<uint16_t, 8>;
+            const int grid = persistent_grid<kern>(rows * ((a.rv + 255) / 256), kThreads);
+            return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+        }
     }
 }
 

@@ -202,4 +202,30 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
+// Resident blocks per SM of a kernel at a block size (queried once per
+// kernel).
+template <auto Kernel>
+inline int blocks_per_sm(int threads, size_t smem = 0) {
+    static int cached = 0;
+    if (cached == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
+            n < 1)
+            n = 1;
+        cached = n;
+    }
+    return cached;
+}
+
+// Grid for a persistent warp-strided loop over `warp_items` items: enough
+// blocks to give every warp an item, capped at what is resident at once.
+template <auto Kernel>
+inline int persistent_grid(int64_t warp_items, int threads, size_t smem = 0) {
+    const int64_t warps_per_block = threads / 32;
+    const int64_t resident = (int64_t)device_sm_count() * blocks_per_sm<Kernel>(threads, smem);
+    int64_t g = (warp_items + warps_per_block - 1) / warps_per_block;
+    if (g > resident) g = resident;
+    return (int)(g < 1 ? 1 : g);
+}
+
 }  // namespace moe
