@@ -47,7 +47,10 @@ ENTRY_POINTS = (
     "moe_status_string", "moe_check_config", "moe_expert_partition",
     "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
+    "moe_layout_noalloc",
 )
+
+MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class MoeConfig(ctypes.Structure):
@@ -97,6 +100,7 @@ def lib() -> ctypes.CDLL:
     L.moe_get_error.argtypes = [LP, P]
     L.moe_dispatch_decoupled.argtypes = [C, LP, P, P, P, P, P]
     L.moe_combine_decoupled.argtypes = [C, LP, P, P, P, P, P, P]
+    L.moe_layout_noalloc.argtypes = [C, P, LP, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -197,3 +201,10 @@ def moe_combine_decoupled(cfg: MoeConfig, layout: MoeLayout, expert_out, topk_we
     _check(lib().moe_combine_decoupled(ctypes.byref(cfg), ctypes.byref(layout), _ptr(expert_out),
                                        _ptr(topk_weights), _ptr(send), _ptr(xfer), _ptr(y),
                                        _stream(stream)), "moe_combine_decoupled")
+
+
+def moe_layout_noalloc(cfg: MoeConfig, topk_idx, layout: MoeLayout, stream=None) -> None:
+    """moe_layout() with the library's fixed device scratch instead of
+    layout.workspace (for callers that cannot allocate device memory)."""
+    _check(lib().moe_layout_noalloc(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(layout),
+                                    _stream(stream)), "moe_layout_noalloc")

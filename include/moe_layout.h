@@ -223,6 +223,32 @@ moe_status_t moe_combine_decoupled(const moe_config_t *cfg,
                                    const float *topk_weights, void *send,
                                    void *xfer, void *y, void *stream);
 
+/* ---- layout without caller-provided scratch ----
+ * No counterpart on the pages: this entry point exists for callers that
+ * cannot allocate device memory (for example code that runs while a stream
+ * is being captured and may not allocate, runtimes without a device
+ * allocator, or plugins whose host framework owns every allocation).
+ *
+ * Same inputs, outputs and results as moe_layout(), but the layout's
+ * scratch comes from a fixed array of MOE_LAYOUT_NOALLOC_SCRATCH_BYTES bytes
+ * inside the library's device memory (held on every GPU that loads the
+ * library until the process exits); layout->workspace is ignored and may be
+ * NULL.  Nothing is allocated.
+ *  - Limit: configurations whose moe_layout_workspace_bytes() exceeds
+ *    MOE_LAYOUT_NOALLOC_SCRATCH_BYTES are refused with MOE_ERR_INVALID_ARG
+ *    before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array: calls that overlap on the
+ *    GPU (other streams, or other threads' streams) race and give wrong
+ *    layouts.  Order them on one stream or with events.
+ *  - The array keeps the last call's contents; a call reads only what it
+ *    wrote itself, so nothing needs clearing between calls. */
+#define MOE_LAYOUT_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status_t moe_layout_noalloc(const moe_config_t *cfg, const int32_t *topk_idx,
+                                const moe_layout_t *layout, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
