@@ -6,14 +6,18 @@ DeepSeek-V3-shaped workload) and fused combine.  The combine reads a separate
 stand-in expert-output buffer (as it would after the expert GEMMs), so no
 step reads rows the same step just wrote through L2.
 
-Timing: W untimed warm-up steps, then exactly K timed steps, each replaying
-the step's CUDA graph between CUDA events on the launching stream, with L2
-flushed (a read of a buffer twice the L2 size) before every step, outside the
-events.  A second pass of K steps replays layout, dispatch and combine as
-three graphs with events between them for the per-kernel breakdown and the
-roofline figure.  Multi-GPU runs are independent replicas (no collective on
-the data path): value = bytes all ranks moved / the max over ranks of the
-timed time.
+Timing: W untimed warm-up steps, then exactly K timed steps back to back,
+bracketed by two CUDA events on the launching stream (and a barrier plus a
+device synchronise on both sides).  Steps alternate between two independent
+buffer sets (inputs, layout, outputs), so no step finds its inputs in L2:
+a buffer is touched again only after about twice the step's traffic (the
+OLMoE-shaped step alone moves 302 MB, 2.4x the L2).  Steps are replayed from
+CUDA graphs of two steps.  Stage costs come from the same protocol applied
+to graphs of layout only and layout + dispatch: dispatch = (layout +
+dispatch) - layout, combine = step - (layout + dispatch).  The decoupled
+pack -> copy -> unpack path is timed the same way for comparison.
+Multi-GPU runs are independent replicas (no collective on the data path):
+value = bytes all ranks moved / the max over ranks of the timed time.
 
 Metric: achieved algorithmic HBM GB/s of dispatch + combine.  Algorithmic
 bytes per step are T*H*2 + T*k*H*2 for dispatch (read each token row once,
@@ -58,7 +62,7 @@ def measured_peak():
 
 KERNEL_SOURCES = {
     "combine": ["combine.cu", "moe_common.cuh"],
-    "dispatch": ["dispatch.cu", "moe_common.cuh"],
+    "dispatch": ["bulk.cu", "dispatch.cu", "moe_common.cuh"],
 }
 
 
@@ -107,7 +111,7 @@ def workload_desc(wl):
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled through NVML every 10 ms
+    """SM clock and clock-event reasons sampled through NVML every 5 ms
     while the timed region runs (read-only queries)."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -139,7 +143,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            self._stop.wait(0.01)
+            self._stop.wait(0.005)
 
     def __enter__(self):
         if self._nv is not None:
@@ -214,6 +218,39 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- HBM probe
+
+def hbm_probe():
+    """Write-only (fill), read-only (sum) and copy bandwidth of 2 GiB bf16
+    buffers with torch's own kernels: the ceilings a write-heavy dispatch and
+    a read-heavy combine are bound by.  Best of 10, CUDA events."""
+    import torch
+    n = 1 << 30
+    a = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    b = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    a.fill_(1.0)
+
+    def best(fn, bytes_moved):
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(10):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            times.append(s.elapsed_time(e) * 1e-3)
+        return round(bytes_moved / min(times) / 1e9, 1)
+
+    out = {"probe": "hbm", "bytes": 2 * n,
+           "write_only_gbs": best(lambda: b.fill_(2.0), 2 * n),
+           "read_only_gbs": best(lambda: a.sum(dtype=torch.float32), 2 * n),
+           "copy_gbs": best(lambda: b.copy_(a), 4 * n)}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- our arm
 
 def main():
@@ -224,14 +261,23 @@ def main():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="olmoe", choices=sorted(inputs.WORKLOADS))
     p.add_argument("--engine", default="auto", choices=["auto", "vector", "bulk"])
+    p.add_argument("--layout", default="kernels", choices=["kernels", "cluster"])
+    p.add_argument("--unfused", action="store_true",
+                   help="moe_layout + moe_dispatch instead of moe_layout_dispatch")
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")
+    p.add_argument("--no-decoupled", action="store_true",
+                   help="skip timing the pack/copy/unpack comparison path")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=0)
+    p.add_argument("--hbm-probe", action="store_true",
+                   help="measure write-only / read-only / copy HBM bandwidth and exit")
     args = p.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         return run_reference(args)
+    if args.hbm_probe:
+        return hbm_probe()
 
     import torch
     import torch.distributed as dist
@@ -254,113 +300,151 @@ def main():
     wl = d["workload"]
     flags = capi.MOE_FLAG_TWO_LEVEL if wl.two_level else 0
     flags |= {"auto": 0, "vector": capi.MOE_FLAG_COPY_VECTOR, "bulk": capi.MOE_FLAG_COPY_BULK}[args.engine]
+    if args.layout == "cluster":
+        flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
     cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
+    # the decoupled comparison path packs per rank: one "node" per rank
+    dcfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R,
+                       capi.MOE_FLAG_TWO_LEVEL | (flags & (capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK)))
     dev = torch.device("cuda", local)
-    lay = buffers.DeviceLayout(cfg, dev)
-    x_dev = buffers.bf16_from_bits(d["x"], dev)
-    topk_dev = torch.from_numpy(d["topk_idx"]).to(dev)
-    w_dev = torch.from_numpy(d["topk_w"]).to(dev)
     eo_bits = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
-    eo_dev = buffers.bf16_from_bits(eo_bits, dev)
-    recv = torch.empty((wl.T * wl.k, wl.H), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device=dev)
-    staging = None
-    if wl.two_level:
-        staging = torch.empty((capi.moe_node_staging_rows(cfg), wl.H), dtype=torch.bfloat16,
-                              device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush_buf = torch.ones(max(2 * l2, 1 << 20) // 4, dtype=torch.float32, device=dev)
+    bf16 = dict(dtype=torch.bfloat16, device=dev)
 
-    def flush():
-        flush_buf.sum()
+    class BufferSet:
+        """One independent set of the step's inputs and outputs."""
 
-    def do_layout():
-        capi.moe_layout(cfg, topk_dev, lay.struct)
+        def __init__(self, decoupled=False):
+            self.lay = buffers.DeviceLayout(cfg, dev)
+            self.x = buffers.bf16_from_bits(d["x"], dev)
+            self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
+            self.w = torch.from_numpy(d["topk_w"]).to(dev)
+            self.eo = buffers.bf16_from_bits(eo_bits, dev)
+            self.recv = torch.empty((wl.T * wl.k, wl.H), **bf16)
+            self.y = torch.empty((wl.T, wl.H), **bf16)
+            self.staging = None
+            if wl.two_level:
+                self.staging = torch.empty((capi.moe_node_staging_rows(cfg), wl.H), **bf16)
+            if decoupled:
+                self.dlay = buffers.DeviceLayout(dcfg, dev)
+                rows = capi.moe_node_staging_rows(dcfg)
+                self.dsend = torch.empty((rows, wl.H), **bf16)
+                self.dxfer = torch.empty((rows, wl.H), **bf16)
+                self.csend = torch.empty((wl.T * wl.k, wl.H), **bf16)
+                self.cxfer = torch.empty((wl.T * wl.k, wl.H), **bf16)
 
-    def do_dispatch():
-        capi.moe_dispatch(cfg, lay.struct, x_dev, recv, staging)
+    with_decoupled = not args.no_decoupled
+    sets = [BufferSet(with_decoupled), BufferSet(with_decoupled)]
 
-    def do_combine():
-        capi.moe_combine(cfg, lay.struct, eo_dev, w_dev, y)
+    def layout(b):
+        capi.moe_layout(cfg, b.topk, b.lay.struct)
 
-    def do_step():
-        do_layout()
-        do_dispatch()
-        do_combine()
+    def layout_dispatch(b):
+        if args.unfused:
+            layout(b)
+            capi.moe_dispatch(cfg, b.lay.struct, b.x, b.recv, b.staging)
+        else:
+            capi.moe_layout_dispatch(cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
 
-    launches_per_step = 3 + (2 if wl.two_level else 1) + 1
+    def step(b):
+        layout_dispatch(b)
+        capi.moe_combine(cfg, b.lay.struct, b.eo, b.w, b.y)
 
-    for _ in range(args.warmup):
-        flush()
-        do_step()
+    def decoupled_step(b):
+        capi.moe_layout(dcfg, b.topk, b.dlay.struct)
+        capi.moe_dispatch_decoupled(dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
+        capi.moe_combine_decoupled(dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
+
+    cluster_layout = args.layout == "cluster" and wl.T <= 131072
+    small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
+    layout_launches = 1 if cluster_layout else (2 if small_layout else 3)
+    launches_per_step = layout_launches + (2 if wl.two_level else 1) + 1
+
+    for i in range(args.warmup):
+        step(sets[i % 2])
+        if with_decoupled:
+            decoupled_step(sets[i % 2])
     torch.cuda.synchronize()
-    st = capi.moe_get_error(lay.struct)
-    if st != capi.MOE_OK:
-        raise SystemExit(f"device error after warm-up: {capi.moe_status_string(st)}")
+    for b in sets:
+        for lay in [b.lay] + ([b.dlay] if with_decoupled else []):
+            st = capi.moe_get_error(lay.struct)
+            if st != capi.MOE_OK:
+                raise SystemExit(f"device error after warm-up: {capi.moe_status_string(st)}")
 
-    # graphs: one for the whole step, one per stage for the breakdown
+    # CUDA graphs over the two buffer sets: a pair of steps (A then B), and a
+    # single step for an odd K; stage prefixes for the breakdown.
     side = torch.cuda.Stream(dev)
-    graphs = {}
-    for name, fn in (("step", do_step), ("layout", do_layout), ("dispatch", do_dispatch),
-                     ("combine", do_combine)):
+
+    def capture(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
             fn()
-        graphs[name] = g
-    for _ in range(3):
-        graphs["step"].replay()
+        return g
+
+    A, B = sets
+    graphs = {
+        "step": (capture(lambda: (step(A), step(B))), capture(lambda: step(A))),
+        "L": (capture(lambda: (layout(A), layout(B))), capture(lambda: layout(A))),
+        "LD": (capture(lambda: (layout_dispatch(A), layout_dispatch(B))),
+               capture(lambda: layout_dispatch(A))),
+    }
+    if with_decoupled:
+        graphs["decoupled"] = (capture(lambda: (decoupled_step(A), decoupled_step(B))),
+                               capture(lambda: decoupled_step(A)))
+    for pair, single in graphs.values():
+        pair.replay()
+        single.replay()
     torch.cuda.synchronize()
+
+    def timed(name, K):
+        """K steps back to back between two events on the stream (ms)."""
+        pair, single = graphs[name]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K // 2):
+            pair.replay()
+        if K % 2:
+            single.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        for i in range(K):
-            flush()
-            ev[i][0].record()
-            graphs["step"].replay()
-            ev[i][1].record()
-        torch.cuda.synchronize()
-    barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-
-    # per-kernel breakdown, same protocol
-    evk = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize()
-    for i in range(K):
-        flush()
-        evk[i][0].record()
-        graphs["layout"].replay()
-        evk[i][1].record()
-        graphs["dispatch"].replay()
-        evk[i][2].record()
-        graphs["combine"].replay()
-        evk[i][3].record()
-    torch.cuda.synchronize()
-    barrier()
-    t_layout = statistics.mean(e[0].elapsed_time(e[1]) for e in evk)
-    t_dispatch = statistics.mean(e[1].elapsed_time(e[2]) for e in evk)
-    t_combine = statistics.mean(e[2].elapsed_time(e[3]) for e in evk)
-    st = capi.moe_get_error(lay.struct)
-    if st != capi.MOE_OK:
-        raise SystemExit(f"device error in the timed region: {capi.moe_status_string(st)}")
+        total_ms = timed("step", K)
+        t_l = timed("L", K) / K
+        t_ld = timed("LD", K) / K
+        dec_ms = timed("decoupled", K) if with_decoupled else None
+    ms_per_step = total_ms / K
+    t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
+    for b in sets:
+        st = capi.moe_get_error(b.lay.struct)
+        if st != capi.MOE_OK:
+            raise SystemExit(f"device error in the timed region: {capi.moe_status_string(st)}")
 
     disp_b, comb_b = algorithmic_bytes(wl)
     step_bytes = disp_b + comb_b
-    ms_per_step = total_ms / K
     value = step_bytes * world * K / (total_ms * 1e-3) / 1e9
     peak, peak_src = measured_peak()
     dom = "dispatch" if t_dispatch >= t_combine else "combine"
     dom_bytes = disp_b if dom == "dispatch" else comb_b
     dom_ms = t_dispatch if dom == "dispatch" else t_combine
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    decoupled = None
+    if dec_ms is not None:
+        dec_value = step_bytes * world * K / (dec_ms * 1e-3) / 1e9
+        decoupled = {"value": round(dec_value, 2), "unit": "GB/s",
+                     "ms_per_step": round(dec_ms / K, 5),
+                     "fused_speedup": round(value / dec_value, 3),
+                     "path": "layout (per-rank groups) + pack/copy/unpack dispatch + "
+                             "pack/copy/unpack combine"}
 
     # end to end through the C ABI from pinned host buffers
     e2e_steps = args.e2e_steps or min(K, 50)
@@ -374,13 +458,12 @@ def main():
     barrier()
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
-        x_dev.copy_(x_h, non_blocking=True)
-        topk_dev.copy_(topk_h, non_blocking=True)
-        w_dev.copy_(w_h, non_blocking=True)
-        do_layout()
-        do_dispatch()
-        capi.moe_combine(cfg, lay.struct, recv, w_dev, y)   # identity expert
-        y_h.copy_(y, non_blocking=True)
+        A.x.copy_(x_h, non_blocking=True)
+        A.topk.copy_(topk_h, non_blocking=True)
+        A.w.copy_(w_h, non_blocking=True)
+        capi.moe_layout_dispatch(cfg, A.topk, A.lay.struct, A.x, A.recv, A.staging)
+        capi.moe_combine(cfg, A.lay.struct, A.recv, A.w, A.y)   # identity expert
+        y_h.copy_(A.y, non_blocking=True)
         torch.cuda.current_stream().synchronize()
     e2e_s = time.perf_counter() - t0
     if world > 1:
@@ -406,8 +489,16 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_desc(wl), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                           l2="flushed before every timed step (read of a 2xL2 buffer, outside the events)",
-                           engine=args.engine, timing="CUDA graph per step, CUDA events"),
+                           l2=("inputs larger than L2: steps alternate between two independent "
+                               "buffer sets, each step moves %.0f MB (%.1fx L2)"
+                               % (step_bytes / 1e6, step_bytes / torch.cuda.get_device_properties(dev).L2_cache_size)),
+                           engine=args.engine,
+                           layout="one cluster launch" if cluster_layout else
+                           ("count + assign kernels" if small_layout else "count/scan/assign kernels"),
+                           entry="moe_layout + moe_dispatch" if args.unfused else "moe_layout_dispatch",
+                           timing="K steps back to back (CUDA graphs of two steps) between two CUDA "
+                                  "events on the launching stream; stage costs from graphs of "
+                                  "layout, layout+dispatch and the full step"),
             "pct_of_peak": round(100 * value / world / peak, 2),
             "peak_gbs": peak, "peak_source": peak_src,
             "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
@@ -418,7 +509,8 @@ def main():
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": profiled_traffic(dom, wl.name),
-                         "peak_kind": f"{peak_src} copy bandwidth (burst: kernel timed alone)"},
+                         "peak_kind": f"{peak_src} copy bandwidth"},
+            "decoupled_3pass": decoupled,
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -426,8 +518,6 @@ def main():
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    for g in graphs.values():
-        del g
     graphs.clear()
     if world > 1:
         dist.destroy_process_group()

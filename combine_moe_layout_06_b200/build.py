@@ -41,16 +41,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str | None = None,
+          defines: tuple = ()) -> str:
+    """Compile the library (to `out` instead of the in-tree path when given,
+    with extra -D `defines` for the compile-time tunables)."""
+    target = out or LIB
+    if out is None and not defines and not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    tmp = target + f".tmp{os.getpid()}"
+    cmd = [NVCC, *FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           *sources()]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

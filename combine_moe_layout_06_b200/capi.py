@@ -24,6 +24,7 @@ MOE_MAX_NODES = 32
 MOE_FLAG_TWO_LEVEL = 0x1
 MOE_FLAG_COPY_VECTOR = 0x2
 MOE_FLAG_COPY_BULK = 0x4
+MOE_FLAG_LAYOUT_CLUSTER = 0x8
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1
@@ -47,7 +48,7 @@ ENTRY_POINTS = (
     "moe_status_string", "moe_check_config", "moe_expert_partition",
     "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
-    "moe_layout_noalloc",
+    "moe_layout_noalloc", "moe_layout_dispatch",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -101,6 +102,7 @@ def lib() -> ctypes.CDLL:
     L.moe_dispatch_decoupled.argtypes = [C, LP, P, P, P, P, P]
     L.moe_combine_decoupled.argtypes = [C, LP, P, P, P, P, P, P]
     L.moe_layout_noalloc.argtypes = [C, P, LP, P]
+    L.moe_layout_dispatch.argtypes = [C, P, LP, P, P, P, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -176,6 +178,13 @@ def moe_dispatch(cfg: MoeConfig, layout: MoeLayout, x, recv, node_staging=None,
                  stream=None) -> None:
     _check(lib().moe_dispatch(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x), _ptr(recv),
                               _ptr(node_staging), _stream(stream)), "moe_dispatch")
+
+
+def moe_layout_dispatch(cfg: MoeConfig, topk_idx, layout: MoeLayout, x, recv, node_staging=None,
+                        stream=None) -> None:
+    _check(lib().moe_layout_dispatch(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(layout),
+                                     _ptr(x), _ptr(recv), _ptr(node_staging), _stream(stream)),
+           "moe_layout_dispatch")
 
 
 def moe_combine(cfg: MoeConfig, layout: MoeLayout, expert_out, topk_weights, y,

@@ -1,0 +1,392 @@
+// bulk.cu -- the bulk-copy (TMA) engine for fused dispatch and combine.
+//
+// Same operations as the register engine in dispatch.cu / combine.cu
+// (FUSCO article, section "FUSCO 的核心创新": rows go straight from where
+// they are to where they belong, with no pack or unpack pass), moved by the
+// SM's bulk-copy unit instead of by registers:
+//
+//  dispatch: each warp runs its own pipeline of kDispStages shared-memory
+//    stages.  Lane 0 starts a cp.async.bulk global->shared load of a row
+//    chunk into a stage (completion counted on the stage's mbarrier); when
+//    it lands, every lane that holds a destination row issues a
+//    cp.async.bulk shared->global store of the stage to that row.  Rows are
+//    read once and written k times without passing through registers, so
+//    store issue no longer throttles the warps.
+//
+//  combine: each warp's stage holds the chunk of all k expert rows of one
+//    token (4 KB: 512-byte chunks for k = 8, one 16-byte vector per lane and
+//    row); lanes j < k each start the bulk load of row j, and when the stage
+//    lands the warp sums the rows in fp32 from shared memory (same FMA order
+//    as the register engine: j = 0 .. k-1 from +0, one RNE store).  Loads
+//    for the next stages are in flight while a stage is summed, and small
+//    stages leave room for 16 warps per SM to hide the summing latency.
+//
+// Every mbarrier wait is bounded; a wait that gives up records kErrTimeout,
+// stops issuing work, drains what it started and returns.  No load uses
+// cluster multicast.  Requires 16-byte aligned rows and base addresses.
+#include <initializer_list>
+
+#include "moe_kernels.h"
+
+namespace moe {
+namespace {
+
+// Pipeline shape (compile-time tunables).
+#ifndef MOE_BULK_DISP_STAGES
+#define MOE_BULK_DISP_STAGES 4
+#endif
+#ifndef MOE_BULK_DISP_CHUNK
+#define MOE_BULK_DISP_CHUNK 4096
+#endif
+#ifndef MOE_BULK_COMB_STAGES
+#define MOE_BULK_COMB_STAGES 3
+#endif
+#ifndef MOE_BULK_COMB_STAGE_BYTES
+#define MOE_BULK_COMB_STAGE_BYTES 4096
+#endif
+constexpr int kBulkWarps = 4;
+constexpr int kBulkThreads = kBulkWarps * 32;
+constexpr int kDispStages = MOE_BULK_DISP_STAGES;
+constexpr uint32_t kDispChunk = MOE_BULK_DISP_CHUNK;
+constexpr int kCombStages = MOE_BULK_COMB_STAGES;
+constexpr uint32_t kCombStageBytes = MOE_BULK_COMB_STAGE_BYTES;  // k row chunks per stage
+
+enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2 };
+
+struct BulkArgs {
+    const char* src;
+    char* dst;
+    const float* w;
+    const int* slot;          // nullptr (combine): row of (t, j) is t*k + j
+    const int* node_slot;
+    const int* node_offsets;
+    const int* rank_offsets;
+    int64_t T;
+    int k, N, ranks_per_node;
+    int64_t row_bytes;
+    uint32_t chunk;           // bytes per row chunk (multiple of 16)
+    int64_t cpr;              // chunks per row
+    int64_t src_rows, dst_rows;
+    int* err;
+    int early;                // start source loads before waiting (see RowMoveParams)
+};
+
+// Drain after a timeout: wait (bounded) for every stage this warp still
+// has a load in flight on, then for its bulk stores.
+__device__ __forceinline__ void drain(uint64_t* full, uint32_t parity_bits, uint32_t inflight,
+                                      int stages) {
+    for (int s = 0; s < stages; ++s)
+        if (inflight & (1u << s)) (void)mbar_wait(&full[s], (parity_bits >> s) & 1u);
+    bulk_wait_all();
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char* stage0 = smem + (size_t)warp * kDispStages * a.chunk;
+    uint64_t* full =
+        reinterpret_cast<uint64_t*>(smem + (size_t)kBulkWarps * kDispStages * a.chunk) + warp * kDispStages;
+    if (lane == 0) {
+        for (int s = 0; s < kDispStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    // Flat and node-pack sources are x rows, which need no layout data: with
+    // early inputs the first stages are loaded while the layout still runs.
+    const bool early = a.early != 0 && MODE != kNodeExpand;
+    pdl_trigger();
+    if (!early) pdl_wait();
+
+    const int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
+    const int64_t items = rows * a.cpr;
+    // a contiguous, row-major range of items per warp
+    const int64_t nwarps = (int64_t)gridDim.x * kBulkWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kBulkWarps + warp;
+    const int64_t first = items * gw / nwarps;
+    const int64_t mine = items * (gw + 1) / nwarps - first;
+    int errbits = 0;
+
+    // Source row of an item (-1: nothing to move), and the chunk geometry.
+    auto source = [&](int64_t item, int64_t& row, int64_t& base, uint32_t& bytes) -> int64_t {
+        row = item / a.cpr;
+        base = (item - row * a.cpr) * (int64_t)a.chunk;
+        const int64_t left = a.row_bytes - base;
+        bytes = left < (int64_t)a.chunk ? (uint32_t)left : a.chunk;
+        if (MODE != kNodeExpand) return row;
+        const int n = (int)(row / a.T);
+        const int64_t t = row - (int64_t)n * a.T;
+        const int ns = __ldg(a.node_slot + t * a.N + n);
+        if (ns < 0) return -1;
+        const int64_t r = (int64_t)__ldg(a.node_offsets + n) + ns;
+        return (r >= 0 && r < a.src_rows) ? r : -2;
+    };
+    auto issue = [&](int64_t q) {
+        const int s = (int)(q % kDispStages);
+        int64_t row, base;
+        uint32_t bytes;
+        const int64_t src_row = source(first + q, row, base, bytes);
+        if (lane == 0) {
+            if (src_row >= 0) {
+                mbar_arrive_expect_tx(&full[s], bytes);
+                bulk_load(stage0 + (size_t)s * a.chunk, a.src + src_row * a.row_bytes + base, bytes, &full[s]);
+            } else {
+                mbar_arrive_expect_tx(&full[s], 0);  // empty item: complete the phase
+            }
+        }
+    };
+
+    uint32_t parity = 0, inflight = 0;
+    for (int64_t q = 0; q < kDispStages && q < mine; ++q) {
+        issue(q);
+        inflight |= 1u << q;
+    }
+    if (early) pdl_wait();
+    for (int64_t q = 0; q < mine; ++q) {
+        const int s = (int)(q % kDispStages);
+        const bool ok = __all_sync(kFullMask, mbar_wait(&full[s], (parity >> s) & 1u));
+        if (!ok) {
+            errbits |= kErrTimeout;
+            drain(full, parity, inflight, kDispStages);
+            break;
+        }
+        parity ^= 1u << s;
+        inflight &= ~(1u << s);
+        int64_t row, base;
+        uint32_t bytes;
+        const int64_t src_row = source(first + q, row, base, bytes);
+        if (src_row == -2) errbits |= kErrBadLayout;
+        int64_t dst = -1;
+        if (src_row >= 0) {
+            if (MODE == kFlat) {
+                if (lane < a.k) {
+                    const int sl = __ldg(a.slot + row * a.k + lane);
+                    if (sl >= 0 && sl < a.dst_rows) dst = sl;
+                    else if (sl != -1) errbits |= kErrBadLayout;
+                }
+            } else if (MODE == kNodePack) {
+                if (lane < a.N) {
+                    const int ns = __ldg(a.node_slot + row * a.N + lane);
+                    if (ns >= 0) {
+                        const int64_t d = (int64_t)__ldg(a.node_offsets + lane) + ns;
+                        if (d >= 0 && d < a.dst_rows) dst = d;
+                        else errbits |= kErrBadLayout;
+                    }
+                }
+            } else {
+                const int n = (int)(row / a.T);
+                const int64_t t = row - (int64_t)n * a.T;
+                const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
+                const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
+                if (lane < a.k) {
+                    const int sl = __ldg(a.slot + t * a.k + lane);
+                    if (sl >= lo && sl < hi && sl < a.dst_rows) dst = sl;
+                }
+            }
+        }
+        if (dst >= 0) bulk_store(a.dst + dst * a.row_bytes + base, stage0 + (size_t)s * a.chunk, bytes);
+        bulk_commit();
+        // the stage of item q-1 is free once its stores have read it
+        bulk_wait_read<1>();
+        __syncwarp();
+        if (q >= 1 && q - 1 + kDispStages < mine) {
+            issue(q - 1 + kDispStages);
+            inflight |= 1u << ((q - 1) % kDispStages);
+        }
+    }
+    bulk_wait_all();
+    warp_report(a.err, errbits);
+}
+
+__global__ void __launch_bounds__(kBulkThreads) combine_bulk_kernel(BulkArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t stage_bytes = (size_t)a.k * a.chunk;
+    unsigned char* stage0 = smem + (size_t)warp * kCombStages * stage_bytes;
+    uint64_t* full =
+        reinterpret_cast<uint64_t*>(smem + (size_t)kBulkWarps * kCombStages * stage_bytes) + warp * kCombStages;
+    if (lane == 0) {
+        for (int s = 0; s < kCombStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    pdl_trigger();
+    pdl_wait();
+
+    const int64_t items = a.T * a.cpr;
+    // a contiguous, row-major range of items per warp
+    const int64_t nwarps = (int64_t)gridDim.x * kBulkWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kBulkWarps + warp;
+    const int64_t first = items * gw / nwarps;
+    const int64_t mine = items * (gw + 1) / nwarps - first;
+    const int64_t eo_rows = a.T * a.k;
+    int errbits = 0;
+
+    auto geometry = [&](int64_t item, int64_t& t, int64_t& base, uint32_t& bytes) {
+        t = item / a.cpr;
+        base = (item - t * a.cpr) * (int64_t)a.chunk;
+        const int64_t left = a.row_bytes - base;
+        bytes = left < (int64_t)a.chunk ? (uint32_t)left : a.chunk;
+    };
+    // lane j < k: expert row of (t, j), or -1
+    auto row_of = [&](int64_t t) -> int {
+        int s = -1;
+        if (lane < a.k) {
+            s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
+            if (s < 0 || s >= eo_rows) {
+                if (s != -1) errbits |= kErrBadLayout;
+                s = -1;
+            }
+        }
+        return s;
+    };
+    auto issue = [&](int64_t q) {
+        const int st = (int)(q % kCombStages);
+        int64_t t, base;
+        uint32_t bytes;
+        geometry(first + q, t, base, bytes);
+        const int s = row_of(t);
+        const unsigned valid = __ballot_sync(kFullMask, s >= 0);
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes * (uint32_t)__popc(valid));
+        __syncwarp();
+        if (s >= 0)
+            bulk_load(stage0 + (size_t)st * stage_bytes + (size_t)lane * a.chunk,
+                      a.src + (int64_t)s * a.row_bytes + base, bytes, &full[st]);
+    };
+
+    uint32_t parity = 0, inflight = 0;
+    for (int64_t q = 0; q < kCombStages && q < mine; ++q) {
+        issue(q);
+        inflight |= 1u << q;
+    }
+    for (int64_t q = 0; q < mine; ++q) {
+        const int st = (int)(q % kCombStages);
+        const bool ok = __all_sync(kFullMask, mbar_wait(&full[st], (parity >> st) & 1u));
+        if (!ok) {
+            errbits |= kErrTimeout;
+            drain(full, parity, inflight, kCombStages);
+            break;
+        }
+        parity ^= 1u << st;
+        inflight &= ~(1u << st);
+        int64_t t, base;
+        uint32_t bytes;
+        geometry(first + q, t, base, bytes);
+        const int s = row_of(t);
+        const unsigned valid = __ballot_sync(kFullMask, s >= 0);
+        const float wl = lane < a.k ? __ldg(a.w + t * a.k + lane) : 0.f;
+        const unsigned char* stage = stage0 + (size_t)st * stage_bytes;
+        char* yrow = a.dst + t * a.row_bytes + base;
+        const int nvec = (int)(bytes >> 4);
+        // every lane runs every pass (the weight shuffles need the whole warp)
+        for (int v0 = 0; v0 < nvec; v0 += 32) {
+            const int v = v0 + lane;
+            const bool active = v < nvec;
+            float acc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+            for (int j = 0; j < a.k; ++j) {
+                const float wj = __shfl_sync(kFullMask, wl, j);
+                if (!active || !((valid >> j) & 1u)) continue;
+                const uint4 x = *reinterpret_cast<const uint4*>(stage + (size_t)j * a.chunk + (size_t)v * 16);
+                float f[8];
+                unpack_bf16<uint4>(x, f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(wj, f[e], acc[e]);
+            }
+            if (active) *reinterpret_cast<uint4*>(yrow + (size_t)v * 16) = pack_bf16<uint4>(acc);
+        }
+        __syncwarp();
+        if (q + kCombStages < mine) {
+            if (lane == 0) fence_proxy_async_smem();
+            __syncwarp();
+            issue(q + kCombStages);
+            inflight |= 1u << st;
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+template <auto Kernel>
+cudaError_t launch_bulk(const BulkArgs& a, int64_t items, size_t smem, cudaStream_t stream) {
+    if (items <= 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid<Kernel>(items, kBulkThreads, smem);
+    return launch_pdl(Kernel, dim3(grid), dim3(kBulkThreads), smem, stream, a);
+}
+
+BulkArgs bulk_args(const RowMoveParams& p, const void* src, void* dst, int64_t src_rows,
+                   int64_t dst_rows, uint32_t chunk) {
+    BulkArgs a;
+    a.src = static_cast<const char*>(src);
+    a.dst = static_cast<char*>(dst);
+    a.w = nullptr;
+    a.slot = p.slot;
+    a.node_slot = p.node_slot;
+    a.node_offsets = p.node_offsets;
+    a.rank_offsets = p.rank_offsets;
+    a.T = p.T;
+    a.k = p.k;
+    a.N = p.N;
+    a.ranks_per_node = p.ranks_per_node;
+    a.row_bytes = (int64_t)p.row_bytes;
+    a.chunk = (uint32_t)((int64_t)chunk < a.row_bytes ? chunk : a.row_bytes);
+    a.cpr = (a.row_bytes + a.chunk - 1) / a.chunk;
+    a.src_rows = src_rows;
+    a.dst_rows = dst_rows;
+    a.err = p.err;
+    a.early = p.early_inputs ? 1 : 0;
+    return a;
+}
+
+template <int MODE>
+cudaError_t launch_disp_bulk(const BulkArgs& a, int64_t rows, cudaStream_t stream) {
+    const size_t smem = (size_t)kBulkWarps * kDispStages * (a.chunk + sizeof(uint64_t));
+    return launch_bulk<dispatch_bulk_kernel<MODE>>(a, rows * a.cpr, smem, stream);
+}
+
+}  // namespace
+
+bool bulk_eligible(size_t row_bytes, std::initializer_list<const void*> ptrs) {
+    uintptr_t bits = row_bytes;
+    for (const void* p : ptrs) bits |= reinterpret_cast<uintptr_t>(p);
+    return row_bytes > 0 && bits % 16 == 0;
+}
+
+cudaError_t launch_dispatch_flat_bulk(const RowMoveParams& p, const void* x, void* recv,
+                                      cudaStream_t stream) {
+    const BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kDispChunk);
+    return launch_disp_bulk<kFlat>(a, p.T, stream);
+}
+
+cudaError_t launch_node_pack_bulk(const RowMoveParams& p, const void* x, void* staging,
+                                  int64_t staging_rows, cudaStream_t stream) {
+    const BulkArgs a = bulk_args(p, x, staging, p.T, staging_rows, kDispChunk);
+    return launch_disp_bulk<kNodePack>(a, p.T, stream);
+}
+
+cudaError_t launch_node_expand_bulk(const RowMoveParams& p, const void* staging,
+                                    int64_t staging_rows, void* recv, cudaStream_t stream) {
+    const BulkArgs a = bulk_args(p, staging, recv, staging_rows, p.T * p.k, kDispChunk);
+    return launch_disp_bulk<kNodeExpand>(a, p.T * p.N, stream);
+}
+
+cudaError_t launch_combine_bulk(const CombineParams& p, const void* expert_out, void* y,
+                                cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    RowMoveParams rp = {};
+    rp.T = p.T;
+    rp.k = p.k;
+    rp.row_bytes = p.row_bytes;
+    rp.slot = p.slot;
+    rp.err = p.err;
+    uint32_t chunk = (kCombStageBytes / (uint32_t)p.k) & ~15u;
+    if (chunk < 16) chunk = 16;
+    BulkArgs a = bulk_args(rp, expert_out, y, p.T * p.k, p.T, chunk);
+    a.w = p.w;
+    const size_t smem = (size_t)kBulkWarps * kCombStages * ((size_t)a.k * a.chunk + sizeof(uint64_t));
+    return launch_bulk<combine_bulk_kernel>(a, p.T * a.cpr, smem, stream);
+}
+
+}  // namespace moe

@@ -8,7 +8,8 @@ namespace {
 
 using moe::CopyEngine;
 
-constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK;
+constexpr uint32_t kKnownFlags =
+    MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK | MOE_FLAG_LAYOUT_CLUSTER;
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -51,6 +52,32 @@ moe::RowMoveParams move_params(const moe_config_t* c, const moe_layout_t* L) {
     p.err = L->error_word;
     p.engine = engine_of(c->flags);
     return p;
+}
+
+moe_status_t check_dispatch_args(const moe_config_t* c, const moe_layout_t* L, const void* x,
+                                 const void* recv, const void* node_staging) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || recv == nullptr) return MOE_ERR_INVALID_ARG;
+    if (two_level(c) && node_staging == nullptr) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// early: the layout kernels were enqueued right before on this stream by
+// this library and x was complete when they started.
+moe_status_t dispatch_impl(const moe_config_t* c, const moe_layout_t* L, const void* x, void* recv,
+                           void* node_staging, cudaStream_t s, bool early) {
+    moe::RowMoveParams p = move_params(c, L);
+    p.early_inputs = early;
+    if (!two_level(c)) return cuda_status(moe::launch_dispatch_flat(p, x, recv, s));
+    const int64_t rows = staging_rows(c);
+    cudaError_t e = moe::launch_node_pack(p, x, node_staging, rows, s);
+    p.early_inputs = false;  // expansion reads staging written by the pack
+    if (e == cudaSuccess) e = moe::launch_node_expand(p, node_staging, rows, recv, s);
+    return cuda_status(e);
 }
 
 }  // namespace
@@ -132,6 +159,7 @@ moe_status_t moe_layout(const moe_config_t* c, const int32_t* topk_idx, const mo
     p.R = c->num_ranks;
     p.N = c->num_nodes;
     p.nodes = two_level(c);
+    p.cluster = (c->flags & MOE_FLAG_LAYOUT_CLUSTER) != 0;
     p.topk = topk_idx;
     p.expert_counts = L->expert_counts;
     p.expert_offsets = L->expert_offsets;
@@ -147,20 +175,19 @@ moe_status_t moe_layout(const moe_config_t* c, const int32_t* topk_idx, const mo
 
 moe_status_t moe_dispatch(const moe_config_t* c, const moe_layout_t* L, const void* x, void* recv,
                           void* node_staging, void* stream) {
-    moe_status_t st = moe_check_config(c);
+    const moe_status_t st = check_dispatch_args(c, L, x, recv, node_staging);
+    if (st != MOE_OK || c->num_tokens == 0) return st;
+    return dispatch_impl(c, L, x, recv, node_staging, static_cast<cudaStream_t>(stream), false);
+}
+
+moe_status_t moe_layout_dispatch(const moe_config_t* c, const int32_t* topk_idx,
+                                 const moe_layout_t* L, const void* x, void* recv,
+                                 void* node_staging, void* stream) {
+    moe_status_t st = check_dispatch_args(c, L, x, recv, node_staging);
     if (st != MOE_OK) return st;
-    st = check_layout_ptrs(c, L);
-    if (st != MOE_OK) return st;
-    if (c->num_tokens == 0) return MOE_OK;
-    if (x == nullptr || recv == nullptr) return MOE_ERR_INVALID_ARG;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const moe::RowMoveParams p = move_params(c, L);
-    if (!two_level(c)) return cuda_status(moe::launch_dispatch_flat(p, x, recv, s));
-    if (node_staging == nullptr) return MOE_ERR_INVALID_ARG;
-    const int64_t rows = staging_rows(c);
-    cudaError_t e = moe::launch_node_pack(p, x, node_staging, rows, s);
-    if (e == cudaSuccess) e = moe::launch_node_expand(p, node_staging, rows, recv, s);
-    return cuda_status(e);
+    st = moe_layout(c, topk_idx, L, stream);
+    if (st != MOE_OK || c->num_tokens == 0) return st;
+    return dispatch_impl(c, L, x, recv, node_staging, static_cast<cudaStream_t>(stream), true);
 }
 
 moe_status_t moe_combine(const moe_config_t* c, const moe_layout_t* L, const void* expert_out,

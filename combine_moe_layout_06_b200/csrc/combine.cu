@@ -12,10 +12,12 @@
 // rounds to nearest even.
 //
 // Work items are (token, row chunk) pairs, a chunk being 32*VPL vectors of
-// the row, handed out warp by warp over a persistent grid sized to what is
-// resident, so every SM stays busy to the end.  Lanes hold the token's k
-// slots and weights; the chunk of up to KB expert rows is loaded before any
-// FMA, so KB*VPL streaming loads per lane are in flight at once.
+// the row, over a persistent grid sized to what is resident; each warp takes
+// a contiguous token-major range of items, so a token's k slots and weights
+// (held one per lane) are loaded once, and the next token's are fetched
+// while the current chunk's rows are in flight.  The chunk of up to KB
+// expert rows is loaded before any FMA, so KB*VPL streaming loads per lane
+// are in flight at once.
 #include "moe_kernels.h"
 
 namespace moe {
@@ -23,6 +25,15 @@ namespace {
 
 constexpr int kWarpsPerCta = 8;
 constexpr int kThreads = kWarpsPerCta * 32;
+
+// 16-byte vectors per lane in one row chunk (1 KB chunks) and expert rows
+// loaded per batch; compile-time tunables.
+#ifndef MOE_COMBINE_VPL
+#define MOE_COMBINE_VPL 2
+#endif
+#ifndef MOE_COMBINE_KB
+#define MOE_COMBINE_KB 8
+#endif
 
 struct CombArgs {
     const void* eo;
@@ -36,77 +47,93 @@ struct CombArgs {
     int* err;
 };
 
+// Lane j < k: expert row and gate weight of (t, j); row -1 when invalid.
+__device__ __forceinline__ void load_route(const CombArgs& a, int64_t t, int lane, int& s, float& w,
+                                           int& bad) {
+    s = -1;
+    w = 0.f;
+    if (lane < a.k) {
+        s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
+        w = __ldg(a.w + t * a.k + lane);
+    }
+    const bool ok = s >= 0 && s < a.eo_rows;
+    bad |= (!ok && s != -1) ? kErrBadLayout : 0;
+    s = ok ? s : -1;
+}
+
 template <typename V, int VPL, int KB>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     constexpr int EPV = VecInfo<V>::kElems;
     constexpr int CHUNK = 32 * VPL;
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = a.T * cpr;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
     const V* eo = static_cast<const V*>(a.eo);
     V* y = static_cast<V*>(a.y);
     int errbits = 0;
-    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
-         item += nwarps) {
-        const int64_t t = item / cpr;
-        const int64_t base = (item - t * cpr) * CHUNK;
-        int s = -1;
-        float wl = 0.f;
-        if (lane < a.k) {
-            s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
-            wl = __ldg(a.w + t * a.k + lane);
-            if (s < 0 || s >= a.eo_rows) {
-                if (s != -1) errbits |= kErrBadLayout;
-                s = -1;
-            }
-        }
-        float acc[VPL][EPV];
+    if (ib < ie) {
+        int64_t t = ib / cpr;
+        int64_t c = ib - t * cpr;
+        int s, s_next = -1;
+        float wl, w_next = 0.f;
+        load_route(a, t, lane, s, wl, errbits);
+        for (int64_t item = ib; item < ie; ++item) {
+            const bool last_chunk = c + 1 == cpr;
+            if (last_chunk && item + 1 < ie) load_route(a, t + 1, lane, s_next, w_next, errbits);
+            const int64_t base = c * CHUNK;
+            float acc[VPL][EPV];
 #pragma unroll
-        for (int i = 0; i < VPL; ++i)
+            for (int i = 0; i < VPL; ++i)
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) acc[i][e] = 0.f;
-        for (int j0 = 0; j0 < a.k; j0 += KB) {
-            V v[KB][VPL];
-            float wq[KB];
-            bool ok[KB];
+                for (int e = 0; e < EPV; ++e) acc[i][e] = 0.f;
+            for (int j0 = 0; j0 < a.k; j0 += KB) {
+                V v[KB][VPL];
+                float wq[KB];
+                bool ok[KB];
 #pragma unroll
-            for (int q = 0; q < KB; ++q) {
-                const int j = j0 + q;
-                const int sj = __shfl_sync(kFullMask, s, j & 31);
-                wq[q] = __shfl_sync(kFullMask, wl, j & 31);
-                ok[q] = j < a.k && sj >= 0;
-                if (ok[q]) {
-                    const V* row = eo + (int64_t)sj * a.rv + base;
+                for (int q = 0; q < KB; ++q) {
+                    const int j = j0 + q;
+                    const int sj = __shfl_sync(kFullMask, s, j & 31);
+                    wq[q] = __shfl_sync(kFullMask, wl, j & 31);
+                    ok[q] = j < a.k && sj >= 0;
+                    if (ok[q]) {
+                        const V* row = eo + (int64_t)sj * a.rv + base;
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i)
+                            if (base + i * 32 + lane < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < KB; ++q) {
+                    if (!ok[q]) continue;
 #pragma unroll
                     for (int i = 0; i < VPL; ++i) {
-                        const int64_t idx = base + i * 32 + lane;
-                        if (idx < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
+                        if (base + i * 32 + lane < a.rv) {
+                            float f[EPV];
+                            unpack_bf16<V>(v[q][i], f);
+#pragma unroll
+                            for (int e = 0; e < EPV; ++e) acc[i][e] = __fmaf_rn(wq[q], f[e], acc[i][e]);
+                        }
                     }
                 }
             }
+            V* yrow = y + t * a.rv + base;
 #pragma unroll
-            for (int q = 0; q < KB; ++q) {
-                if (!ok[q]) continue;
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int64_t idx = base + i * 32 + lane;
-                    if (idx < a.rv) {
-                        float f[EPV];
-                        unpack_bf16<V>(v[q][i], f);
-#pragma unroll
-                        for (int e = 0; e < EPV; ++e) acc[i][e] = __fmaf_rn(wq[q], f[e], acc[i][e]);
-                    }
-                }
+            for (int i = 0; i < VPL; ++i)
+                if (base + i * 32 + lane < a.rv) yrow[i * 32 + lane] = pack_bf16<V>(acc[i]);
+            if (last_chunk) {
+                s = s_next;
+                wl = w_next;
+                ++t;
+                c = 0;
+            } else {
+                ++c;
             }
-        }
-        V* yrow = y + t * a.rv + base;
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int64_t idx = base + i * 32 + lane;
-            if (idx < a.rv) yrow[i * 32 + lane] = pack_bf16<V>(acc[i]);
         }
     }
     warp_report(a.err, errbits);
@@ -122,7 +149,8 @@ cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
 
 template <typename V, int VPL>
 cudaError_t launch_combine_k(CombArgs a, cudaStream_t stream) {
-    return a.k <= 4 ? launch_combine_v<V, VPL, 4>(a, stream) : launch_combine_v<V, VPL, 8>(a, stream);
+    if (a.k <= 4) return launch_combine_v<V, VPL, 4>(a, stream);
+    return launch_combine_v<V, VPL, (MOE_COMBINE_KB > 4 ? MOE_COMBINE_KB : 4)>(a, stream);
 }
 
 inline int vec_bytes(size_t row_bytes, const void* a, const void* b) {
@@ -137,6 +165,9 @@ inline int vec_bytes(size_t row_bytes, const void* a, const void* b) {
 cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void* y,
                            cudaStream_t stream) {
     if (p.T <= 0) return cudaSuccess;
+    // register engine unless the bulk engine is asked for
+    if (p.engine == CopyEngine::kBulk && bulk_eligible(p.row_bytes, {expert_out, y}))
+        return launch_combine_bulk(p, expert_out, y, stream);
     CombArgs a;
     a.eo = expert_out;
     a.w = p.w;
@@ -149,7 +180,7 @@ cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void*
     switch (vec_bytes(p.row_bytes, expert_out, y)) {
         case 16:
             a.rv = (int64_t)(p.row_bytes / 16);
-            return launch_combine_k<uint4, 2>(a, stream);
+            return launch_combine_k<uint4, MOE_COMBINE_VPL>(a, stream);
         case 4:
             a.rv = (int64_t)(p.row_bytes / 4);
             return launch_combine_k<uint32_t, 4>(a, stream);

@@ -58,74 +58,105 @@ struct FanArgs {
 
 // Flat and node-pack rows are tokens; node-expand rows are (node, token)
 // pairs, node-major, so each node's forwarder work is one contiguous run.
+//
+// Where row r's data comes from and goes to: the source row (-1 = nothing to
+// move) and, per lane, one destination row (-1 = none).  Computed without
+// branching on loaded values, so the loads can be issued a row ahead and
+// waited on only when used.
+struct RowPlan {
+    int64_t src;
+    int64_t dst;
+    int bad;
+};
+
+template <int MODE>
+__device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int lane) {
+    RowPlan p;
+    p.dst = -1;
+    p.bad = 0;
+    if (MODE == kFlat) {
+        p.src = row;
+        const int s = lane < a.k ? __ldg(a.slot + row * a.k + lane) : -1;
+        const bool ok = s >= 0 && s < a.dst_rows;
+        p.dst = ok ? s : -1;
+        p.bad = (!ok && s != -1) ? kErrBadLayout : 0;
+    } else if (MODE == kNodePack) {
+        p.src = row;
+        const int ns = lane < a.N ? __ldg(a.node_slot + row * a.N + lane) : -1;
+        const int64_t off = lane < a.N ? (int64_t)__ldg(a.node_offsets + lane) : 0;
+        const int64_t d = off + ns;
+        const bool ok = ns >= 0 && d >= 0 && d < a.dst_rows;
+        p.dst = ok ? d : -1;
+        p.bad = (ns >= 0 && !ok) ? kErrBadLayout : 0;
+    } else {
+        const int n = (int)(row / a.T);
+        const int64_t t = row - (int64_t)n * a.T;
+        const int ns = __ldg(a.node_slot + t * a.N + n);  // same for all lanes
+        const int64_t srow = (int64_t)__ldg(a.node_offsets + n) + ns;
+        const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
+        const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
+        const int s = lane < a.k ? __ldg(a.slot + t * a.k + lane) : -1;
+        const bool src_ok = ns >= 0 && srow >= 0 && srow < a.src_rows;
+        p.src = src_ok ? srow : -1;
+        p.bad = (ns >= 0 && !src_ok) ? kErrBadLayout : 0;
+        p.dst = (src_ok && s >= lo && s < hi && s < a.dst_rows) ? s : -1;
+    }
+    return p;
+}
+
+// Each warp moves a contiguous, row-major range of (row, chunk) items, so a
+// row's plan is loaded once and the next row's plan is fetched while the
+// current chunk's loads and stores are in flight.
 template <int MODE, typename V, int VPL>
 __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
     constexpr int CHUNK = 32 * VPL;
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = rows * cpr;
-    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
     int errbits = 0;
-    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
-         item += nwarps) {
-        const int64_t row = item / cpr;
-        const int64_t base = (item - row * cpr) * CHUNK;
-        int64_t src_row;
-        int64_t dst = -1;
-        if (MODE == kFlat) {
-            src_row = row;
-            if (lane < a.k) {
-                const int s = __ldg(a.slot + row * a.k + lane);
-                if (s >= 0 && s < a.dst_rows) dst = s;
-                else if (s != -1) errbits |= kErrBadLayout;
-            }
-        } else if (MODE == kNodePack) {
-            src_row = row;
-            if (lane < a.N) {
-                const int ns = __ldg(a.node_slot + row * a.N + lane);
-                if (ns >= 0) {
-                    const int64_t d = (int64_t)__ldg(a.node_offsets + lane) + ns;
-                    if (d >= 0 && d < a.dst_rows) dst = d;
-                    else errbits |= kErrBadLayout;
+    if (ib < ie) {
+        int64_t row = ib / cpr;
+        int64_t c = ib - row * cpr;
+        RowPlan cur = plan_row<MODE>(a, row, lane);
+        RowPlan nxt = cur;
+        for (int64_t item = ib; item < ie; ++item) {
+            const bool last_chunk = c + 1 == cpr;
+            if (last_chunk && item + 1 < ie) nxt = plan_row<MODE>(a, row + 1, lane);
+            if (cur.src >= 0) {
+                const int64_t base = c * CHUNK;
+                const V* src = static_cast<const V*>(a.src) + cur.src * a.rv + base;
+                V v[VPL];
+#pragma unroll
+                for (int i = 0; i < VPL; ++i)
+                    if (base + i * 32 + lane < a.rv) v[i] = ld_stream(src + i * 32 + lane);
+                unsigned m = __ballot_sync(kFullMask, cur.dst >= 0);
+                V* dbase = static_cast<V*>(a.dst) + base;
+                while (m) {
+                    const int j = __ffs(m) - 1;
+                    m &= m - 1;
+                    const int64_t d = __shfl_sync(kFullMask, cur.dst, j);
+                    V* drow = dbase + d * a.rv;
+#pragma unroll
+                    for (int i = 0; i < VPL; ++i)
+                        if (base + i * 32 + lane < a.rv) st_stream(drow + i * 32 + lane, v[i]);
                 }
             }
-        } else {
-            const int n = (int)(row / a.T);
-            const int64_t t = row - (int64_t)n * a.T;
-            const int ns = __ldg(a.node_slot + t * a.N + n);  // same for all lanes
-            if (ns < 0) continue;
-            src_row = (int64_t)__ldg(a.node_offsets + n) + ns;
-            if (src_row < 0 || src_row >= a.src_rows) {
-                errbits |= kErrBadLayout;
-                continue;
-            }
-            const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
-            const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
-            if (lane < a.k) {
-                const int s = __ldg(a.slot + t * a.k + lane);
-                if (s >= lo && s < hi && s < a.dst_rows) dst = s;
+            if (last_chunk) {
+                errbits |= cur.bad;
+                cur = nxt;
+                ++row;
+                c = 0;
+            } else {
+                ++c;
             }
         }
-        const unsigned dmask = __ballot_sync(kFullMask, dst >= 0);
-        const V* src = static_cast<const V*>(a.src) + src_row * a.rv + base;
-        V* dbase = static_cast<V*>(a.dst) + base;
-        V v[VPL];
-#pragma unroll
-        for (int i = 0; i < VPL; ++i)
-            if (base + i * 32 + lane < a.rv) v[i] = ld_stream(src + i * 32 + lane);
-        unsigned m = dmask;
-        while (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1;
-            const int64_t d = __shfl_sync(kFullMask, dst, j);
-            V* drow = dbase + d * a.rv;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i)
-                if (base + i * 32 + lane < a.rv) st_stream(drow + i * 32 + lane, v[i]);
-        }
+        if (c != 0) errbits |= cur.bad;
     }
     warp_report(a.err, errbits);
 }
@@ -135,15 +166,16 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
 template <typename V, int VPL>
 __global__ void __launch_bounds__(kThreads) gather_kernel(FanArgs a) {
     constexpr int CHUNK = 32 * VPL;
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = a.T * a.k * cpr;
-    const int64_t nwarps = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
     int errbits = 0;
-    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items;
-         item += nwarps) {
+    for (int64_t item = ib; item < ie; ++item) {
         const int64_t drow = item / cpr;
         const int64_t base = (item - drow * cpr) * CHUNK;
         const int s = __ldg(a.slot + drow);   // same for all lanes
@@ -170,8 +202,8 @@ template <typename V>
 __global__ void __launch_bounds__(kThreads) copy_kernel(const V* __restrict__ src, V* __restrict__ dst,
                                                         const int* rows_dev, int64_t max_rows,
                                                         int64_t rv) {
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     int64_t rows = max_rows;
     if (rows_dev != nullptr) {
         const int64_t r = *rows_dev;
@@ -208,11 +240,17 @@ cudaError_t launch_fan_vpl(FanArgs a, int64_t rows, cudaStream_t stream) {
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
 }
 
+// Vectors per lane in one row chunk (compile-time tunable; 4 = 2 KB chunks
+// of 16-byte vectors).
+#ifndef MOE_DISPATCH_VPL
+#define MOE_DISPATCH_VPL 4
+#endif
+
 template <int MODE, typename V>
 cudaError_t launch_fan_v(FanArgs a, int64_t rows, cudaStream_t stream) {
+    constexpr int VPL = MOE_DISPATCH_VPL;
     a.rv /= sizeof(V);
-    // chunks that tile the row exactly where possible
-    if (a.rv % (32 * 4) == 0 || a.rv > 32 * 4) return launch_fan_vpl<MODE, V, 4>(a, rows, stream);
+    if (a.rv >= 32 * VPL) return launch_fan_vpl<MODE, V, VPL>(a, rows, stream);
     return launch_fan_vpl<MODE, V, 2>(a, rows, stream);
 }
 
@@ -248,20 +286,30 @@ FanArgs fan_args(const RowMoveParams& p, const void* src, void* dst, int64_t src
 
 }  // namespace
 
+// The bulk engine is used unless the register engine is forced or the rows
+// are not 16-byte aligned.
+inline bool use_bulk(const RowMoveParams& p, std::initializer_list<const void*> ptrs) {
+    return p.engine != CopyEngine::kVector && bulk_eligible(p.row_bytes, ptrs);
+}
+
 cudaError_t launch_dispatch_flat(const RowMoveParams& p, const void* x, void* recv,
-                                        cudaStream_t stream) {
+                                 cudaStream_t stream) {
+    if (use_bulk(p, {x, recv})) return launch_dispatch_flat_bulk(p, x, recv, stream);
     FanArgs a = fan_args(p, x, recv, p.T, p.T * p.k);
     return launch_fan<kFlat>(a, p.T, stream);
 }
 
 cudaError_t launch_node_pack(const RowMoveParams& p, const void* x, void* staging,
                              int64_t staging_rows, cudaStream_t stream) {
+    if (use_bulk(p, {x, staging})) return launch_node_pack_bulk(p, x, staging, staging_rows, stream);
     FanArgs a = fan_args(p, x, staging, p.T, staging_rows);
     return launch_fan<kNodePack>(a, p.T, stream);
 }
 
 cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging, int64_t staging_rows,
                                void* recv, cudaStream_t stream) {
+    if (use_bulk(p, {staging, recv}))
+        return launch_node_expand_bulk(p, staging, staging_rows, recv, stream);
     FanArgs a = fan_args(p, staging, recv, staging_rows, p.T * p.k);
     return launch_fan<kNodeExpand>(a, p.T * p.N, stream);
 }

@@ -8,7 +8,25 @@
 // partition of TensorRT-LLM PR #13888, the per-(token, column) receive row
 // ("slot") and, for node staging, per-node token ranks.
 //
-// Three kernels, no global sort and no atomics on positions:
+// With MOE_FLAG_LAYOUT_CLUSTER and up to kClusterMaxTokens tokens, one
+// launch does it all: a thread-block cluster of up to 16 CTAs, each owning a
+// contiguous token range.
+//   phase 1: each CTA builds its expert (and node) histogram in shared memory;
+//   cluster barrier (hardware, barrier.cluster);
+//   phase 2: each CTA reads every peer's histogram through distributed shared
+//            memory: the totals give expert_offsets (a block scan), the peers
+//            of lower rank give this CTA's first row per expert;
+//   cluster barrier (no CTA leaves while a peer may still read its histogram);
+//   phase 3: the CTA ranks its tokens block by block exactly as the assign
+//            kernel below does, carrying the per-expert base from block to
+//            block.
+// No workspace, no global atomics, no spin-waits.  Measured on B200 it is
+// slower inside a CUDA-graph step than the three kernels below, whose launch
+// latencies overlap through programmatic dependent launch, so it is opt-in.
+//
+// By default, count then assign with the scan folded in (up to 256 chunks of
+// 256 tokens), else three kernels; no global sort and no atomics on
+// positions:
 //   count  : one CTA per chunk of 256 tokens builds an expert histogram (and a
 //            node-touch histogram) in shared memory and writes it to the
 //            workspace column of its chunk, cnt[e][chunk].
@@ -16,11 +34,15 @@
 //            chunk-minor order.  Entry (e, c) becomes expert_offsets[e] plus
 //            the rows of expert e in chunks before c, which is exactly where
 //            chunk c's first row of expert e goes.
-//   assign : one CTA per chunk again; per-warp histograms and a scan across
+//   assign : one CTA per chunk again (up to 256 chunks it also does the scan
+//            for itself, reading the whole [E][C] histogram; see
+//            layout_assign_scan_kernel); per-warp histograms and a scan across
 //            the 8 warps give each warp its base, and inside a warp a token's
 //            rank among equal experts is the popcount of the lower lanes in a
 //            shared-memory lane mask for that expert.  Because a token never
 //            names an expert twice, this ordering is by token index.
+#include <cooperative_groups.h>
+
 #include "moe_kernels.h"
 
 namespace moe {
@@ -29,6 +51,8 @@ namespace {
 constexpr int kLayoutWarps = 8;
 constexpr int kTokensPerCta = kLayoutWarps * 32;
 constexpr int kScanThreads = 1024;
+constexpr int64_t kClusterMaxTokens = 131072;
+constexpr int kClusterMinTokensPerCta = 256;
 
 struct LayoutArgs {
     const int* topk;
@@ -178,8 +202,8 @@ __device__ void block_scan_inplace(int* data, int64_t L, int* s_warp, int& total
 
 __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a) {
     __shared__ int s_warp[32];
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     int total = 0;
     block_scan_inplace(a.cnt, (int64_t)a.E * a.C, s_warp, total);
     __syncthreads();
@@ -217,8 +241,8 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs
     int* s_wn = smem + 2 * kLayoutWarps * a.E;                             // [8][N]
     const int words = 2 * kLayoutWarps * a.E + kLayoutWarps * a.N;
     for (int i = threadIdx.x; i < words; i += blockDim.x) smem[i] = 0;
-    pdl_wait();
     pdl_trigger();
+    pdl_wait();
     __syncthreads();
 
     const int warp = threadIdx.x >> 5;
@@ -296,6 +320,356 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs
     }
 }
 
+// In-place exclusive scan of an int array in shared memory (length L) by
+// one block; returns the total.  s_warp holds 32 ints.
+__device__ int smem_exclusive_scan(int* data, int L, int* s_warp) {
+    const int span = (L + blockDim.x - 1) / blockDim.x;
+    const int beg = min(L, (int)threadIdx.x * span);
+    const int end = min(L, beg + span);
+    int sum = 0;
+    for (int i = beg; i < end; ++i) sum += data[i];
+    int total = 0;
+    int run = block_exclusive_scan(sum, s_warp, total);
+    for (int i = beg; i < end; ++i) {
+        const int v = data[i];
+        data[i] = run;
+        run += v;
+    }
+    __syncthreads();
+    return total;
+}
+
+// Assign with the scan folded in (up to kFusedScanMaxChunks chunks): each CTA
+// reads the whole [E][C] histogram the count kernel wrote, so it finds the
+// totals (and from them expert_offsets) and the rows of each expert in
+// earlier chunks itself; CTA 0 also writes the offsets.  One kernel boundary
+// less than count / scan / assign.  The routes are read and counted before
+// waiting for the count kernel: topk_idx was written before the layout
+// began, and the count kernel waits for its writer before it lets this grid
+// launch.  Shared memory (ints): tot[E+N] base[E+N] wcnt[8][E] mask[8][E]
+// wn[8][N].
+constexpr int kFusedScanMaxChunks = 256;
+
+template <int KMAX>
+__global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(LayoutArgs a) {
+    __shared__ int s_warp[32];
+    extern __shared__ int smem[];
+    const int E = a.E, N = a.N, EN = a.E + a.N, C = a.C;
+    int* tot = smem;
+    int* base = tot + EN;
+    int* s_wcnt = base + EN;
+    unsigned* s_mask = reinterpret_cast<unsigned*>(s_wcnt + kLayoutWarps * E);
+    int* s_wn = reinterpret_cast<int*>(s_mask + kLayoutWarps * E);
+    const int words = 2 * kLayoutWarps * E + kLayoutWarps * N;
+    for (int i = threadIdx.x; i < words; i += blockDim.x) s_wcnt[i] = 0;
+    __syncthreads();
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * kTokensPerCta + threadIdx.x;
+    int e[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) e[j] = -1;
+    uint32_t nm = 0;
+    if (t < a.T) {
+        load_route<KMAX>(a.topk, t, a.k, E, e);  // errors were reported by count
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (e[j] >= 0) {
+                atomicAdd(&s_wcnt[warp * E + e[j]], 1);
+                atomicOr(&s_mask[warp * E + e[j]], 1u << lane);
+            }
+        if (a.nodes) {
+            nm = node_mask<KMAX>(a.part, e);
+            uint32_t m = nm;
+            while (m) {
+                const int n = __ffs(m) - 1;
+                m &= m - 1;
+                atomicAdd(&s_wn[warp * N + n], 1);
+            }
+        }
+    }
+    pdl_trigger();
+    pdl_wait();
+
+    // totals and earlier-chunk rows of each expert / node: 4 histogram rows
+    // per warp at a time, up to 8 chunk columns per lane, loads issued
+    // together
+    for (int i0 = warp * 4; i0 < EN; i0 += kLayoutWarps * 4) {
+        int sum[4], pre[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            sum[r] = 0;
+            pre[r] = 0;
+            const int i = i0 + r;
+            if (i < EN) {
+                const int* row = i < E ? a.cnt + (int64_t)i * C : a.ncnt + (int64_t)(i - E) * C;
+#pragma unroll
+                for (int q = 0; q < kFusedScanMaxChunks / 32; ++q) {
+                    const int c = lane + 32 * q;
+                    if (c < C) {
+                        const int v = row[c];
+                        sum[r] += v;
+                        pre[r] += c < (int)blockIdx.x ? v : 0;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                sum[r] += __shfl_xor_sync(kFullMask, sum[r], o);
+                pre[r] += __shfl_xor_sync(kFullMask, pre[r], o);
+            }
+            if (lane == 0 && i0 + r < EN) {
+                tot[i0 + r] = sum[r];
+                base[i0 + r] = pre[r];
+            }
+        }
+    }
+    __syncthreads();
+    const int total = smem_exclusive_scan(tot, E, s_warp);
+    const int ntotal = a.nodes ? smem_exclusive_scan(tot + E, N, s_warp) : 0;
+    if (blockIdx.x == 0) {
+        for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+            const int off = i < E ? tot[i] : total;
+            a.expert_offsets[i] = off;
+            if (i < E) a.expert_counts[i] = (i + 1 < E ? tot[i + 1] : total) - off;
+        }
+        for (int r = threadIdx.x; r <= a.part.R; r += blockDim.x) {
+            const int fe = a.part.first_expert(r);
+            a.rank_offsets[r] = fe < E ? tot[fe] : total;
+        }
+        if (a.nodes) {
+            for (int i = threadIdx.x; i <= N; i += blockDim.x) {
+                const int off = i < N ? tot[E + i] : ntotal;
+                a.node_offsets[i] = off;
+                if (i < N) a.node_counts[i] = (i + 1 < N ? tot[E + i + 1] : ntotal) - off;
+            }
+        }
+    }
+    // per-warp first rows: chunk base, then earlier warps' counts
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        int run = tot[i] + base[i];
+#pragma unroll
+        for (int w = 0; w < kLayoutWarps; ++w) {
+            const int v = s_wcnt[w * E + i];
+            s_wcnt[w * E + i] = run;
+            run += v;
+        }
+    }
+    if (a.nodes) {
+        for (int i = threadIdx.x; i < N; i += blockDim.x) {
+            int run = base[E + i];
+#pragma unroll
+            for (int w = 0; w < kLayoutWarps; ++w) {
+                const int v = s_wn[w * N + i];
+                s_wn[w * N + i] = run;
+                run += v;
+            }
+        }
+    }
+    __syncthreads();
+    const unsigned lt = lanemask_lt();
+    if (t < a.T) {
+        int* out = a.slot + t * a.k;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j < a.k) {
+                int sl = -1;
+                if (e[j] >= 0) {
+                    const int idx = warp * E + e[j];
+                    sl = s_wcnt[idx] + __popc(s_mask[idx] & lt);
+                }
+                out[j] = sl;
+            }
+        }
+    }
+    if (a.nodes) {
+        for (int n = 0; n < N; ++n) {
+            const bool touched = (nm >> n) & 1u;
+            const unsigned b = __ballot_sync(kFullMask, touched);
+            if (t < a.T) a.node_slot[t * N + n] = touched ? s_wn[warp * N + n] + __popc(b & lt) : -1;
+        }
+    }
+}
+
+// Whole layout in one cluster launch (see the file comment).  Shared memory
+// (ints): hist[E+N] | tot[E+N] | base[E+N] | wbase[W][ES] wmask[W][ES] wn[W][N],
+// W = blockDim.x / 32, ES = E rounded to an odd stride (conflict-free columns).
+constexpr int kMaxCluster = 16;
+
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFullMask, v, o);
+        if (lane >= o) v += y;
+    }
+    return v;
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(1024) layout_cluster_kernel(LayoutArgs a, int64_t tokens_per_cta) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ int s_warp[32];
+    extern __shared__ int smem[];
+    const int E = a.E, N = a.N, EN = a.E + a.N;
+    const int ES = (E & 1) ? E : E + 1;
+    const int W = blockDim.x >> 5;
+    int* hist = smem;
+    int* tot = hist + EN;
+    int* base = tot + EN;
+    int* wbase = base + EN;
+    unsigned* wmask = reinterpret_cast<unsigned*>(wbase + W * ES);
+    int* wn = reinterpret_cast<int*>(wmask + W * ES);
+
+    const int rank = (int)cluster.block_rank();
+    const int csize = (int)cluster.num_blocks();
+    const int64_t t0 = min(a.T, (int64_t)rank * tokens_per_cta);
+    const int64_t t1 = min(a.T, t0 + tokens_per_cta);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const unsigned lt = lanemask_lt();
+
+    for (int i = tid; i < EN; i += blockDim.x) hist[i] = 0;
+    pdl_wait();
+    pdl_trigger();
+    __syncthreads();
+
+    // phase 1: histogram of this CTA's tokens (the first pass stays in
+    // registers for phase 3 when k is small)
+    constexpr bool kKeep = KMAX <= 8;
+    int e0[KMAX];
+    uint32_t nm0 = 0;
+    int bits = 0;
+    for (int64_t b0 = t0; b0 < t1; b0 += blockDim.x) {
+        const int64_t t = b0 + tid;
+        int e[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) e[j] = -1;
+        if (t < t1) bits |= load_route<KMAX>(a.topk, t, a.k, E, e);
+        uint32_t nm = a.nodes ? node_mask<KMAX>(a.part, e) : 0u;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= a.k) break;
+            // one atomic per distinct expert among the warp's lanes
+            const unsigned same = __match_any_sync(kFullMask, e[j]);
+            if (e[j] >= 0 && (same & lt) == 0) atomicAdd(&hist[e[j]], __popc(same));
+        }
+        for (int n = 0; n < N; ++n) {
+            const unsigned bal = __ballot_sync(kFullMask, (nm >> n) & 1u);
+            if (lane == 0 && bal) atomicAdd(&hist[E + n], __popc(bal));
+        }
+        if (kKeep && b0 == t0) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) e0[j] = e[j];
+            nm0 = nm;
+        }
+    }
+    warp_report(a.err, bits);
+    cluster.sync();
+
+    // phase 2: totals and this CTA's bases from every peer's histogram
+    for (int i = tid; i < EN; i += blockDim.x) {
+        int v[kMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r)
+            v[r] = r < csize ? cluster.map_shared_rank(hist, r)[i] : 0;
+        int all = 0, before = 0;
+#pragma unroll
+        for (int r = 0; r < kMaxCluster; ++r) {
+            all += v[r];
+            before += r < rank ? v[r] : 0;
+        }
+        tot[i] = all;
+        base[i] = before;
+    }
+    cluster.sync();
+    // counts into hist[] (peers no longer read it), offsets into tot[]
+    for (int i = tid; i < EN; i += blockDim.x) hist[i] = tot[i];
+    __syncthreads();
+    const int total = smem_exclusive_scan(tot, E, s_warp);
+    const int ntotal = a.nodes ? smem_exclusive_scan(tot + E, N, s_warp) : 0;
+    for (int i = tid; i < E; i += blockDim.x) base[i] += tot[i];
+    if (rank == 0) {
+        for (int i = tid; i <= E; i += blockDim.x) {
+            a.expert_offsets[i] = i < E ? tot[i] : total;
+            if (i < E) a.expert_counts[i] = hist[i];
+        }
+        for (int r = tid; r <= a.part.R; r += blockDim.x) {
+            const int fe = a.part.first_expert(r);
+            a.rank_offsets[r] = fe < E ? tot[fe] : total;
+        }
+        if (a.nodes) {
+            for (int i = tid; i <= N; i += blockDim.x) {
+                a.node_offsets[i] = i < N ? tot[E + i] : ntotal;
+                if (i < N) a.node_counts[i] = hist[E + i];
+            }
+        }
+    }
+    __syncthreads();
+
+    // phase 3: stable ranks, one block of blockDim.x tokens at a time.  A
+    // warp's count of expert e is the popcount of its lane mask for e; a scan
+    // of those counts across warps (one warp-shuffle scan per expert) gives
+    // each warp its first row.
+    int* my_base = wbase + warp * ES;
+    unsigned* my_mask = wmask + warp * ES;
+    for (int64_t b0 = t0; b0 < t1; b0 += blockDim.x) {
+        for (int i = lane; i < E; i += 32) my_mask[i] = 0u;
+        __syncwarp();
+        const int64_t t = b0 + tid;
+        int e[KMAX];
+        uint32_t nm;
+        if (kKeep && b0 == t0) {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) e[j] = e0[j];
+            nm = nm0;
+        } else {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) e[j] = -1;
+            if (t < t1) load_route<KMAX>(a.topk, t, a.k, E, e);
+            nm = a.nodes ? node_mask<KMAX>(a.part, e) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+            if (e[j] >= 0) atomicOr(&my_mask[e[j]], 1u << lane);
+        for (int n = 0; n < N; ++n) {
+            const unsigned bal = __ballot_sync(kFullMask, (nm >> n) & 1u);
+            if (lane == 0) wn[warp * N + n] = __popc(bal);
+        }
+        __syncthreads();
+        for (int i = warp; i < EN; i += W) {
+            int v = 0;
+            if (lane < W) v = i < E ? __popc(wmask[lane * ES + i]) : wn[lane * N + (i - E)];
+            const int incl = warp_inclusive_scan(v);
+            const int b = base[i];
+            if (lane < W) {
+                if (i < E) wbase[lane * ES + i] = b + incl - v;
+                else wn[lane * N + (i - E)] = b + incl - v;
+            }
+            if (lane == 31) base[i] = b + incl;
+        }
+        __syncthreads();
+        if (t < t1) {
+            int* out = a.slot + t * a.k;
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j) {
+                if (j < a.k)
+                    out[j] = e[j] >= 0 ? my_base[e[j]] + __popc(my_mask[e[j]] & lt) : -1;
+            }
+        }
+        for (int n = 0; n < N; ++n) {
+            const bool touched = (nm >> n) & 1u;
+            const unsigned bal = __ballot_sync(kFullMask, touched);
+            if (t < t1) a.node_slot[t * N + n] = touched ? wn[warp * N + n] + __popc(bal & lt) : -1;
+        }
+        __syncthreads();
+    }
+}
+
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 template <int KMAX>
@@ -305,6 +679,17 @@ cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t stream) {
         const size_t smem = sizeof(int) * (size_t)(a.E + a.N);
         err = launch_pdl(layout_count_kernel<KMAX>, dim3(a.C), dim3(kTokensPerCta), smem, stream, a);
         if (err != cudaSuccess) return err;
+    }
+    if (a.C > 0 && a.C <= kFusedScanMaxChunks) {
+        const size_t smem =
+            sizeof(int) * (size_t)(2 * (a.E + a.N) + 2 * kLayoutWarps * a.E + kLayoutWarps * a.N);
+        if (smem > 48 * 1024) {
+            err = cudaFuncSetAttribute(layout_assign_scan_kernel<KMAX>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (err != cudaSuccess) return err;
+        }
+        return launch_pdl(layout_assign_scan_kernel<KMAX>, dim3(a.C), dim3(kTokensPerCta), smem,
+                          stream, a);
     }
     err = launch_pdl(layout_scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, a);
     if (err != cudaSuccess) return err;
@@ -318,6 +703,88 @@ cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t stream) {
         err = launch_pdl(layout_assign_kernel<KMAX>, dim3(a.C), dim3(kTokensPerCta), smem, stream, a);
     }
     return err;
+}
+
+// Threads per CTA for the cluster kernel: no more warps than tokens need,
+// and few enough that the per-warp lane masks fit in about 64 KB.
+inline int cluster_threads(int E, int64_t tokens_per_cta) {
+    int w = 8192 / (E > 0 ? E : 1);
+    w = w > 32 ? 32 : (w < 8 ? 8 : w);
+    const int64_t need = (tokens_per_cta + 31) / 32;
+    if (need < w) w = need < 1 ? 1 : (int)need;
+    return w * 32;
+}
+
+inline size_t cluster_smem(int E, int N, int threads) {
+    const int W = threads / 32;
+    const int ES = (E & 1) ? E : E + 1;
+    return sizeof(int) * (size_t)(3 * (E + N) + W * (2 * ES + N));
+}
+
+// Upper bound of cluster_smem() over E <= MOE_MAX_EXPERTS (1024), N <= 32 and
+// the warps cluster_threads() picks: W * 2 * ES <= 16448, W * N <= 1024,
+// 3 * (E + N) <= 3168 ints, i.e. under 83 KB.
+constexpr size_t kClusterSmemBound = 96 * 1024;
+
+// Largest cluster size (16 if the device runs it, else 8) for this kernel.
+template <int KMAX>
+int max_cluster_size(int threads, size_t smem) {
+    static int cached = 0;
+    if (cached == 0) {
+        cached = 8;
+        auto kern = layout_cluster_kernel<KMAX>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(16);
+            cfg.blockDim = dim3(threads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 16;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0)
+                cached = 16;
+        }
+        cudaGetLastError();  // clear a refused probe
+    }
+    return cached;
+}
+
+template <int KMAX>
+cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t stream) {
+    auto kern = layout_cluster_kernel<KMAX>;
+    const int cmax = max_cluster_size<KMAX>(1024, kClusterSmemBound);
+    int64_t csize = (a.T + kClusterMinTokensPerCta - 1) / kClusterMinTokensPerCta;
+    if (csize > cmax) csize = cmax;
+    if (csize < 1) csize = 1;
+    const int64_t per_cta = (a.T + csize - 1) / csize;
+    const int threads = cluster_threads(a.E, per_cta);
+    const size_t smem = cluster_smem(a.E, a.N, threads);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kClusterSmemBound);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)csize);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, a, per_cta);
 }
 
 }  // namespace
@@ -350,6 +817,8 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     a.node_offsets = p.node_offsets;
     a.node_slot = p.node_slot;
     a.err = p.err;
+    if (p.cluster && p.T <= kClusterMaxTokens)
+        return p.k <= 8 ? launch_layout_cluster<8>(a, stream) : launch_layout_cluster<32>(a, stream);
     return p.k <= 8 ? launch_layout_k<8>(a, stream) : launch_layout_k<32>(a, stream);
 }
 

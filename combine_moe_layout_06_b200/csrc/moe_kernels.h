@@ -4,6 +4,8 @@
 
 #include <cuda_runtime.h>
 #include <stddef.h>
+
+#include <initializer_list>
 #include <stdint.h>
 
 #include "moe_common.cuh"
@@ -18,6 +20,7 @@ struct LayoutParams {
     int64_t T;
     int k, E, R, N;
     bool nodes;             // also build node staging maps
+    bool cluster;           // single cluster launch (T <= 131072)
     const int* topk;        // [T*k]
     int* expert_counts;     // [E]
     int* expert_offsets;    // [E+1]
@@ -45,6 +48,10 @@ struct RowMoveParams {
     const int* rank_offsets;  // [R+1]
     int* err;
     CopyEngine engine;
+    // The source rows (x) were complete before the layout began and the
+    // kernel runs right behind the layout kernels: the bulk engine may start
+    // loading source rows before waiting for the layout.
+    bool early_inputs = false;
 };
 
 // recv[slot[t][j]] = x[t]
@@ -76,5 +83,17 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void* y,
                            cudaStream_t stream);
+
+// ---- bulk-copy (TMA) engine (bulk.cu) ------------------------------------------
+// Usable when the row size and every base address are multiples of 16 bytes.
+bool bulk_eligible(size_t row_bytes, std::initializer_list<const void*> ptrs);
+cudaError_t launch_dispatch_flat_bulk(const RowMoveParams& p, const void* x, void* recv,
+                                      cudaStream_t stream);
+cudaError_t launch_node_pack_bulk(const RowMoveParams& p, const void* x, void* staging,
+                                  int64_t staging_rows, cudaStream_t stream);
+cudaError_t launch_node_expand_bulk(const RowMoveParams& p, const void* staging,
+                                    int64_t staging_rows, void* recv, cudaStream_t stream);
+cudaError_t launch_combine_bulk(const CombineParams& p, const void* expert_out, void* y,
+                                cudaStream_t stream);
 
 }  // namespace moe

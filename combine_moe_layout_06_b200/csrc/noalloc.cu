@@ -71,6 +71,7 @@ extern "C" moe_status_t moe_layout_noalloc(const moe_config_t* c, const int32_t*
     p.R = c->num_ranks;
     p.N = c->num_nodes;
     p.nodes = nodes;
+    p.cluster = (c->flags & MOE_FLAG_LAYOUT_CLUSTER) != 0;
     p.topk = topk_idx;
     p.expert_counts = L->expert_counts;
     p.expert_offsets = L->expert_offsets;

@@ -67,6 +67,9 @@ extern "C" {
 #define MOE_FLAG_COPY_VECTOR 0x2u /* force the register (16-byte vector)
                                      copy kernels */
 #define MOE_FLAG_COPY_BULK 0x4u   /* force the bulk-copy (TMA) kernels */
+#define MOE_FLAG_LAYOUT_CLUSTER 0x8u /* layout in one thread-block-cluster
+                                        launch (up to 131072 tokens) instead
+                                        of the count/scan/assign kernels */
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -177,6 +180,18 @@ moe_status_t moe_layout(const moe_config_t *cfg, const int32_t *topk_idx,
 moe_status_t moe_dispatch(const moe_config_t *cfg, const moe_layout_t *layout,
                           const void *x, void *recv, void *node_staging,
                           void *stream);
+
+/* Layout and dispatch in one call, the layout transformation fused with
+ * the data movement (FUSCO article, "FUSCO 的核心创新": the transfer itself
+ * carries where each row comes from and goes to).  Same results as
+ * moe_layout() followed by moe_dispatch() with the same arguments, but the
+ * dispatch kernel starts loading x rows while the layout kernels still run
+ * (bulk-copy engine), because x and topk_idx are known to be complete when
+ * the layout starts.  Arguments as for moe_layout() and moe_dispatch(); all
+ * are checked before anything is enqueued. */
+moe_status_t moe_layout_dispatch(const moe_config_t *cfg, const int32_t *topk_idx,
+                                 const moe_layout_t *layout, const void *x, void *recv,
+                                 void *node_staging, void *stream);
 
 /* Fused combine: y[t] = bf16_rne( sum_{j=0..k-1} w[t][j] * eo[slot[t][j]] ),
  * accumulated in fp32 with one fused multiply-add per j in column order,

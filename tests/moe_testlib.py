@@ -3,7 +3,7 @@ ABI on seeded inputs and bring results back as numpy arrays."""
 import numpy as np
 import torch
 
-from combine_moe_layout_06_b200 import build, buffers, capi
+from combine_moe_layout_06_b200 import build, buffers, capi  # noqa: F401  (buffers re-exported)
 
 _built = False
 

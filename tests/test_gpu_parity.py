@@ -16,6 +16,9 @@ from combine_moe_layout_06_b200 import capi, inputs
 pytestmark = pytest.mark.gpu
 
 TWO = capi.MOE_FLAG_TWO_LEVEL
+VEC = capi.MOE_FLAG_COPY_VECTOR
+BULK = capi.MOE_FLAG_COPY_BULK
+CL = capi.MOE_FLAG_LAYOUT_CLUSTER
 
 SMALL = [
     # T, H, E, k, R, N
@@ -42,10 +45,10 @@ def _small_inputs(T, H, E, k, seed):
 @pytest.mark.parametrize("T,H,E,k,R,N", SMALL)
 def test_layout_small(oracle_mod, T, H, E, k, R, N):
     _, topk, _ = _small_inputs(T, H, E, k, seed=T + E)
-    for flags in (0, TWO):
+    for flags in (0, TWO, CL, TWO | CL):
         cfg = M.cfg_of(T, H, E, k, R, N, flags)
         lay, _ = M.gpu_layout(cfg, topk)
-        ref = oracle_mod.layout(topk, E, R, N, nodes=bool(flags))
+        ref = oracle_mod.layout(topk, E, R, N, nodes=bool(flags & TWO))
         M.assert_layout_equal(lay.host(), ref)
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
@@ -60,12 +63,17 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
     eo = inputs.random_bf16_bits((T * k, H), seed=T * k + H)
     y_ref = oracle_mod.combine(eo, w, ref["slot"])
     x_dev = M.to_dev(x)
-    for flags in (0, TWO):
+    for flags in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK):
         cfg = M.cfg_of(T, H, E, k, R, N, flags)
         lay, _ = M.gpu_layout(cfg, topk)
         recv, staging = M.gpu_dispatch(cfg, lay, x_dev, fill=0x7F81)
         assert np.array_equal(M.bits(recv), recv_ref)
-        if flags:
+        lay2 = M.buffers.DeviceLayout(cfg)
+        recv2 = torch.empty_like(recv)
+        st2 = M.staging_buffer(cfg) if flags & TWO else None
+        capi.moe_layout_dispatch(cfg, torch.from_numpy(topk).cuda(), lay2.struct, x_dev, recv2, st2)
+        assert np.array_equal(M.bits(recv2), recv_ref), "fused layout + dispatch"
+        if flags & TWO:
             U = int(ref["node_offsets"][-1])
             st = M.bits(staging)
             assert np.array_equal(st[:U], staging_ref)
@@ -73,6 +81,24 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
         y = M.gpu_combine(cfg, lay, M.to_dev(eo), w)
         M.assert_combine_close(M.bits(y), y_ref)
         assert np.array_equal(M.bits(y), y_ref), "fixed-order fp32 FMA is bit-exact"
+        assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_large_batch_multi_kernel_layout(oracle_mod):
+    """Above the single-cluster limit (131072 tokens) the layout runs as
+    count / scan / assign kernels over a workspace."""
+    T, H, E, k, R, N = 140001, 8, 64, 4, 8, 2
+    x, topk, w = _small_inputs(T, H, E, k, seed=77)
+    ref = oracle_mod.layout(topk, E, R, N, nodes=True)
+    for flags in (0, TWO):
+        cfg = M.cfg_of(T, H, E, k, R, N, flags)
+        lay, _ = M.gpu_layout(cfg, topk)
+        want = ref if flags else {k_: v for k_, v in ref.items() if not k_.startswith("node")}
+        M.assert_layout_equal(lay.host(), want)
+        recv, _ = M.gpu_dispatch(cfg, lay, M.to_dev(x))
+        assert np.array_equal(M.bits(recv), oracle_mod.dispatch_flat(x, ref["slot"]))
+        y = M.gpu_combine(cfg, lay, recv, w)
+        assert np.array_equal(M.bits(y), oracle_mod.combine(M.bits(recv), w, ref["slot"]))
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
@@ -152,6 +178,14 @@ def test_workload_layout_dispatch(oracle_mod, name):
         want = ref if two else {k_: v for k_, v in ref.items() if not k_.startswith("node")}
         M.assert_layout_equal(got, want)
         recv, staging = M.gpu_dispatch(cfg, lay, x_dev)
+        # the fused entry point gives the same layout and rows
+        lay2 = M.buffers.DeviceLayout(cfg)
+        recv2 = torch.empty_like(recv)
+        st2 = M.staging_buffer(cfg) if two else None
+        capi.moe_layout_dispatch(cfg, torch.from_numpy(topk).cuda(), lay2.struct, x_dev, recv2, st2)
+        M.assert_layout_equal(lay2.host(), want)
+        assert torch.equal(recv2.view(torch.int16), recv.view(torch.int16))
+        del recv2, st2
         # every receive row equals its token's row (full check on the device)
         slot_dev = torch.from_numpy(ref["slot"].reshape(-1).astype(np.int64)).cuda()
         tok_dev = torch.arange(wl.T, device="cuda").repeat_interleave(wl.k)
@@ -169,6 +203,41 @@ def test_workload_layout_dispatch(oracle_mod, name):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
         del recv, staging
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("engine", [VEC, BULK], ids=["register", "bulk"])
+@pytest.mark.parametrize("name", ["olmoe", "dsv3", "longctx"])
+def test_workload_forced_engine(oracle_mod, name, engine):
+    """Each copy engine, forced, on the full workloads."""
+    d = inputs.make(name)
+    wl = d["workload"]
+    x, topk, w = d["x"], d["topk_idx"], d["topk_w"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, (TWO if wl.two_level else 0) | engine)
+    lay, _ = M.gpu_layout(cfg, topk)
+    x_dev = M.to_dev(x)
+    recv, _ = M.gpu_dispatch(cfg, lay, x_dev)
+    slot_dev = torch.from_numpy(ref["slot"].reshape(-1).astype(np.int64)).cuda()
+    tok_dev = torch.arange(wl.T, device="cuda").repeat_interleave(wl.k)
+    assert torch.equal(recv.view(torch.int16)[slot_dev], x_dev.view(torch.int16)[tok_dev])
+    del slot_dev, tok_dev
+    eo = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 9)
+    y = M.bits(M.gpu_combine(cfg, lay, M.to_dev(eo), w))
+    assert np.array_equal(y, oracle_mod.combine(eo, w, ref["slot"]))
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_workload_layout_cluster(oracle_mod, name):
+    """The single-cluster layout kernel against the oracle at full size."""
+    d = inputs.make(name)
+    wl = d["workload"]
+    topk = d["topk_idx"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, TWO | CL)
+    lay, _ = M.gpu_layout(cfg, topk)
+    M.assert_layout_equal(lay.host(), ref)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
 @pytest.mark.parametrize("name", NAMES)

@@ -49,6 +49,14 @@ def test_noalloc_layout_matches_allocating_layout_twice():
         assert got.keys() == ref.keys()
         for key in ref:
             assert np.array_equal(got[key], ref[key]), (name, key)
+    # a batch above the single-cluster limit, whose layout uses the scratch
+    big = inputs.make_random(140001, 8, 64, 4, seed=5)
+    cfg = capi.config(140001, 8, 64, 4, 8, 2, TWO)
+    assert capi.moe_layout_workspace_bytes(cfg) <= capi.MOE_LAYOUT_NOALLOC_SCRATCH_BYTES
+    for _ in range(2):
+        got, ref = _both(cfg, big["topk_idx"])
+        for key in ref:
+            assert np.array_equal(got[key], ref[key]), ("big", key)
     # and the same small problem twice in a row
     small = inputs.make_random(1000, 8, 60, 4, seed=3)
     cfg = capi.config(1000, 8, 60, 4, 7, 7, TWO)
