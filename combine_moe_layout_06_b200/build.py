@@ -5,7 +5,9 @@ B200 (sm_100a) with nvcc, in-tree next to this file.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -44,16 +46,30 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose_ptxas: bool = False, out: str | None = None,
           defines: tuple = ()) -> str:
     """Compile the library (to `out` instead of the in-tree path when given,
-    with extra -D `defines` for the compile-time tunables)."""
+    with extra -D `defines` for the compile-time tunables).  Each source is
+    compiled to an object in parallel, then the objects are linked."""
     target = out or LIB
     if out is None and not defines and not force and up_to_date():
         return LIB
-    tmp = target + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC, "-o", tmp,
-           *sources()]
+    tag = hashlib.sha1(" ".join(defines).encode()).hexdigest()[:8]
+    objdir = os.path.join(PKG, "_build", tag)
+    os.makedirs(objdir, exist_ok=True)
+    base = [NVCC, *FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC]
     if verbose_ptxas:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+        base.insert(1, "-Xptxas=-v")
+    objs = []
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [c for c in base if c != "-shared"] + ["-c", "-o", obj, src]
+        subprocess.run(cmd, check=True)
+        return obj
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, sources()))
+    tmp = target + f".tmp{os.getpid()}"
+    subprocess.run([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart",
+                    "static", "-o", tmp, *objs], check=True)
     os.replace(tmp, target)
     return target
 

@@ -76,12 +76,16 @@ struct LayoutArgs {
 // Load token t's k expert ids.  Invalid entries become -1 and set error
 // bits: an id outside [0, E), or a repeat of an id earlier in the row (the
 // later copy is dropped).  Count and assign use the same rule, so the
-// histogram and the ranks always agree even on bad input.
+// histogram and the ranks always agree even on bad input.  Repeats are found
+// with a 64-bit mask of ids seen so far (id mod 64); only when the mask hits
+// are the earlier raw entries re-read (from cache) to confirm, which is exact
+// because a valid id equal to an earlier raw id is a repeat.
 template <int KMAX>
 __device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t t, int k, int E,
                                           int (&e)[KMAX]) {
     int bits = 0;
     const int* row = topk + t * k;
+    uint64_t seen = 0;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
         int v = -1;
@@ -90,19 +94,21 @@ __device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t 
             if (v < 0 || v >= E) {
                 bits |= kErrExpertOob;
                 v = -1;
+            } else {
+                const uint64_t bit = 1ull << (v & 63);
+                if (seen & bit) {
+                    bool repeat = false;
+#pragma unroll 1
+                    for (int i = 0; i < j; ++i) repeat |= __ldg(row + i) == v;
+                    if (repeat) {
+                        bits |= kErrDupExpert;
+                        v = -1;
+                    }
+                }
+                seen |= bit;
             }
         }
         e[j] = v;
-    }
-#pragma unroll
-    for (int j = 1; j < KMAX; ++j) {
-#pragma unroll
-        for (int i = 0; i < j; ++i) {
-            if (e[j] >= 0 && e[i] == e[j]) {
-                bits |= kErrDupExpert;
-                e[j] = -1;
-            }
-        }
     }
     return bits;
 }
@@ -346,8 +352,8 @@ __device__ int smem_exclusive_scan(int* data, int L, int* s_warp) {
 // less than count / scan / assign.  The routes are read and counted before
 // waiting for the count kernel: topk_idx was written before the layout
 // began, and the count kernel waits for its writer before it lets this grid
-// launch.  Shared memory (ints): tot[E+N] base[E+N] wcnt[8][E] mask[8][E]
-// wn[8][N].
+// launch.  It lets its dependent grid launch only after the histogram reads.
+// Shared memory (ints): tot[E+N] base[E+N] wcnt[8][E] mask[8][E] wn[8][N].
 constexpr int kFusedScanMaxChunks = 256;
 
 template <int KMAX>
@@ -389,46 +395,83 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
             }
         }
     }
-    pdl_trigger();
     pdl_wait();
 
-    // totals and earlier-chunk rows of each expert / node: 4 histogram rows
-    // per warp at a time, up to 8 chunk columns per lane, loads issued
-    // together
-    for (int i0 = warp * 4; i0 < EN; i0 += kLayoutWarps * 4) {
-        int sum[4], pre[4];
+    // totals and earlier-chunk rows of each expert / node.  Each round of
+    // loads costs an L2 round trip, so the shape of the read follows C:
+    //  - C <= 32: the [E+N][C] histogram is walked column-major (neighbouring
+    //    threads on different rows, so their shared-memory adds do not
+    //    collide), eight loads per thread in flight -- one round for E*C up
+    //    to 2048;
+    //  - larger C: four rows per warp, each lane summing up to 8 columns of
+    //    a row and a warp reduction per row -- two rounds for E up to 64.
+    for (int i = threadIdx.x; i < EN; i += blockDim.x) {
+        tot[i] = 0;
+        base[i] = 0;
+    }
+    __syncthreads();
+    if (C <= 32) {
+        const int64_t nall = (int64_t)EN * C;
+        for (int64_t f0 = threadIdx.x; f0 < nall; f0 += 8 * (int64_t)blockDim.x) {
+            int v[8], row[8], col[8];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            sum[r] = 0;
-            pre[r] = 0;
-            const int i = i0 + r;
-            if (i < EN) {
-                const int* row = i < E ? a.cnt + (int64_t)i * C : a.ncnt + (int64_t)(i - E) * C;
+            for (int q = 0; q < 8; ++q) {
+                const int64_t f = f0 + (int64_t)q * blockDim.x;
+                col[q] = (int)(f / EN);
+                row[q] = (int)(f - (int64_t)col[q] * EN);
+                v[q] = 0;
+                if (f < nall)
+                    v[q] = row[q] < E ? a.cnt[(int64_t)row[q] * C + col[q]]
+                                      : a.ncnt[(int64_t)(row[q] - E) * C + col[q]];
+            }
 #pragma unroll
-                for (int q = 0; q < kFusedScanMaxChunks / 32; ++q) {
-                    const int c = lane + 32 * q;
-                    if (c < C) {
-                        const int v = row[c];
-                        sum[r] += v;
-                        pre[r] += c < (int)blockIdx.x ? v : 0;
-                    }
+            for (int q = 0; q < 8; ++q) {
+                if (v[q] != 0) {
+                    atomicAdd(&tot[row[q]], v[q]);
+                    if (col[q] < (int)blockIdx.x) atomicAdd(&base[row[q]], v[q]);
                 }
             }
         }
+    } else {
+        for (int i0 = warp * 4; i0 < EN; i0 += kLayoutWarps * 4) {
+            int sum[4], pre[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < 4; ++r) {
+                sum[r] = 0;
+                pre[r] = 0;
+                const int i = i0 + r;
+                if (i < EN) {
+                    const int* row = i < E ? a.cnt + (int64_t)i * C : a.ncnt + (int64_t)(i - E) * C;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                sum[r] += __shfl_xor_sync(kFullMask, sum[r], o);
-                pre[r] += __shfl_xor_sync(kFullMask, pre[r], o);
+                    for (int q = 0; q < kFusedScanMaxChunks / 32; ++q) {
+                        const int c = lane + 32 * q;
+                        if (c < C) {
+                            const int v = row[c];
+                            sum[r] += v;
+                            pre[r] += c < (int)blockIdx.x ? v : 0;
+                        }
+                    }
+                }
             }
-            if (lane == 0 && i0 + r < EN) {
-                tot[i0 + r] = sum[r];
-                base[i0 + r] = pre[r];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sum[r] += __shfl_xor_sync(kFullMask, sum[r], o);
+                    pre[r] += __shfl_xor_sync(kFullMask, pre[r], o);
+                }
+                if (lane == 0 && i0 + r < EN) {
+                    tot[i0 + r] = sum[r];
+                    base[i0 + r] = pre[r];
+                }
             }
         }
     }
     __syncthreads();
+    // Let the dispatch launch only now: its first loads (x rows, started
+    // before it waits for this grid) would otherwise queue ahead of the
+    // histogram reads above, which are this kernel's critical path.
+    pdl_trigger();
     const int total = smem_exclusive_scan(tot, E, s_warp);
     const int ntotal = a.nodes ? smem_exclusive_scan(tot + E, N, s_warp) : 0;
     if (blockIdx.x == 0) {

@@ -84,10 +84,12 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
-def test_large_batch_multi_kernel_layout(oracle_mod):
-    """Above the single-cluster limit (131072 tokens) the layout runs as
-    count / scan / assign kernels over a workspace."""
-    T, H, E, k, R, N = 140001, 8, 64, 4, 8, 2
+@pytest.mark.parametrize("T", [40000, 140001])
+def test_large_batch_multi_kernel_layout(oracle_mod, T):
+    """Above 16384 tokens the layout runs as count + assign kernels over a
+    workspace (the scan folded into assign up to 65536 tokens, a separate
+    scan kernel beyond)."""
+    H, E, k, R, N = 8, 64, 4, 8, 2
     x, topk, w = _small_inputs(T, H, E, k, seed=77)
     ref = oracle_mod.layout(topk, E, R, N, nodes=True)
     for flags in (0, TWO):
