@@ -91,6 +91,23 @@ def profiled_traffic(stage, workload):
     return None
 
 
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (each rank passes its own)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_step, world, steps, seconds):
+    """Whole-job throughput: every rank moved bytes_per_step per step, and the
+    job took the slowest rank's time."""
+    return bytes_per_step * world * steps / seconds / 1e9
+
+
 def algorithmic_bytes(wl, tokens=None):
     T = wl.T if tokens is None else tokens
     row = wl.H * 2
@@ -409,12 +426,7 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     K = args.steps
     with ClockSampler(local) as clocks:
@@ -431,7 +443,7 @@ def main():
 
     disp_b, comb_b = algorithmic_bytes(wl)
     step_bytes = disp_b + comb_b
-    value = step_bytes * world * K / (total_ms * 1e-3) / 1e9
+    value = job_gbs(step_bytes, world, K, total_ms * 1e-3)
     peak, peak_src = measured_peak()
     dom = "dispatch" if t_dispatch >= t_combine else "combine"
     dom_bytes = disp_b if dom == "dispatch" else comb_b
@@ -439,7 +451,7 @@ def main():
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     decoupled = None
     if dec_ms is not None:
-        dec_value = step_bytes * world * K / (dec_ms * 1e-3) / 1e9
+        dec_value = job_gbs(step_bytes, world, K, dec_ms * 1e-3)
         decoupled = {"value": round(dec_value, 2), "unit": "GB/s",
                      "ms_per_step": round(dec_ms / K, 5),
                      "fused_speedup": round(value / dec_value, 3),
@@ -465,12 +477,8 @@ def main():
         capi.moe_combine(cfg, A.lay.struct, A.recv, A.w, A.y)   # identity expert
         y_h.copy_(A.y, non_blocking=True)
         torch.cuda.current_stream().synchronize()
-    e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e_value = step_bytes * world * e2e_steps / e2e_s / 1e9
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
+    e2e_value = job_gbs(step_bytes, world, e2e_steps, e2e_s)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
