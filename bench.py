@@ -284,6 +284,8 @@ def main():
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")
     p.add_argument("--no-decoupled", action="store_true",
                    help="skip timing the pack/copy/unpack comparison path")
+    p.add_argument("--no-agrs", action="store_true",
+                   help="skip timing the all-gather / reduce-scatter comparison path")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=0)
@@ -330,7 +332,7 @@ def main():
     class BufferSet:
         """One independent set of the step's inputs and outputs."""
 
-        def __init__(self, decoupled=False):
+        def __init__(self, decoupled=False, agrs=False):
             self.lay = buffers.DeviceLayout(cfg, dev)
             self.x = buffers.bf16_from_bits(d["x"], dev)
             self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
@@ -348,9 +350,13 @@ def main():
                 self.dxfer = torch.empty((rows, wl.H), **bf16)
                 self.csend = torch.empty((wl.T * wl.k, wl.H), **bf16)
                 self.cxfer = torch.empty((wl.T * wl.k, wl.H), **bf16)
+            if agrs:
+                self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
+                self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
 
     with_decoupled = not args.no_decoupled
-    sets = [BufferSet(with_decoupled), BufferSet(with_decoupled)]
+    with_agrs = not args.no_agrs and wl.R <= capi.MOE_MAX_NODES
+    sets = [BufferSet(with_decoupled, with_agrs), BufferSet(with_decoupled, with_agrs)]
 
     def layout(b):
         capi.moe_layout(cfg, b.topk, b.lay.struct)
@@ -371,6 +377,11 @@ def main():
         capi.moe_dispatch_decoupled(dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
         capi.moe_combine_decoupled(dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
 
+    def agrs_step(b):
+        layout(b)
+        capi.moe_dispatch_allgather(cfg, b.lay.struct, b.x, b.gathered, b.recv)
+        capi.moe_combine_reducescatter(cfg, b.lay.struct, b.eo, b.w, b.partial, b.y)
+
     cluster_layout = args.layout == "cluster" and wl.T <= 131072
     small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
     layout_launches = 1 if cluster_layout else (2 if small_layout else 3)
@@ -380,6 +391,8 @@ def main():
         step(sets[i % 2])
         if with_decoupled:
             decoupled_step(sets[i % 2])
+        if with_agrs:
+            agrs_step(sets[i % 2])
     torch.cuda.synchronize()
     for b in sets:
         for lay in [b.lay] + ([b.dlay] if with_decoupled else []):
@@ -407,6 +420,8 @@ def main():
     if with_decoupled:
         graphs["decoupled"] = (capture(lambda: (decoupled_step(A), decoupled_step(B))),
                                capture(lambda: decoupled_step(A)))
+    if with_agrs:
+        graphs["agrs"] = (capture(lambda: (agrs_step(A), agrs_step(B))), capture(lambda: agrs_step(A)))
     for pair, single in graphs.values():
         pair.replay()
         single.replay()
@@ -434,6 +449,7 @@ def main():
         t_l = timed("L", K) / K
         t_ld = timed("LD", K) / K
         dec_ms = timed("decoupled", K) if with_decoupled else None
+        agrs_ms = timed("agrs", K) if with_agrs else None
     ms_per_step = total_ms / K
     t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
     for b in sets:
@@ -457,6 +473,14 @@ def main():
                      "fused_speedup": round(value / dec_value, 3),
                      "path": "layout (per-rank groups) + pack/copy/unpack dispatch + "
                              "pack/copy/unpack combine"}
+
+    agrs = None
+    if agrs_ms is not None:
+        ag_value = job_gbs(step_bytes, world, K, agrs_ms * 1e-3)
+        agrs = {"value": round(ag_value, 2), "unit": "GB/s", "ms_per_step": round(agrs_ms / K, 5),
+                "fused_speedup": round(value / ag_value, 3),
+                "path": "layout + all-gather dispatch (R copies, per-rank select) + "
+                        "reduce-scatter combine (per-rank fp32 partials, rank-order sum)"}
 
     # end to end through the C ABI from pinned host buffers
     e2e_steps = args.e2e_steps or min(K, 50)
@@ -519,6 +543,7 @@ def main():
                          "traffic": profiled_traffic(dom, wl.name),
                          "peak_kind": f"{peak_src} copy bandwidth"},
             "decoupled_3pass": decoupled,
+            "allgather_reducescatter": agrs,
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

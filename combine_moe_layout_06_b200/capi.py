@@ -48,7 +48,8 @@ ENTRY_POINTS = (
     "moe_status_string", "moe_check_config", "moe_expert_partition",
     "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
-    "moe_layout_noalloc", "moe_layout_dispatch",
+    "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
+    "moe_combine_reducescatter",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -103,6 +104,8 @@ def lib() -> ctypes.CDLL:
     L.moe_combine_decoupled.argtypes = [C, LP, P, P, P, P, P, P]
     L.moe_layout_noalloc.argtypes = [C, P, LP, P]
     L.moe_layout_dispatch.argtypes = [C, P, LP, P, P, P, P]
+    L.moe_dispatch_allgather.argtypes = [C, LP, P, P, P, P]
+    L.moe_combine_reducescatter.argtypes = [C, LP, P, P, P, P, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -217,3 +220,18 @@ def moe_layout_noalloc(cfg: MoeConfig, topk_idx, layout: MoeLayout, stream=None)
     layout.workspace (for callers that cannot allocate device memory)."""
     _check(lib().moe_layout_noalloc(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(layout),
                                     _stream(stream)), "moe_layout_noalloc")
+
+
+def moe_dispatch_allgather(cfg: MoeConfig, layout: MoeLayout, x, gathered, recv,
+                           stream=None) -> None:
+    _check(lib().moe_dispatch_allgather(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x),
+                                        _ptr(gathered), _ptr(recv), _stream(stream)),
+           "moe_dispatch_allgather")
+
+
+def moe_combine_reducescatter(cfg: MoeConfig, layout: MoeLayout, expert_out, topk_weights,
+                              partial, y, stream=None) -> None:
+    _check(lib().moe_combine_reducescatter(ctypes.byref(cfg), ctypes.byref(layout),
+                                           _ptr(expert_out), _ptr(topk_weights), _ptr(partial),
+                                           _ptr(y), _stream(stream)),
+           "moe_combine_reducescatter")

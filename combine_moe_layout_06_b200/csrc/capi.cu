@@ -275,4 +275,47 @@ moe_status_t moe_combine_decoupled(const moe_config_t* c, const moe_layout_t* L,
     return cuda_status(e);
 }
 
+moe_status_t moe_dispatch_allgather(const moe_config_t* c, const moe_layout_t* L, const void* x,
+                                    void* gathered, void* recv, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (c->num_ranks > MOE_MAX_NODES) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || gathered == nullptr || recv == nullptr) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    moe::RowMoveParams p = move_params(c, L);
+    p.N = c->num_ranks;  // one lane per rank in the all-gather
+    cudaError_t e = moe::launch_allgather_rows(p, x, gathered, s);
+    if (e == cudaSuccess) e = moe::launch_rank_select(p, gathered, recv, s);
+    return cuda_status(e);
+}
+
+moe_status_t moe_combine_reducescatter(const moe_config_t* c, const moe_layout_t* L,
+                                       const void* expert_out, const float* topk_weights,
+                                       float* partial, void* y, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (c->num_ranks > MOE_MAX_NODES) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (expert_out == nullptr || topk_weights == nullptr || partial == nullptr || y == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    moe::CombineParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.row_bytes = (size_t)c->hidden * 2;
+    p.slot = L->slot;
+    p.w = topk_weights;
+    p.err = L->error_word;
+    p.engine = engine_of(c->flags);
+    cudaError_t e = moe::launch_combine_rank_partials(p, c->num_ranks, L->rank_offsets, expert_out,
+                                                      partial, s);
+    if (e == cudaSuccess) e = moe::launch_reduce_rank_partials(p, c->num_ranks, partial, y, s);
+    return cuda_status(e);
+}
+
 }  // extern "C"

@@ -153,6 +153,111 @@ cudaError_t launch_combine_k(CombArgs a, cudaStream_t stream) {
     return launch_combine_v<V, VPL, (MOE_COMBINE_KB > 4 ? MOE_COMBINE_KB : 4)>(a, stream);
 }
 
+// ---- reduce-scatter formulation (comparison path) -------------------------
+// INC-MoE abstract: combine as a ReduceScatter; TensorRT-LLM PR #13888: the
+// AllGather + ReduceScatter fallback.  On one GPU: every virtual rank r
+// first sums, for every token, its own experts' rows (fp32, FMA in column
+// order) into partial[r][t]; the partials are then added in rank order and
+// rounded once.
+
+template <int EPV>
+__device__ __forceinline__ void store_f32(float* p, const float (&f)[EPV]) {
+    if constexpr (EPV == 8) {
+        reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+        reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+    } else if constexpr (EPV == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(f[0], f[1]);
+    } else {
+        p[0] = f[0];
+    }
+}
+
+template <int EPV>
+__device__ __forceinline__ void load_f32(const float* p, float (&f)[EPV]) {
+    if constexpr (EPV == 8) {
+        const float4 a = reinterpret_cast<const float4*>(p)[0];
+        const float4 b = reinterpret_cast<const float4*>(p)[1];
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else if constexpr (EPV == 2) {
+        const float2 a = *reinterpret_cast<const float2*>(p);
+        f[0] = a.x; f[1] = a.y;
+    } else {
+        f[0] = p[0];
+    }
+}
+
+struct RankArgs {
+    CombArgs c;
+    int R;
+    const int* rank_offsets;
+    float* partial;       // [R*T][H] fp32
+};
+
+// Items (r, t, chunk), rank-major; a warp per item.
+template <typename V>
+__global__ void __launch_bounds__(kThreads) rank_partial_kernel(RankArgs ra) {
+    constexpr int EPV = VecInfo<V>::kElems;
+    const CombArgs& a = ra.c;
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t cpr = (a.rv + 31) / 32;
+    const int64_t items = (int64_t)ra.R * a.T * cpr;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t H = a.rv * EPV;
+    int errbits = 0;
+    for (int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); item < items; item += nw) {
+        const int64_t row = item / cpr;                 // r*T + t
+        const int64_t base = (item - row * cpr) * 32;
+        const int r = (int)(row / a.T);
+        const int64_t t = row - (int64_t)r * a.T;
+        const int lo = __ldg(ra.rank_offsets + r), hi = __ldg(ra.rank_offsets + r + 1);
+        int s = -1;
+        float wl = 0.f;
+        load_route(a, t, lane, s, wl, errbits);
+        float acc[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+        const int64_t idx = base + lane;
+        for (int j = 0; j < a.k; ++j) {
+            const int sj = __shfl_sync(kFullMask, s, j);
+            const float wj = __shfl_sync(kFullMask, wl, j);
+            if (sj < lo || sj >= hi || idx >= a.rv) continue;
+            float f[EPV];
+            unpack_bf16<V>(ld_stream(static_cast<const V*>(a.eo) + (int64_t)sj * a.rv + idx), f);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) acc[e] = __fmaf_rn(wj, f[e], acc[e]);
+        }
+        if (idx < a.rv) store_f32<EPV>(ra.partial + row * H + idx * EPV, acc);
+    }
+    warp_report(a.err, errbits);
+}
+
+template <typename V>
+__global__ void __launch_bounds__(kThreads) rank_reduce_kernel(RankArgs ra) {
+    constexpr int EPV = VecInfo<V>::kElems;
+    const CombArgs& a = ra.c;
+    pdl_trigger();
+    pdl_wait();
+    const int64_t n = a.T * a.rv;                      // output vectors
+    const int64_t H = a.rv * EPV;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const int64_t t = i / a.rv, v = i - t * a.rv;
+        float acc[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
+        for (int r = 0; r < ra.R; ++r) {
+            float f[EPV];
+            load_f32<EPV>(ra.partial + ((int64_t)r * a.T + t) * H + v * EPV, f);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) acc[e] = acc[e] + f[e];
+        }
+        static_cast<V*>(a.y)[i] = pack_bf16<V>(acc);
+    }
+}
+
 inline int vec_bytes(size_t row_bytes, const void* a, const void* b) {
     const uintptr_t bits = row_bytes | reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b);
     if (bits % 16 == 0) return 16;
@@ -188,6 +293,60 @@ cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void*
             a.rv = (int64_t)(p.row_bytes / 2);
             return launch_combine_k<uint16_t, 4>(a, stream);
     }
+}
+
+static CombArgs comb_args(const CombineParams& p, const void* expert_out, void* y) {
+    CombArgs a;
+    a.eo = expert_out;
+    a.w = p.w;
+    a.slot = p.slot;
+    a.y = y;
+    a.T = p.T;
+    a.k = p.k;
+    a.eo_rows = p.T * p.k;
+    a.err = p.err;
+    a.rv = 0;
+    return a;
+}
+
+cudaError_t launch_combine_rank_partials(const CombineParams& p, int R, const int* rank_offsets,
+                                         const void* expert_out, float* partial,
+                                         cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    RankArgs ra;
+    ra.c = comb_args(p, expert_out, nullptr);
+    ra.R = R;
+    ra.rank_offsets = rank_offsets;
+    ra.partial = partial;
+    const int vb = vec_bytes(p.row_bytes, expert_out, partial);
+    auto go = [&](auto kern, int bytes) {
+        ra.c.rv = (int64_t)(p.row_bytes / bytes);
+        const int64_t cpr = (ra.c.rv + 31) / 32;
+        int64_t g = ((int64_t)R * p.T * cpr + kWarpsPerCta - 1) / kWarpsPerCta;
+        const int64_t cap = (int64_t)device_sm_count() * 16;
+        return launch_pdl(kern, dim3((unsigned)(g > cap ? cap : g)), dim3(kThreads), 0, stream, ra);
+    };
+    if (vb == 16) return go(rank_partial_kernel<uint4>, 16);
+    if (vb == 4) return go(rank_partial_kernel<uint32_t>, 4);
+    return go(rank_partial_kernel<uint16_t>, 2);
+}
+
+cudaError_t launch_reduce_rank_partials(const CombineParams& p, int R, const float* partial,
+                                        void* y, cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    RankArgs ra;
+    ra.c = comb_args(p, nullptr, y);
+    ra.R = R;
+    ra.rank_offsets = nullptr;
+    ra.partial = const_cast<float*>(partial);
+    const int vb = vec_bytes(p.row_bytes, partial, y);
+    auto go = [&](auto kern, int bytes) {
+        ra.c.rv = (int64_t)(p.row_bytes / bytes);
+        return launch_pdl(kern, dim3((unsigned)(device_sm_count() * 8)), dim3(kThreads), 0, stream, ra);
+    };
+    if (vb == 16) return go(rank_reduce_kernel<uint4>, 16);
+    if (vb == 4) return go(rank_reduce_kernel<uint32_t>, 4);
+    return go(rank_reduce_kernel<uint16_t>, 2);
 }
 
 }  // namespace moe

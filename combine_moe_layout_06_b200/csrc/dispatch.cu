@@ -39,7 +39,7 @@ namespace {
 constexpr int kWarpsPerCta = 8;
 constexpr int kThreads = kWarpsPerCta * 32;
 
-enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2 };
+enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2, kAllGather = 3, kRankSelect = 4 };
 
 struct FanArgs {
     const void* src;
@@ -88,6 +88,19 @@ __device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int l
         const bool ok = ns >= 0 && d >= 0 && d < a.dst_rows;
         p.dst = ok ? d : -1;
         p.bad = (ns >= 0 && !ok) ? kErrBadLayout : 0;
+    } else if (MODE == kAllGather) {
+        // every virtual rank (lane r < N) receives a copy of every token
+        p.src = row;
+        p.dst = lane < a.N ? (int64_t)lane * a.T + row : -1;
+    } else if (MODE == kRankSelect) {
+        // rank r keeps, from its gathered copy, the token's rows on its experts
+        const int r = (int)(row / a.T);
+        const int64_t t = row - (int64_t)r * a.T;
+        const int lo = __ldg(a.rank_offsets + r);
+        const int hi = __ldg(a.rank_offsets + r + 1);
+        const int s = lane < a.k ? __ldg(a.slot + t * a.k + lane) : -1;
+        p.src = row;
+        p.dst = (s >= lo && s < hi && s < a.dst_rows) ? s : -1;
     } else {
         const int n = (int)(row / a.T);
         const int64_t t = row - (int64_t)n * a.T;
@@ -113,7 +126,7 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
+    const int64_t rows = (MODE == kNodeExpand || MODE == kRankSelect) ? a.T * a.N : a.T;
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = rows * cpr;
     const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
@@ -312,6 +325,19 @@ cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging, int6
         return launch_node_expand_bulk(p, staging, staging_rows, recv, stream);
     FanArgs a = fan_args(p, staging, recv, staging_rows, p.T * p.k);
     return launch_fan<kNodeExpand>(a, p.T * p.N, stream);
+}
+
+cudaError_t launch_allgather_rows(const RowMoveParams& p, const void* x, void* gathered,
+                                  cudaStream_t stream) {
+    // lanes are ranks: N carries the rank count here
+    FanArgs a = fan_args(p, x, gathered, p.T, p.T * p.N);
+    return launch_fan<kAllGather>(a, p.T, stream);
+}
+
+cudaError_t launch_rank_select(const RowMoveParams& p, const void* gathered, void* recv,
+                               cudaStream_t stream) {
+    FanArgs a = fan_args(p, gathered, recv, p.T * p.N, p.T * p.k);
+    return launch_fan<kRankSelect>(a, p.T * p.N, stream);
 }
 
 cudaError_t launch_gather_rows(const RowMoveParams& p, const void* src, void* dst,

@@ -67,6 +67,13 @@ cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging,
 // when rows_dev is given, else max_rows.
 cudaError_t launch_copy_rows(const void* src, void* dst, const int* rows_dev, int64_t max_rows,
                              size_t row_bytes, cudaStream_t stream);
+// gathered[r*T + t] = x[t] for r < p.N (p.N = rank count; all-gather)
+cudaError_t launch_allgather_rows(const RowMoveParams& p, const void* x, void* gathered,
+                                  cudaStream_t stream);
+// recv[slot[t][j]] = gathered[r*T + t] for the j whose row lies on rank r
+// (p.N = rank count, rows of rank r in [rank_offsets[r], rank_offsets[r+1]))
+cudaError_t launch_rank_select(const RowMoveParams& p, const void* gathered, void* recv,
+                               cudaStream_t stream);
 // dst[t*k + j] = src[slot[t][j]]
 cudaError_t launch_gather_rows(const RowMoveParams& p, const void* src, void* dst,
                                cudaStream_t stream);
@@ -83,6 +90,15 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void* y,
                            cudaStream_t stream);
+
+// partial[r*T + t] = fp32 sum over the j whose row lies on rank r of
+// w[t][j] * eo[slot[t][j]] (j order, FMA), for r < R
+cudaError_t launch_combine_rank_partials(const CombineParams& p, int R, const int* rank_offsets,
+                                         const void* expert_out, float* partial,
+                                         cudaStream_t stream);
+// y[t] = bf16_rne(sum over r in order of partial[r*T + t])
+cudaError_t launch_reduce_rank_partials(const CombineParams& p, int R, const float* partial,
+                                        void* y, cudaStream_t stream);
 
 // ---- bulk-copy (TMA) engine (bulk.cu) ------------------------------------------
 // Usable when the row size and every base address are multiples of 16 bytes.

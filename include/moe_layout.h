@@ -238,6 +238,33 @@ moe_status_t moe_combine_decoupled(const moe_config_t *cfg,
                                    const float *topk_weights, void *send,
                                    void *xfer, void *y, void *stream);
 
+/* ---- AllGather / ReduceScatter comparison path ----
+ * The collective formulation of dispatch and combine: INC-MoE abstract
+ * (dispatch as an in-network AllGather, combine as a ReduceScatter) and the
+ * AllGather + ReduceScatter fallback of TensorRT-LLM PR #13888.  On one GPU
+ * the R virtual ranks are regions of HBM.  Requires num_ranks <=
+ * MOE_MAX_NODES and a layout from moe_layout() with the same cfg. */
+
+/* Dispatch, all-gather form.  All-gather: every rank r receives a copy of
+ * every token, gathered[r*T + t] = x[t].  Select: rank r copies, from its
+ * gathered rows, each token's rows on its experts into recv (rank r's rows
+ * are [rank_offsets[r], rank_offsets[r+1])).  recv equals moe_dispatch()'s
+ * bit for bit.
+ *   gathered  device bf16 [R*T][H] */
+moe_status_t moe_dispatch_allgather(const moe_config_t *cfg, const moe_layout_t *layout,
+                                    const void *x, void *gathered, void *recv, void *stream);
+
+/* Combine, reduce-scatter form.  Every rank r sums, for every token, the
+ * weighted rows of its own experts in fp32 (one FMA per column j in order,
+ * from +0) into partial[r*T + t]; then y[t] = bf16_rne(partial[0*T+t] +
+ * partial[1*T+t] + ... ) added in rank order from +0.  Agrees with
+ * moe_combine() within the combine tolerance (the additions are ordered
+ * differently).
+ *   partial  device fp32 [R*T][H] */
+moe_status_t moe_combine_reducescatter(const moe_config_t *cfg, const moe_layout_t *layout,
+                                       const void *expert_out, const float *topk_weights,
+                                       float *partial, void *y, void *stream);
+
 /* ---- layout without caller-provided scratch ----
  * No counterpart on the pages: this entry point exists for callers that
  * cannot allocate device memory (for example code that runs while a stream

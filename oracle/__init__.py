@@ -85,6 +85,8 @@ def _bind(path: str):
     lib.oracle_combine.restype = None
     lib.oracle_combine_tokens.argtypes = [i64, p, i32, i32, p, p, p, p]
     lib.oracle_combine_tokens.restype = None
+    lib.oracle_combine_rank_partials.argtypes = [i64, i32, i32, i32, p, p, p, p, p]
+    lib.oracle_combine_rank_partials.restype = None
     lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
     lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
     lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -226,4 +228,20 @@ def combine_tokens(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray,
     y = np.zeros((tokens.size, H), np.uint16)
     _load().oracle_combine_tokens(tokens.size, _ptr(tokens), H, k, _ptr(slot),
                                   _ptr(w), _ptr(eo_bits), _ptr(y))
+    return y
+
+
+def combine_rank_partials(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray,
+                          rank_offsets: np.ndarray) -> np.ndarray:
+    """Combine in the reduce-scatter order: per-rank fp32 partial sums, added
+    in rank order, one bf16 rounding."""
+    eo_bits = _c(eo_bits, np.uint16)
+    w = _c(w, np.float32)
+    slot = _c(slot, np.int32)
+    ro = _c(rank_offsets, np.int32)
+    T, k = slot.shape
+    H = eo_bits.shape[1]
+    y = np.zeros((T, H), np.uint16)
+    _load().oracle_combine_rank_partials(T, H, k, ro.size - 1, _ptr(slot), _ptr(ro), _ptr(w),
+                                         _ptr(eo_bits), _ptr(y))
     return y

@@ -381,3 +381,29 @@ void oracle_combine_tokens(int64_t n_tokens, const int64_t *tokens,
         }
     }
 }
+
+/* Combine in the reduce-scatter order (INC-MoE abstract: combine as a
+ * ReduceScatter; TensorRT-LLM PR #13888: the AllGather + ReduceScatter
+ * fallback path).  Each rank r first sums, in fp32 with one FMA per column
+ * j in order, the token's expert rows that live on r (its receive rows lie in
+ * [rank_offsets[r], rank_offsets[r+1])); the R partial sums are then added
+ * in rank order starting from +0, and the total is rounded once to bf16. */
+void oracle_combine_rank_partials(int64_t T, int32_t H, int32_t k, int32_t R,
+                                  const int32_t *slot, const int32_t *rank_offsets,
+                                  const float *w, const uint16_t *eo, uint16_t *y)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            float total = 0.0f;
+            for (int32_t r = 0; r < R; ++r) {
+                float part = 0.0f;
+                for (int32_t j = 0; j < k; ++j) {
+                    int32_t row = slot[t * k + j];
+                    if (row >= rank_offsets[r] && row < rank_offsets[r + 1])
+                        part = fmaf(w[t * k + j], oracle_bf16_to_f32(eo[(int64_t)row * H + h]), part);
+                }
+                total = total + part;
+            }
+            y[t * H + h] = oracle_f32_to_bf16(total);
+        }
+}

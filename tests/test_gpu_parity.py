@@ -330,3 +330,42 @@ def test_bad_slot_is_reported_and_skipped():
     y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
     capi.moe_combine(cfg, lay.struct, recv, torch.from_numpy(w).cuda(), y)
     assert capi.moe_get_error(lay.struct) == capi.MOE_ERR_BAD_LAYOUT
+
+
+# ---------------------------------------------------------- all-gather / reduce-scatter
+
+@pytest.mark.parametrize("name", ["tiny", "olmoe", "longctx", "small"])
+def test_allgather_reducescatter(oracle_mod, name):
+    if name == "small":
+        T, H, E, k, R = 333, 72, 24, 5, 6
+        x, topk, w = _small_inputs(T, H, E, k, seed=12)
+    else:
+        d = inputs.make(name)
+        wl = d["workload"]
+        T, H, E, k, R = wl.T, wl.H, wl.E, wl.k, wl.R
+        x, topk, w = d["x"], d["topk_idx"], d["topk_w"]
+    ref = oracle_mod.layout(topk, E, R)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, topk)
+    x_dev = M.to_dev(x)
+    gathered = torch.empty((R * T, H), dtype=torch.bfloat16, device="cuda")
+    recv = torch.empty((T * k, H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_dispatch_allgather(cfg, lay.struct, x_dev, gathered, recv)
+    assert torch.equal(gathered.view(R, T, H).view(torch.int16),
+                       x_dev.view(torch.int16).unsqueeze(0).expand(R, T, H))
+    if T * k * H <= 1 << 28:
+        assert np.array_equal(M.bits(recv), oracle_mod.dispatch_flat(x, ref["slot"]))
+    else:
+        slot_dev = torch.from_numpy(ref["slot"].reshape(-1).astype(np.int64)).cuda()
+        tok_dev = torch.arange(T, device="cuda").repeat_interleave(k)
+        assert torch.equal(recv.view(torch.int16)[slot_dev], x_dev.view(torch.int16)[tok_dev])
+    eo = inputs.random_bf16_bits((T * k, H), seed=T + H + 1)
+    partial = torch.empty((R * T, H), dtype=torch.float32, device="cuda")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_combine_reducescatter(cfg, lay.struct, M.to_dev(eo), torch.from_numpy(w).cuda(),
+                                   partial, y)
+    y_bits = M.bits(y)
+    assert np.array_equal(y_bits, oracle_mod.combine_rank_partials(eo, w, ref["slot"],
+                                                                   ref["rank_offsets"]))
+    M.assert_combine_close(y_bits, oracle_mod.combine(eo, w, ref["slot"]))
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK

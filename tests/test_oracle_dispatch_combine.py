@@ -191,3 +191,49 @@ def test_combine_accumulation_order_is_column_order(oracle_mod):
     eo2 = oracle_mod.f32_to_bf16(np.array([[2.0 ** 20], [2.0 ** -9], [-(2.0 ** 20)]], np.float32))
     y2 = _bits_to_f64(oracle_mod.combine(eo2, w, slot))
     assert y2[0, 0] == 0.0, "2^20 + 2^-9 rounds back to 2^20 in fp32 before the subtraction"
+
+
+# ------------------------------------------------------------ reduce-scatter order
+
+@pytest.mark.parametrize("T,H,E,k,R,N", CASES)
+def test_rank_partial_combine_within_rounding_bound(oracle_mod, T, H, E, k, R, N):
+    """Per-rank fp32 partials added in rank order: within the bound of the
+    fp64 sum (k FMAs plus R adds, one bf16 rounding)."""
+    x, topk, w = _case(T, H, E, k, R, N, seed=11 * T + H)
+    lay = oracle_mod.layout(topk, E, R, N)
+    eo = inputs.random_bf16_bits((T * k, H), seed=T + 3 * H)
+    y = _bits_to_f64(oracle_mod.combine_rank_partials(eo, w, lay["slot"], lay["rank_offsets"]))
+    eof = _bits_to_f64(eo)
+    terms = w.astype(np.float64)[:, None, :] * np.stack(
+        [eof[lay["slot"][:, j]] for j in range(k)], axis=-1)
+    exact = terms.sum(-1)
+    bound = (2.0 ** -8 * np.abs(exact)
+             + (1 + 2.0 ** -8) * (k + R) * 2.0 ** -24 * np.abs(terms).sum(-1) + 1e-45)
+    assert np.all(np.abs(y - exact) <= bound)
+
+
+def test_rank_partial_combine_single_rank_equals_column_order(oracle_mod):
+    """With one rank the partial is the whole column-order sum (+0 + p = p)."""
+    x, topk, w = _case(90, 48, 12, 3, 1, 1, seed=4)
+    lay = oracle_mod.layout(topk, 12, 1)
+    eo = inputs.random_bf16_bits((270, 48), seed=8)
+    assert np.array_equal(oracle_mod.combine_rank_partials(eo, w, lay["slot"], lay["rank_offsets"]),
+                          oracle_mod.combine(eo, w, lay["slot"]))
+
+
+def test_rank_partial_combine_order_is_rank_order(oracle_mod):
+    """fp32 addition is not associative: a token whose expert on rank 1 carries
+    -2^20 and whose experts on rank 0 carry 2^20 and 2^-9 must give the
+    rank-order result (2^20 + 2^-9 rounds to 2^20 before the -2^20 is added)."""
+    E, R = 4, 2                      # ranks own experts {0,1} and {2,3}
+    topk = np.array([[2, 0, 1]], np.int32)
+    lay = oracle_mod.layout(topk, E, R)
+    vals = {0: 2.0 ** 20, 1: 2.0 ** -9, 2: -(2.0 ** 20)}
+    eo = np.zeros((3, 1), np.uint16)
+    for j, e in enumerate(topk[0]):
+        eo[lay["slot"][0, j], 0] = oracle_mod.f32_to_bf16(np.float32(vals[e]))
+    w = np.ones((1, 3), np.float32)
+    y_rs = _bits_to_f64(oracle_mod.combine_rank_partials(eo, w, lay["slot"], lay["rank_offsets"]))
+    y_col = _bits_to_f64(oracle_mod.combine(eo, w, lay["slot"]))
+    assert y_rs[0, 0] == 0.0          # (2^20 + 2^-9) - 2^20 in fp32 = 0
+    assert y_col[0, 0] == 2.0 ** -9   # -2^20 + 2^20 + 2^-9 in column order

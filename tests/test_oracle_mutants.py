@@ -51,6 +51,9 @@ MUTANTS = {
     "validation_misses_adjacent_repeat": (
         "for (int32_t i = 0; i < j; ++i)",
         "for (int32_t i = 0; i + 1 < j; ++i)"),
+    "rank_partial_range_off_by_one": (
+        "if (row >= rank_offsets[r] && row < rank_offsets[r + 1])",
+        "if (row >= rank_offsets[r] && row <= rank_offsets[r + 1])"),
     "widening_drops_low_bit": (
         "    uint32_t u = ((uint32_t)h) << 16;",
         "    uint32_t u = ((uint32_t)(h & 0xFFFEu)) << 16;"),
