@@ -87,6 +87,16 @@ def _bind(path: str):
     lib.oracle_combine_tokens.restype = None
     lib.oracle_combine_rank_partials.argtypes = [i64, i32, i32, i32, p, p, p, p, p]
     lib.oracle_combine_rank_partials.restype = None
+    lib.oracle_e4m3_to_f32.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_f32.restype = ctypes.c_float
+    lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.oracle_quantize_rows_fp8.argtypes = [i64, i32, p, p, p]
+    lib.oracle_quantize_rows_fp8.restype = None
+    lib.oracle_dispatch_fp8.argtypes = [i64, i32, i32, p, p, p, p]
+    lib.oracle_dispatch_fp8.restype = None
+    lib.oracle_combine_fp8.argtypes = [i64, i32, i32, p, p, p, p, p]
+    lib.oracle_combine_fp8.restype = None
     lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
     lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
     lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
@@ -244,4 +254,51 @@ def combine_rank_partials(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray,
     y = np.zeros((T, H), np.uint16)
     _load().oracle_combine_rank_partials(T, H, k, ro.size - 1, _ptr(slot), _ptr(ro), _ptr(w),
                                          _ptr(eo_bits), _ptr(y))
+    return y
+
+
+# ---------------------------------------------------------------- fp8 payload
+
+def e4m3_to_f32(codes) -> np.ndarray:
+    codes = _c(codes, np.uint8).ravel()
+    L = _load()
+    return np.array([L.oracle_e4m3_to_f32(int(c)) for c in codes], np.float32)
+
+
+def f32_to_e4m3(vals) -> np.ndarray:
+    vals = _c(vals, np.float32).ravel()
+    L = _load()
+    return np.array([L.oracle_f32_to_e4m3(float(v)) for v in vals], np.uint8)
+
+
+def quantize_rows_fp8(src_bits: np.ndarray):
+    """bf16 rows -> (e4m3 codes uint8 [rows, H], fp32 scale [rows])."""
+    src_bits = _c(src_bits, np.uint16)
+    rows, H = src_bits.shape
+    q = np.zeros((rows, H), np.uint8)
+    scale = np.zeros(rows, np.float32)
+    _load().oracle_quantize_rows_fp8(rows, H, _ptr(src_bits), _ptr(q), _ptr(scale))
+    return q, scale
+
+
+def dispatch_fp8(x_bits: np.ndarray, slot: np.ndarray):
+    x_bits = _c(x_bits, np.uint16)
+    slot = _c(slot, np.int32)
+    T, H = x_bits.shape
+    k = slot.shape[1]
+    q = np.zeros((T * k, H), np.uint8)
+    scale = np.zeros(T * k, np.float32)
+    _load().oracle_dispatch_fp8(T, H, k, _ptr(slot), _ptr(x_bits), _ptr(q), _ptr(scale))
+    return q, scale
+
+
+def combine_fp8(eo_q: np.ndarray, eo_scale: np.ndarray, w: np.ndarray, slot: np.ndarray):
+    eo_q = _c(eo_q, np.uint8)
+    eo_scale = _c(eo_scale, np.float32)
+    w = _c(w, np.float32)
+    slot = _c(slot, np.int32)
+    T, k = slot.shape
+    H = eo_q.shape[1]
+    y = np.zeros((T, H), np.uint16)
+    _load().oracle_combine_fp8(T, H, k, _ptr(slot), _ptr(w), _ptr(eo_q), _ptr(eo_scale), _ptr(y))
     return y

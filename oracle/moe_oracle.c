@@ -407,3 +407,114 @@ void oracle_combine_rank_partials(int64_t T, int32_t H, int32_t k, int32_t R,
             y[t * H + h] = oracle_f32_to_bf16(total);
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 (e4m3) payload                                                  */
+/* ------------------------------------------------------------------ */
+/* TensorRT-LLM PR #13888 (the ConfigurableMoE commit) validates an fp8
+ * low-precision combine at rtol 0.02 / atol 0.15.  The encoding is the OCP
+ * FP8 E4M3 format: sign, 4 exponent bits (bias 7), 3 mantissa bits, no
+ * infinities, S.1111.111 is NaN, largest finite value 448.  The reading
+ * taken for the payload: one fp32 scale per row, scale = amax / 448 (amax =
+ * largest |value| of the row; a zero row uses scale 1), values stored as
+ * e4m3(v * (448 / amax)) rounded to nearest even and saturated to +-448. */
+
+/* Decode one e4m3 code (exact in fp32). */
+float oracle_e4m3_to_f32(uint8_t c)
+{
+    int sign = (c >> 7) & 1;
+    int exp_bits = (c >> 3) & 0xF;
+    int man = c & 7;
+    float v;
+    if (exp_bits == 0xF && man == 7)
+        return sign ? -NAN : NAN;
+    if (exp_bits == 0)
+        v = ldexpf((float)man, -9);                 /* subnormal: m/8 * 2^-6 */
+    else
+        v = ldexpf((float)(8 + man), exp_bits - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Encode: round to nearest (ties to even code) over the finite e4m3 values,
+ * saturating beyond 448; NaN maps to the NaN code. Written as a search over
+ * the 127 non-negative finite codes, which are in increasing order. */
+uint8_t oracle_f32_to_e4m3(float f)
+{
+    if (f != f)
+        return 0x7F;
+    uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    float a = fabsf(f);
+    if (a >= 448.0f)
+        return (uint8_t)(sign | 0x7E);
+    uint8_t lo = 0;
+    for (uint8_t c = 0; c < 0x7E; ++c)
+        if (oracle_e4m3_to_f32((uint8_t)(c + 1)) <= a)
+            lo = (uint8_t)(c + 1);
+    /* a lies in [val(lo), val(lo+1)) */
+    float vlo = oracle_e4m3_to_f32(lo);
+    float vhi = oracle_e4m3_to_f32((uint8_t)(lo + 1));
+    double dlo = (double)a - (double)vlo, dhi = (double)vhi - (double)a;
+    uint8_t pick;
+    if (dlo < dhi)
+        pick = lo;
+    else if (dhi < dlo)
+        pick = (uint8_t)(lo + 1);
+    else
+        pick = (lo & 1) ? (uint8_t)(lo + 1) : lo;   /* tie: even code */
+    return (uint8_t)(sign | pick);
+}
+
+/* Quantize `rows` bf16 rows of H values to e4m3 with one scale per row. */
+void oracle_quantize_rows_fp8(int64_t rows, int32_t H, const uint16_t *src, uint8_t *q,
+                              float *scale)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int32_t h = 0; h < H; ++h) {
+            float v = fabsf(oracle_bf16_to_f32(src[r * H + h]));
+            if (v > amax)
+                amax = v;
+        }
+        float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+        scale[r] = amax > 0.0f ? amax / 448.0f : 1.0f;
+        for (int32_t h = 0; h < H; ++h)
+            q[r * H + h] = oracle_f32_to_e4m3(oracle_bf16_to_f32(src[r * H + h]) * inv);
+    }
+}
+
+/* fp8 dispatch: quantize x, then every destination row receives the token's
+ * codes and scale. */
+void oracle_dispatch_fp8(int64_t T, int32_t H, int32_t k, const int32_t *slot,
+                         const uint16_t *x, uint8_t *recv_q, float *recv_scale)
+{
+    uint8_t *qt = (uint8_t *)malloc((size_t)H);
+    float st;
+    for (int64_t t = 0; t < T; ++t) {
+        oracle_quantize_rows_fp8(1, H, x + t * H, qt, &st);
+        for (int32_t j = 0; j < k; ++j) {
+            int64_t dst = slot[t * k + j];
+            memcpy(recv_q + dst * H, qt, (size_t)H);
+            recv_scale[dst] = st;
+        }
+    }
+    free(qt);
+}
+
+/* fp8 combine: coef_j = w[t][j] * scale[slot[t][j]] (fp32), then
+ * acc = fma(coef_j, e4m3(eo_q[slot][h]), acc) for j = 0..k-1 from +0, one
+ * bf16 rounding. */
+void oracle_combine_fp8(int64_t T, int32_t H, int32_t k, const int32_t *slot,
+                        const float *w, const uint8_t *eo_q, const float *eo_scale,
+                        uint16_t *y)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                int64_t row = slot[t * k + j];
+                float coef = w[t * k + j] * eo_scale[row];
+                acc = fmaf(coef, oracle_e4m3_to_f32(eo_q[row * H + h]), acc);
+            }
+            y[t * H + h] = oracle_f32_to_bf16(acc);
+        }
+}

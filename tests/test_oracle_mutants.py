@@ -54,6 +54,15 @@ MUTANTS = {
     "rank_partial_range_off_by_one": (
         "if (row >= rank_offsets[r] && row < rank_offsets[r + 1])",
         "if (row >= rank_offsets[r] && row <= rank_offsets[r + 1])"),
+    "e4m3_ties_to_odd_code": (
+        "pick = (lo & 1) ? (uint8_t)(lo + 1) : lo;",
+        "pick = (lo & 1) ? lo : (uint8_t)(lo + 1);"),
+    "fp8_scale_inverted": (
+        "scale[r] = amax > 0.0f ? amax / 448.0f : 1.0f;",
+        "scale[r] = amax > 0.0f ? 448.0f / amax : 1.0f;"),
+    "fp8_combine_drops_scale": (
+        "float coef = w[t * k + j] * eo_scale[row];",
+        "float coef = w[t * k + j];"),
     "widening_drops_low_bit": (
         "    uint32_t u = ((uint32_t)h) << 16;",
         "    uint32_t u = ((uint32_t)(h & 0xFFFEu)) << 16;"),
@@ -75,7 +84,8 @@ def test_pins_catch_mutant(name, tmp_path):
            "-k", "not full_workloads",
            os.path.join(ROOT, "tests", "test_oracle_partition.py"),
            os.path.join(ROOT, "tests", "test_oracle_layout.py"),
-           os.path.join(ROOT, "tests", "test_oracle_dispatch_combine.py")]
+           os.path.join(ROOT, "tests", "test_oracle_dispatch_combine.py"),
+           os.path.join(ROOT, "tests", "test_oracle_fp8.py")]
     res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode == 1, (
         f"mutant {name} passed every pin:\n{res.stdout[-2000:]}\n{res.stderr[-2000:]}")
