@@ -284,6 +284,8 @@ def main():
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")
     p.add_argument("--no-decoupled", action="store_true",
                    help="skip timing the pack/copy/unpack comparison path")
+    p.add_argument("--no-fp8", action="store_true",
+                   help="skip timing the fp8 (e4m3) payload path")
     p.add_argument("--no-agrs", action="store_true",
                    help="skip timing the all-gather / reduce-scatter comparison path")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -332,7 +334,7 @@ def main():
     class BufferSet:
         """One independent set of the step's inputs and outputs."""
 
-        def __init__(self, decoupled=False, agrs=False):
+        def __init__(self, decoupled=False, agrs=False, fp8=False):
             self.lay = buffers.DeviceLayout(cfg, dev)
             self.x = buffers.bf16_from_bits(d["x"], dev)
             self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
@@ -350,13 +352,22 @@ def main():
                 self.dxfer = torch.empty((rows, wl.H), **bf16)
                 self.csend = torch.empty((wl.T * wl.k, wl.H), **bf16)
                 self.cxfer = torch.empty((wl.T * wl.k, wl.H), **bf16)
+            if fp8:
+                rows = wl.T * wl.k
+                self.recv_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
+                self.recv_s = torch.empty(rows, dtype=torch.float32, device=dev)
+                self.eo_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
+                self.eo_s = torch.empty(rows, dtype=torch.float32, device=dev)
+                # expert outputs as an fp8 producer would emit them
+                capi.moe_quantize_rows_fp8(self.eo, rows, wl.H, self.eo_q, self.eo_s)
             if agrs:
                 self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
                 self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
 
     with_decoupled = not args.no_decoupled
     with_agrs = not args.no_agrs and wl.R <= capi.MOE_MAX_NODES
-    sets = [BufferSet(with_decoupled, with_agrs), BufferSet(with_decoupled, with_agrs)]
+    with_fp8 = not args.no_fp8 and wl.H % 8 == 0 and not wl.two_level
+    sets = [BufferSet(with_decoupled, with_agrs, with_fp8), BufferSet(with_decoupled, with_agrs, with_fp8)]
 
     def layout(b):
         capi.moe_layout(cfg, b.topk, b.lay.struct)
@@ -377,6 +388,11 @@ def main():
         capi.moe_dispatch_decoupled(dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
         capi.moe_combine_decoupled(dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
 
+    def fp8_step(b):
+        layout(b)
+        capi.moe_dispatch_fp8(cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
+        capi.moe_combine_fp8(cfg, b.lay.struct, b.eo_q, b.eo_s, b.w, b.y)
+
     def agrs_step(b):
         layout(b)
         capi.moe_dispatch_allgather(cfg, b.lay.struct, b.x, b.gathered, b.recv)
@@ -393,6 +409,8 @@ def main():
             decoupled_step(sets[i % 2])
         if with_agrs:
             agrs_step(sets[i % 2])
+        if with_fp8:
+            fp8_step(sets[i % 2])
     torch.cuda.synchronize()
     for b in sets:
         for lay in [b.lay] + ([b.dlay] if with_decoupled else []):
@@ -422,6 +440,8 @@ def main():
                                capture(lambda: decoupled_step(A)))
     if with_agrs:
         graphs["agrs"] = (capture(lambda: (agrs_step(A), agrs_step(B))), capture(lambda: agrs_step(A)))
+    if with_fp8:
+        graphs["fp8"] = (capture(lambda: (fp8_step(A), fp8_step(B))), capture(lambda: fp8_step(A)))
     for pair, single in graphs.values():
         pair.replay()
         single.replay()
@@ -450,6 +470,7 @@ def main():
         t_ld = timed("LD", K) / K
         dec_ms = timed("decoupled", K) if with_decoupled else None
         agrs_ms = timed("agrs", K) if with_agrs else None
+        fp8_ms = timed("fp8", K) if with_fp8 else None
     ms_per_step = total_ms / K
     t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
     for b in sets:
@@ -481,6 +502,17 @@ def main():
                 "fused_speedup": round(value / ag_value, 3),
                 "path": "layout + all-gather dispatch (R copies, per-rank select) + "
                         "reduce-scatter combine (per-rank fp32 partials, rank-order sum)"}
+
+    fp8 = None
+    if fp8_ms is not None:
+        fp8_bytes = 2 * (wl.T * wl.H * 2 + wl.T * wl.k * (wl.H + 4))
+        fp8 = {"value": round(job_gbs(fp8_bytes, world, K, fp8_ms * 1e-3), 2), "unit": "GB/s",
+               "ms_per_step": round(fp8_ms / K, 5),
+               "tokens_per_s": round(wl.T * world * K / (fp8_ms * 1e-3), 1),
+               "speedup_vs_bf16_step": round(total_ms / fp8_ms, 3),
+               "bytes_per_step": fp8_bytes,
+               "path": "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + "
+                       "fp8 combine (expert rows already e4m3)"}
 
     # end to end through the C ABI from pinned host buffers
     e2e_steps = args.e2e_steps or min(K, 50)
@@ -544,6 +576,7 @@ def main():
                          "peak_kind": f"{peak_src} copy bandwidth"},
             "decoupled_3pass": decoupled,
             "allgather_reducescatter": agrs,
+            "fp8_payload": fp8,
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},

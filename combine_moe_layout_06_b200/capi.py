@@ -49,7 +49,7 @@ ENTRY_POINTS = (
     "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
     "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
-    "moe_combine_reducescatter",
+    "moe_combine_reducescatter", "moe_quantize_rows_fp8", "moe_dispatch_fp8", "moe_combine_fp8",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -106,6 +106,9 @@ def lib() -> ctypes.CDLL:
     L.moe_layout_dispatch.argtypes = [C, P, LP, P, P, P, P]
     L.moe_dispatch_allgather.argtypes = [C, LP, P, P, P, P]
     L.moe_combine_reducescatter.argtypes = [C, LP, P, P, P, P, P]
+    L.moe_quantize_rows_fp8.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P]
+    L.moe_dispatch_fp8.argtypes = [C, LP, P, P, P, P]
+    L.moe_combine_fp8.argtypes = [C, LP, P, P, P, P, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -235,3 +238,22 @@ def moe_combine_reducescatter(cfg: MoeConfig, layout: MoeLayout, expert_out, top
                                            _ptr(expert_out), _ptr(topk_weights), _ptr(partial),
                                            _ptr(y), _stream(stream)),
            "moe_combine_reducescatter")
+
+
+def moe_quantize_rows_fp8(src, rows: int, hidden: int, q, scale, stream=None) -> None:
+    """bf16 rows -> e4m3 codes (uint8) plus one fp32 scale per row."""
+    _check(lib().moe_quantize_rows_fp8(_ptr(src), int(rows), int(hidden), _ptr(q), _ptr(scale),
+                                       _stream(stream)), "moe_quantize_rows_fp8")
+
+
+def moe_dispatch_fp8(cfg: MoeConfig, layout: MoeLayout, x, recv_q, recv_scale,
+                     stream=None) -> None:
+    _check(lib().moe_dispatch_fp8(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x), _ptr(recv_q),
+                                  _ptr(recv_scale), _stream(stream)), "moe_dispatch_fp8")
+
+
+def moe_combine_fp8(cfg: MoeConfig, layout: MoeLayout, eo_q, eo_scale, topk_weights, y,
+                    stream=None) -> None:
+    _check(lib().moe_combine_fp8(ctypes.byref(cfg), ctypes.byref(layout), _ptr(eo_q),
+                                 _ptr(eo_scale), _ptr(topk_weights), _ptr(y), _stream(stream)),
+           "moe_combine_fp8")

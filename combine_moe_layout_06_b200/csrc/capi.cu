@@ -318,4 +318,52 @@ moe_status_t moe_combine_reducescatter(const moe_config_t* c, const moe_layout_t
     return cuda_status(e);
 }
 
+moe_status_t moe_quantize_rows_fp8(const void* src, int64_t rows, int32_t hidden, void* q,
+                                   float* scale, void* stream) {
+    if (rows < 0 || hidden < 1) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (src == nullptr || q == nullptr || scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!moe::fp8_eligible(hidden, {src}, {q})) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_quantize_fp8(src, rows, hidden, nullptr, 1, rows, q, scale, nullptr,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch_fp8(const moe_config_t* c, const moe_layout_t* L, const void* x,
+                              void* recv_q, float* recv_scale, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (two_level(c)) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || recv_q == nullptr || recv_scale == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!moe::fp8_eligible(c->hidden, {x}, {recv_q})) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_quantize_fp8(x, c->num_tokens, c->hidden, L->slot, c->top_k,
+                                                c->num_tokens * (int64_t)c->top_k, recv_q,
+                                                recv_scale, L->error_word,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_combine_fp8(const moe_config_t* c, const moe_layout_t* L, const void* eo_q,
+                             const float* eo_scale, const float* topk_weights, void* y,
+                             void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (eo_q == nullptr || eo_scale == nullptr || topk_weights == nullptr || y == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!moe::fp8_eligible(c->hidden, {y}, {eo_q})) return MOE_ERR_INVALID_ARG;
+    moe::CombineParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.row_bytes = (size_t)c->hidden * 2;
+    p.slot = L->slot;
+    p.w = topk_weights;
+    p.err = L->error_word;
+    p.engine = engine_of(c->flags);
+    return cuda_status(moe::launch_combine_fp8(p, eo_q, eo_scale, y, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -1,0 +1,257 @@
+// fp8.cu -- fp8 (e4m3) payload for dispatch and combine.
+//
+// TensorRT-LLM PR #13888 (ConfigurableMoE commit) validates an fp8
+// low-precision combine at rtol 0.02 / atol 0.15.  Rows travel as OCP E4M3
+// codes with one fp32 scale per row: scale = amax / 448 (amax = the row's
+// largest |value|; a zero row uses scale 1) and code = e4m3(v * (448 / amax)),
+// rounded to nearest even and saturated to +-448 (cvt.rn.satfinite).  The
+// receive buffer then carries H bytes plus 4 per row instead of 2H.
+//
+//  quantize_fp8_kernel: one warp per source row; the first pass finds amax,
+//    the second converts 16-byte vectors of 8 bf16 values into 8 codes and
+//    stores them to every destination row: the row itself (row-wise
+//    quantization of expert outputs) or the token's k receive rows (fp8
+//    dispatch: quantize once, write k copies).
+//  combine_fp8_kernel: the fused combine on codes, coef_j = w[t][j] *
+//    scale[slot[t][j]] and acc = fma(coef_j, decode(code), acc) for j = 0 ..
+//    k-1 from +0, one RNE bf16 store.
+#include <cuda_fp8.h>
+
+#include "moe_kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+constexpr int kThreads = kWarpsPerCta * 32;
+
+// 8 floats -> 8 e4m3 codes (byte i = element i).
+__device__ __forceinline__ uint2 to_e4m3x8(const float (&f)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(f[2 * i], f[2 * i + 1]), __NV_SATFINITE,
+                                                  __NV_E4M3);
+    return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// 8 e4m3 codes -> 8 floats (exact).
+__device__ __forceinline__ void from_e4m3x8(uint2 c, float (&f)[8]) {
+    const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)(w[i >> 1] >> (16 * (i & 1)));
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        f[2 * i] = __half2float(__half(__half_raw{h.x}));
+        f[2 * i + 1] = __half2float(__half(__half_raw{h.y}));
+    }
+}
+
+struct Fp8Args {
+    const uint4* src;     // bf16 rows, 8 values per vector
+    uint2* q;             // e4m3 rows, 8 codes per vector
+    float* scale;         // one per destination row
+    const int* slot;      // nullptr: the destination of row r is row r
+    int64_t rows;         // source rows
+    int k;                // destinations per source row (slot mode)
+    int64_t rv;           // vectors per row (H / 8)
+    int64_t dst_rows;
+    int* err;
+};
+
+__global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    int errbits = 0;
+    for (int64_t r = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); r < a.rows; r += nw) {
+        int64_t dst = -1;
+        if (a.slot == nullptr) {
+            dst = lane == 0 ? r : -1;
+        } else if (lane < a.k) {
+            const int s = __ldg(a.slot + r * a.k + lane);
+            if (s >= 0 && s < a.dst_rows) dst = s;
+            else if (s != -1) errbits |= kErrBadLayout;
+        }
+        const uint4* src = a.src + r * a.rv;
+        uint32_t amax_bits = 0;
+        for (int64_t v = lane; v < a.rv; v += 32) {
+            float f[8];
+            unpack_bf16<uint4>(ld_stream(src + v), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax_bits = max(amax_bits, __float_as_uint(fabsf(f[e])));
+        }
+        amax_bits = __reduce_max_sync(kFullMask, amax_bits);
+        const float amax = __uint_as_float(amax_bits);
+        const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
+        const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+        const unsigned dmask = __ballot_sync(kFullMask, dst >= 0);
+        if (dst >= 0) a.scale[dst] = scale;
+        // every lane runs every pass (the destination shuffles need the warp)
+        for (int64_t v0 = 0; v0 < a.rv; v0 += 32) {
+            const int64_t v = v0 + lane;
+            const bool active = v < a.rv;
+            float f[8];
+            unpack_bf16<uint4>(active ? __ldg(src + v) : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
+            const uint2 code = to_e4m3x8(f);
+            unsigned m = dmask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int64_t d = __shfl_sync(kFullMask, dst, j);
+                if (active) a.q[d * a.rv + v] = code;
+            }
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+struct Fp8CombArgs {
+    const uint2* q;        // e4m3 expert rows
+    const float* scale;    // per expert row
+    const float* w;        // [T*k]
+    const int* slot;       // [T*k]
+    uint4* y;              // bf16 rows
+    int64_t T;
+    int k;
+    int64_t rv;            // 8-value vectors per row
+    int64_t q_rows;
+    int* err;
+};
+
+// Items are (token, chunk of 32*VPL vectors), a contiguous token-major range
+// per warp; lanes hold the token's slots and coefficients; up to 8 rows'
+// codes are loaded before their FMAs.
+template <int VPL>
+__global__ void __launch_bounds__(kThreads) combine_fp8_kernel(Fp8CombArgs a) {
+    constexpr int CHUNK = 32 * VPL;
+    constexpr int KB = 8;
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
+    const int64_t items = a.T * cpr;
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
+    int errbits = 0;
+    int64_t t_loaded = -1;
+    int s = -1;
+    float coef = 0.f;
+    for (int64_t item = ib; item < ie; ++item) {
+        const int64_t t = item / cpr;
+        const int64_t base = (item - t * cpr) * CHUNK;
+        if (t != t_loaded) {
+            s = -1;
+            coef = 0.f;
+            if (lane < a.k) {
+                s = __ldg(a.slot + t * a.k + lane);
+                if (s >= 0 && s < a.q_rows) coef = __ldg(a.w + t * a.k + lane) * __ldg(a.scale + s);
+                else {
+                    if (s != -1) errbits |= kErrBadLayout;
+                    s = -1;
+                }
+            }
+            t_loaded = t;
+        }
+        float acc[VPL][8];
+#pragma unroll
+        for (int i = 0; i < VPL; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+        for (int j0 = 0; j0 < a.k; j0 += KB) {
+            uint2 v[KB][VPL];
+            float cq[KB];
+            bool ok[KB];
+#pragma unroll
+            for (int q = 0; q < KB; ++q) {
+                const int j = j0 + q;
+                const int sj = __shfl_sync(kFullMask, s, j & 31);
+                cq[q] = __shfl_sync(kFullMask, coef, j & 31);
+                ok[q] = j < a.k && sj >= 0;
+                if (ok[q]) {
+#pragma unroll
+                    for (int i = 0; i < VPL; ++i) {
+                        const int64_t idx = base + i * 32 + lane;
+                        if (idx < a.rv) v[q][i] = ld_stream(a.q + (int64_t)sj * a.rv + idx);
+                    }
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < KB; ++q) {
+                if (!ok[q]) continue;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    if (base + i * 32 + lane < a.rv) {
+                        float f[8];
+                        from_e4m3x8(v[q][i], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[i][e] = __fmaf_rn(cq[q], f[e], acc[i][e]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int64_t idx = base + i * 32 + lane;
+            if (idx < a.rv) a.y[t * a.rv + idx] = pack_bf16<uint4>(acc[i]);
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+}  // namespace
+
+bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
+                  std::initializer_list<const void*> q_ptrs) {
+    if (hidden % 8 != 0) return false;
+    for (const void* p : bf16_ptrs)
+        if (reinterpret_cast<uintptr_t>(p) % 16) return false;
+    for (const void* p : q_ptrs)
+        if (reinterpret_cast<uintptr_t>(p) % 8) return false;
+    return true;
+}
+
+cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
+                                int64_t dst_rows, void* q, float* scale, int* err,
+                                cudaStream_t stream) {
+    if (rows <= 0) return cudaSuccess;
+    Fp8Args a;
+    a.src = static_cast<const uint4*>(src);
+    a.q = static_cast<uint2*>(q);
+    a.scale = scale;
+    a.slot = slot;
+    a.rows = rows;
+    a.k = k;
+    a.rv = hidden / 8;
+    a.dst_rows = dst_rows;
+    a.err = err;
+    constexpr auto kern = quantize_fp8_kernel;
+    const int grid = persistent_grid<kern>(rows, kThreads);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
+cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,
+                               cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    Fp8CombArgs a;
+    a.q = static_cast<const uint2*>(q);
+    a.scale = scale;
+    a.w = p.w;
+    a.slot = p.slot;
+    a.y = static_cast<uint4*>(y);
+    a.T = p.T;
+    a.k = p.k;
+    a.rv = (int64_t)(p.row_bytes / 16);
+    a.q_rows = p.T * p.k;
+    a.err = p.err;
+    constexpr auto kern = combine_fp8_kernel<2>;
+    const int64_t cpr = (a.rv + 63) / 64;
+    const int grid = persistent_grid<kern>(a.T * cpr, kThreads);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
+}  // namespace moe

@@ -71,6 +71,14 @@ __device__ __forceinline__ uint4 ld_stream<uint4>(const uint4* p) {
     return v;
 }
 template <>
+__device__ __forceinline__ uint2 ld_stream<uint2>(const uint2* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+template <>
 __device__ __forceinline__ uint32_t ld_stream<uint32_t>(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));

@@ -100,6 +100,19 @@ cudaError_t launch_combine_rank_partials(const CombineParams& p, int R, const in
 cudaError_t launch_reduce_rank_partials(const CombineParams& p, int R, const float* partial,
                                         void* y, cudaStream_t stream);
 
+// ---- fp8 (e4m3) payload (fp8.cu) ------------------------------------------------
+// hidden % 8 == 0, bf16 buffers 16-byte aligned, code buffers 8-byte aligned.
+bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
+                  std::initializer_list<const void*> q_ptrs);
+// Quantize `rows` bf16 rows (amax scale per row).  slot == nullptr: row r ->
+// q row r; else row r goes to q rows slot[r*k + j] (j < k), bounded by dst_rows.
+cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
+                                int64_t dst_rows, void* q, float* scale, int* err,
+                                cudaStream_t stream);
+// y[t] = bf16_rne(sum_j fma(w[t][j] * scale[slot], decode(q[slot]), .))
+cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,
+                               cudaStream_t stream);
+
 // ---- bulk-copy (TMA) engine (bulk.cu) ------------------------------------------
 // Usable when the row size and every base address are multiples of 16 bytes.
 bool bulk_eligible(size_t row_bytes, std::initializer_list<const void*> ptrs);

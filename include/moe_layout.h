@@ -265,6 +265,39 @@ moe_status_t moe_combine_reducescatter(const moe_config_t *cfg, const moe_layout
                                        const void *expert_out, const float *topk_weights,
                                        float *partial, void *y, void *stream);
 
+/* ---- fp8 (e4m3) payload ----
+ * TensorRT-LLM PR #13888 (ConfigurableMoE commit) validates an fp8
+ * low-precision combine at rtol 0.02 / atol 0.15.  Rows are carried as OCP
+ * E4M3 codes (1 byte per value) with one fp32 scale per row: scale = amax /
+ * 448 (a zero row uses 1) and code = e4m3(v * (448 / amax)), round to
+ * nearest even, saturated to +-448.  Requirements: hidden % 8 == 0, bf16
+ * buffers 16-byte aligned, code buffers 8-byte aligned (else
+ * MOE_ERR_INVALID_ARG). */
+
+/* Quantize `rows` bf16 rows of `hidden` values (e.g. expert outputs).
+ *   src    device bf16 [rows][hidden]
+ *   q      device uint8 [rows][hidden] e4m3 codes
+ *   scale  device fp32 [rows] */
+moe_status_t moe_quantize_rows_fp8(const void *src, int64_t rows, int32_t hidden, void *q,
+                                   float *scale, void *stream);
+
+/* Fused dispatch with an fp8 payload: each x row is quantized once and its
+ * codes and scale are written to all its receive rows (flat mode only;
+ * MOE_FLAG_TWO_LEVEL gives MOE_ERR_INVALID_ARG).
+ *   recv_q      device uint8 [T*k][H]
+ *   recv_scale  device fp32 [T*k] */
+moe_status_t moe_dispatch_fp8(const moe_config_t *cfg, const moe_layout_t *layout, const void *x,
+                              void *recv_q, float *recv_scale, void *stream);
+
+/* Fused combine of fp8 expert rows: coef_j = w[t][j] * scale[slot[t][j]]
+ * (fp32), acc = fma(coef_j, decode(code), acc) for j = 0..k-1 from +0, one
+ * bf16 round-to-nearest-even store.
+ *   eo_q      device uint8 [T*k][H] (receive-buffer layout)
+ *   eo_scale  device fp32 [T*k] */
+moe_status_t moe_combine_fp8(const moe_config_t *cfg, const moe_layout_t *layout,
+                             const void *eo_q, const float *eo_scale, const float *topk_weights,
+                             void *y, void *stream);
+
 /* ---- layout without caller-provided scratch ----
  * No counterpart on the pages: this entry point exists for callers that
  * cannot allocate device memory (for example code that runs while a stream

@@ -91,6 +91,10 @@ def _bind(path: str):
     lib.oracle_e4m3_to_f32.restype = ctypes.c_float
     lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
     lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.oracle_e4m3_to_f32_array.argtypes = [p, p, i64]
+    lib.oracle_e4m3_to_f32_array.restype = None
+    lib.oracle_f32_to_e4m3_array.argtypes = [p, p, i64]
+    lib.oracle_f32_to_e4m3_array.restype = None
     lib.oracle_quantize_rows_fp8.argtypes = [i64, i32, p, p, p]
     lib.oracle_quantize_rows_fp8.restype = None
     lib.oracle_dispatch_fp8.argtypes = [i64, i32, i32, p, p, p, p]
@@ -260,15 +264,19 @@ def combine_rank_partials(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray,
 # ---------------------------------------------------------------- fp8 payload
 
 def e4m3_to_f32(codes) -> np.ndarray:
+    """Decode e4m3 codes (flat result)."""
     codes = _c(codes, np.uint8).ravel()
-    L = _load()
-    return np.array([L.oracle_e4m3_to_f32(int(c)) for c in codes], np.float32)
+    out = np.empty(codes.size, np.float32)
+    _load().oracle_e4m3_to_f32_array(_ptr(codes), _ptr(out), codes.size)
+    return out
 
 
 def f32_to_e4m3(vals) -> np.ndarray:
+    """Encode to e4m3 codes (flat result)."""
     vals = _c(vals, np.float32).ravel()
-    L = _load()
-    return np.array([L.oracle_f32_to_e4m3(float(v)) for v in vals], np.uint8)
+    out = np.empty(vals.size, np.uint8)
+    _load().oracle_f32_to_e4m3_array(_ptr(vals), _ptr(out), vals.size)
+    return out
 
 
 def quantize_rows_fp8(src_bits: np.ndarray):

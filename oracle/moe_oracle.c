@@ -436,32 +436,54 @@ float oracle_e4m3_to_f32(uint8_t c)
 }
 
 /* Encode: round to nearest (ties to even code) over the finite e4m3 values,
- * saturating beyond 448; NaN maps to the NaN code. Written as a search over
- * the 127 non-negative finite codes, which are in increasing order. */
+ * saturating beyond 448; NaN maps to the NaN code.  The 127 non-negative
+ * finite codes decode to increasing values, so the code just below |f| is
+ * found by binary search over their decoded values. */
+static float e4m3_value[127];
+static int e4m3_value_ready = 0;
+
 uint8_t oracle_f32_to_e4m3(float f)
 {
+    if (!e4m3_value_ready) {
+        for (int c = 0; c < 127; ++c)
+            e4m3_value[c] = oracle_e4m3_to_f32((uint8_t)c);
+        e4m3_value_ready = 1;
+    }
     if (f != f)
         return 0x7F;
     uint8_t sign = signbit(f) ? 0x80 : 0x00;
     float a = fabsf(f);
     if (a >= 448.0f)
         return (uint8_t)(sign | 0x7E);
-    uint8_t lo = 0;
-    for (uint8_t c = 0; c < 0x7E; ++c)
-        if (oracle_e4m3_to_f32((uint8_t)(c + 1)) <= a)
-            lo = (uint8_t)(c + 1);
-    /* a lies in [val(lo), val(lo+1)) */
-    float vlo = oracle_e4m3_to_f32(lo);
-    float vhi = oracle_e4m3_to_f32((uint8_t)(lo + 1));
-    double dlo = (double)a - (double)vlo, dhi = (double)vhi - (double)a;
-    uint8_t pick;
+    int lo = 0, hi = 126;            /* invariant: value[lo] <= a < value[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (e4m3_value[mid] <= a)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    double dlo = (double)a - (double)e4m3_value[lo], dhi = (double)e4m3_value[hi] - (double)a;
+    int pick;
     if (dlo < dhi)
         pick = lo;
     else if (dhi < dlo)
-        pick = (uint8_t)(lo + 1);
+        pick = hi;
     else
-        pick = (lo & 1) ? (uint8_t)(lo + 1) : lo;   /* tie: even code */
+        pick = (lo & 1) ? hi : lo;   /* tie: even code */
     return (uint8_t)(sign | pick);
+}
+
+void oracle_e4m3_to_f32_array(const uint8_t *src, float *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = oracle_e4m3_to_f32(src[i]);
+}
+
+void oracle_f32_to_e4m3_array(const float *src, uint8_t *dst, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = oracle_f32_to_e4m3(src[i]);
 }
 
 /* Quantize `rows` bf16 rows of H values to e4m3 with one scale per row. */

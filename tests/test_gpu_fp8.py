@@ -1,0 +1,135 @@
+"""GPU parity of the fp8 (e4m3) payload against the oracle: codes and scales
+bit for bit (quantization, fp8 dispatch) and fp8 combine bit for bit (same
+FMA order).  Against the bf16 combine of the unquantized rows, the fp8
+result stays within e4m3's quantization bound for any magnitudes, and for
+unit-scale expert outputs within rtol 0.02 / atol 0.15, the tolerance
+TensorRT-LLM PR #13888 validates its fp8 combine with."""
+import numpy as np
+import pytest
+import torch
+
+import moe_testlib as M
+from combine_moe_layout_06_b200 import capi, inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # T, H, E, k, R
+    (1, 8, 4, 1, 1),
+    (33, 136, 13, 4, 5),
+    (257, 72, 64, 8, 4),
+    (300, 16, 32, 16, 8),      # k > 8, rows shorter than a warp's vectors
+    (1000, 2048, 60, 4, 7),
+]
+
+
+def _u8(t):
+    return t.detach().cpu().contiguous().numpy().view(np.uint8)
+
+
+def _assert_fp8_error_bound(y_bits, eo_bits, w, slot, scale_rows):
+    """|fp8 combine - bf16 combine| within the e4m3 quantization bound: each
+    term w_j x_j carries a relative error <= 2^-4 (3 mantissa bits, half an
+    ulp) plus, below e4m3's normal range, an absolute error <= scale * 2^-10;
+    both results carry a bf16 rounding (2^-8 relative) and fp32 sums."""
+    y = M.bf16_bits_to_f64(y_bits)
+    xf = M.bf16_bits_to_f64(eo_bits)
+    wf = w.astype(np.float64)
+    T, k = slot.shape
+    terms = np.stack([wf[:, j:j + 1] * np.abs(xf[slot[:, j]]) for j in range(k)], -1)
+    sub = np.stack([wf[:, j:j + 1] * scale_rows[slot[:, j]][:, None] for j in range(k)], -1)
+    exact = np.stack([wf[:, j:j + 1] * xf[slot[:, j]] for j in range(k)], -1).sum(-1)
+    bound = ((2.0 ** -4 + 2.0 ** -20) * terms.sum(-1) + 2.0 ** -10 * sub.sum(-1)
+             + 2 * 2.0 ** -8 * (np.abs(exact) + 2.0 ** -4 * terms.sum(-1)) + 1e-30)
+    ok = np.abs(y - exact) <= bound
+    assert ok.all(), f"outside the e4m3 error bound at {np.argwhere(~ok)[:5].tolist()}"
+
+
+def _run_fp8(cfg, lay, x_dev, eo_bits, w):
+    T, H, k = cfg.num_tokens, cfg.hidden, cfg.top_k
+    recv_q = torch.empty((T * k, H), dtype=torch.uint8, device="cuda")
+    recv_s = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    capi.moe_dispatch_fp8(cfg, lay.struct, x_dev, recv_q, recv_s)
+    eo_dev = M.to_dev(eo_bits)
+    eo_q = torch.empty((T * k, H), dtype=torch.uint8, device="cuda")
+    eo_s = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    capi.moe_quantize_rows_fp8(eo_dev, T * k, H, eo_q, eo_s)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    capi.moe_combine_fp8(cfg, lay.struct, eo_q, eo_s, torch.from_numpy(w).cuda(), y)
+    return recv_q, recv_s, eo_q, eo_s, y
+
+
+@pytest.mark.parametrize("T,H,E,k,R", CASES)
+def test_fp8_small(oracle_mod, T, H, E, k, R):
+    d = inputs.make_random(T, H, E, k, seed=T + H + 5)
+    x, topk, w = d["x"], d["topk_idx"], d["topk_w"]
+    ref = oracle_mod.layout(topk, E, R)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, topk)
+    eo = inputs.random_bf16_bits((T * k, H), seed=3 * T + H)
+    recv_q, recv_s, eo_q, eo_s, y = _run_fp8(cfg, lay, M.to_dev(x), eo, w)
+    rq, rs = oracle_mod.dispatch_fp8(x, ref["slot"])
+    assert np.array_equal(_u8(recv_q), rq)
+    assert np.array_equal(recv_s.cpu().numpy(), rs)
+    eq, es = oracle_mod.quantize_rows_fp8(eo)
+    assert np.array_equal(_u8(eo_q), eq)
+    assert np.array_equal(eo_s.cpu().numpy(), es)
+    y_bits = M.bits(y)
+    assert np.array_equal(y_bits, oracle_mod.combine_fp8(eq, es, w, ref["slot"]))
+    _assert_fp8_error_bound(y_bits, eo, w, ref["slot"], es.astype(np.float64))
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_fp8_zero_and_extreme_rows(oracle_mod):
+    T, H, E, k, R = 64, 32, 8, 2, 2
+    d = inputs.make_random(T, H, E, k, seed=1)
+    x = d["x"].copy()
+    x[3] = 0                                     # zero row: scale 1, codes 0
+    x[5, 7] = 0x7F7F                             # bf16 max: scale huge
+    x[6] = 0x0001                                # a bf16 subnormal row
+    ref = oracle_mod.layout(d["topk_idx"], E, R)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, d["topk_idx"])
+    eo = inputs.random_bf16_bits((T * k, H), seed=2)
+    recv_q, recv_s, _, _, _ = _run_fp8(cfg, lay, M.to_dev(x), eo, d["topk_w"])
+    rq, rs = oracle_mod.dispatch_fp8(x, ref["slot"])
+    assert np.array_equal(_u8(recv_q), rq)
+    assert np.array_equal(recv_s.cpu().numpy(), rs)
+
+
+def test_fp8_workload_olmoe(oracle_mod):
+    d = inputs.make("olmoe")
+    wl = d["workload"]
+    ref = oracle_mod.layout(d["topk_idx"], wl.E, wl.R)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R)
+    lay, _ = M.gpu_layout(cfg, d["topk_idx"])
+    eo = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
+    recv_q, recv_s, eo_q, eo_s, y = _run_fp8(cfg, lay, M.to_dev(d["x"]), eo, d["topk_w"])
+    rq, rs = oracle_mod.dispatch_fp8(d["x"], ref["slot"])
+    assert np.array_equal(_u8(recv_q), rq) and np.array_equal(recv_s.cpu().numpy(), rs)
+    eq, es = oracle_mod.quantize_rows_fp8(eo)
+    assert np.array_equal(_u8(eo_q), eq) and np.array_equal(eo_s.cpu().numpy(), es)
+    y_bits = M.bits(y)
+    assert np.array_equal(y_bits, oracle_mod.combine_fp8(eq, es, d["topk_w"], ref["slot"]))
+    _assert_fp8_error_bound(y_bits, eo, d["topk_w"], ref["slot"], es.astype(np.float64))
+    # unit-scale expert outputs: the pages' fp8 combine tolerance
+    eo_n = inputs.random_bf16((wl.T * wl.k, wl.H), seed=wl.seed + 8)
+    _, _, _, _, y_n = _run_fp8(cfg, lay, M.to_dev(d["x"]), eo_n, d["topk_w"])
+    M.assert_combine_close(M.bits(y_n), oracle_mod.combine(eo_n, d["topk_w"], ref["slot"]),
+                           rtol=0.02, atol=0.15)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_fp8_refusals():
+    cfg = M.cfg_of(4, 12, 8, 2, 2)                       # hidden % 8 != 0
+    lay, _ = M.gpu_layout(cfg, np.array([[0, 1], [2, 3], [4, 5], [6, 7]], np.int32))
+    x = torch.zeros((4, 12), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((8, 12), dtype=torch.uint8, device="cuda")
+    s = torch.empty(8, dtype=torch.float32, device="cuda")
+    with pytest.raises(capi.MoeError) as ei:
+        capi.moe_dispatch_fp8(cfg, lay.struct, x, q, s)
+    assert ei.value.status == capi.MOE_ERR_INVALID_ARG
+    two = M.cfg_of(4, 16, 8, 2, 2, 2, capi.MOE_FLAG_TWO_LEVEL)
+    with pytest.raises(capi.MoeError) as ei:
+        capi.moe_dispatch_fp8(two, lay.struct, x, q, s)
+    assert ei.value.status == capi.MOE_ERR_INVALID_ARG

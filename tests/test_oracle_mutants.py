@@ -55,8 +55,8 @@ MUTANTS = {
         "if (row >= rank_offsets[r] && row < rank_offsets[r + 1])",
         "if (row >= rank_offsets[r] && row <= rank_offsets[r + 1])"),
     "e4m3_ties_to_odd_code": (
-        "pick = (lo & 1) ? (uint8_t)(lo + 1) : lo;",
-        "pick = (lo & 1) ? lo : (uint8_t)(lo + 1);"),
+        "pick = (lo & 1) ? hi : lo;   /* tie: even code */",
+        "pick = (lo & 1) ? lo : hi;   /* tie: even code */"),
     "fp8_scale_inverted": (
         "scale[r] = amax > 0.0f ? amax / 448.0f : 1.0f;",
         "scale[r] = amax > 0.0f ? 448.0f / amax : 1.0f;"),
