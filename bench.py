@@ -116,6 +116,11 @@ def algorithmic_bytes(wl, tokens=None):
     return dispatch, combine
 
 
+# One hot node: DeepSeek-V3-shaped rows (H=7168, E=256, k=8, R=8) over
+# N=2 nodes, 90% of the tokens routing all k choices to node 0.
+NODE_SKEW = dict(T=16384, H=7168, E=256, k=8, R=8, N=2, hot_frac=0.9, seed=1240)
+
+
 def workload_desc(wl):
     return {
         "workload": f"{wl.name}: {inputs.DESCRIPTIONS[wl.name]}",
@@ -270,6 +275,94 @@ def hbm_probe():
 
 # ---------------------------------------------------------------- our arm
 
+def node_balance(args, dev, world, barrier, flags):
+    """Two-level dispatch on a hot-node routing (NODE_SKEW), with the second
+    phase walking (node, token) pairs (no node_src) and staging rows
+    (node_src given).  Same protocol as the main step: two buffer sets,
+    graphs of two steps, K steps between two events; dispatch = (layout +
+    dispatch) - layout."""
+    import torch
+
+    from combine_moe_layout_06_b200 import buffers, capi
+    sk = NODE_SKEW
+    T, H, E, k, R, N = (sk[c] for c in ("T", "H", "E", "k", "R", "N"))
+    d = inputs.make_node_skewed(T, H, E, k, N, sk["hot_frac"], sk["seed"])
+    cfg = capi.config(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | (flags & (
+        capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK)))
+    bf16 = dict(dtype=torch.bfloat16, device=dev)
+    rows = capi.moe_node_staging_rows(cfg)
+
+    class Set:
+        def __init__(self):
+            self.x = buffers.bf16_from_bits(d["x"], dev)
+            self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
+            self.recv = torch.empty((T * k, H), **bf16)
+            self.staging = torch.empty((rows, H), **bf16)
+            self.lay = {v: buffers.DeviceLayout(cfg, dev, node_src=v) for v in (False, True)}
+
+    sets = [Set(), Set()]
+
+    def ld(b, v):
+        capi.moe_layout_dispatch(cfg, b.topk, b.lay[v].struct, b.x, b.recv, b.staging)
+
+    def lo(b, v):
+        capi.moe_layout(cfg, b.topk, b.lay[v].struct)
+
+    for i in range(args.warmup):
+        for v in (False, True):
+            ld(sets[i % 2], v)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(dev)
+    A, B = sets
+    graphs = {}
+    for v in (False, True):
+        for name, fn in (("LD", ld), ("L", lo)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn(A, v)
+                fn(B, v)
+            graphs[(name, v)] = g
+    for g in graphs.values():
+        g.replay()
+    torch.cuda.synchronize()
+    K2 = max(args.steps // 2, 1)
+
+    def timed(key):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K2):
+            graphs[key].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) / (2 * K2)
+
+    out = {}
+    disp_b = T * H * 2 + T * k * H * 2
+    for v, name in ((False, "pairs"), (True, "rows")):
+        t_ld, t_l = timed(("LD", v)), timed(("L", v))
+        ms = t_ld - t_l
+        out[name] = {"dispatch_ms": round(ms, 5), "layout_ms": round(t_l, 5),
+                     "dispatch_gbs": round(disp_b * world / (ms * 1e-3) / 1e9, 2)}
+    for b in sets:
+        for v in (False, True):
+            st = capi.moe_get_error(b.lay[v].struct)
+            if st != capi.MOE_OK:
+                raise SystemExit(f"device error in the node-balance run: {capi.moe_status_string(st)}")
+    counts = sets[0].lay[True].node_counts.cpu().tolist()
+    graphs.clear()
+    return {"workload": f"DeepSeek-V3-shaped rows T={T} H={H} E={E} k={k} R={R} N={N}, "
+                        f"{int(sk['hot_frac'] * 100)}% of tokens send all k choices to node 0",
+            "node_counts": counts,
+            "pairs": out["pairs"], "rows": out["rows"],
+            "rows_speedup": round(out["pairs"]["dispatch_ms"] / out["rows"]["dispatch_ms"], 3),
+            "path": "two-level dispatch (node pack + node expansion); pairs: the expansion "
+                    "walks (node, token) pairs, rows: it walks staging rows (node_src)",
+            "bytes_per_step": disp_b}
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -288,6 +381,8 @@ def main():
                    help="skip timing the fp8 (e4m3) payload path")
     p.add_argument("--no-agrs", action="store_true",
                    help="skip timing the all-gather / reduce-scatter comparison path")
+    p.add_argument("--no-node-balance", action="store_true",
+                   help="skip timing the two node expansions on a hot-node routing")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=0)
@@ -388,9 +483,12 @@ def main():
         capi.moe_dispatch_decoupled(dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
         capi.moe_combine_decoupled(dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
 
-    def fp8_step(b):
+    def fp8_layout_dispatch(b):
         layout(b)
         capi.moe_dispatch_fp8(cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
+
+    def fp8_step(b):
+        fp8_layout_dispatch(b)
         capi.moe_combine_fp8(cfg, b.lay.struct, b.eo_q, b.eo_s, b.w, b.y)
 
     def agrs_step(b):
@@ -442,6 +540,8 @@ def main():
         graphs["agrs"] = (capture(lambda: (agrs_step(A), agrs_step(B))), capture(lambda: agrs_step(A)))
     if with_fp8:
         graphs["fp8"] = (capture(lambda: (fp8_step(A), fp8_step(B))), capture(lambda: fp8_step(A)))
+        graphs["fp8_LD"] = (capture(lambda: (fp8_layout_dispatch(A), fp8_layout_dispatch(B))),
+                            capture(lambda: fp8_layout_dispatch(A)))
     for pair, single in graphs.values():
         pair.replay()
         single.replay()
@@ -471,6 +571,7 @@ def main():
         dec_ms = timed("decoupled", K) if with_decoupled else None
         agrs_ms = timed("agrs", K) if with_agrs else None
         fp8_ms = timed("fp8", K) if with_fp8 else None
+        fp8_ld = timed("fp8_LD", K) / K if with_fp8 else None
     ms_per_step = total_ms / K
     t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
     for b in sets:
@@ -510,9 +611,18 @@ def main():
                "ms_per_step": round(fp8_ms / K, 5),
                "tokens_per_s": round(wl.T * world * K / (fp8_ms * 1e-3), 1),
                "speedup_vs_bf16_step": round(total_ms / fp8_ms, 3),
+               "kernels_ms": {"dispatch": round(fp8_ld - t_l, 5),
+                              "combine": round(fp8_ms / K - fp8_ld, 5)},
                "bytes_per_step": fp8_bytes,
                "path": "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + "
                        "fp8 combine (expert rows already e4m3)"}
+
+    graphs.clear()
+    balance = None
+    if not args.no_node_balance:
+        with ClockSampler(local) as nb_clocks:
+            balance = node_balance(args, dev, world, barrier, flags)
+        balance["clocks"] = nb_clocks.summary()
 
     # end to end through the C ABI from pinned host buffers
     e2e_steps = args.e2e_steps or min(K, 50)
@@ -577,6 +687,7 @@ def main():
             "decoupled_3pass": decoupled,
             "allgather_reducescatter": agrs,
             "fp8_payload": fp8,
+            "node_balance": balance,
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -584,7 +695,6 @@ def main():
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    graphs.clear()
     if world > 1:
         dist.destroy_process_group()
     return 0

@@ -11,9 +11,12 @@ from . import capi
 
 
 class DeviceLayout:
-    """The moe_layout_t arrays of one configuration, plus its workspace."""
+    """The moe_layout_t arrays of one configuration, plus its workspace.
 
-    def __init__(self, cfg: capi.MoeConfig, device="cuda"):
+    ``node_src`` (two-level only): also allocate the staging-row -> token map,
+    which makes the second dispatch phase divide its work by staging rows."""
+
+    def __init__(self, cfg: capi.MoeConfig, device="cuda", node_src: bool = True):
         T, k, E, R, N = cfg.num_tokens, cfg.top_k, cfg.num_experts, cfg.num_ranks, cfg.num_nodes
         i32 = dict(dtype=torch.int32, device=device)
         self.cfg = cfg
@@ -29,11 +32,14 @@ class DeviceLayout:
             self.node_counts = torch.zeros(N, **i32)
             self.node_offsets = torch.zeros(N + 1, **i32)
             self.node_slot = torch.zeros(T * N, **i32)
+            self.node_src = (torch.full((max(capi.moe_node_staging_rows(cfg), 1),), -1, **i32)
+                             if node_src else None)
         else:
-            self.node_counts = self.node_offsets = self.node_slot = None
+            self.node_counts = self.node_offsets = self.node_slot = self.node_src = None
         self.struct = capi.layout_struct(
             self.expert_counts, self.expert_offsets, self.rank_offsets, self.slot,
-            self.error_word, self.workspace, self.node_counts, self.node_offsets, self.node_slot)
+            self.error_word, self.workspace, self.node_counts, self.node_offsets, self.node_slot,
+            self.node_src)
 
     def host(self) -> dict:
         """Copy of the arrays on the host (numpy), shaped like the oracle's."""
@@ -48,6 +54,9 @@ class DeviceLayout:
             out["node_counts"] = self.node_counts.cpu().numpy()
             out["node_offsets"] = self.node_offsets.cpu().numpy()
             out["node_slot"] = self.node_slot.cpu().numpy().reshape(cfg.num_tokens, cfg.num_nodes)
+            if self.node_src is not None:
+                U = int(out["node_offsets"][cfg.num_nodes])
+                out["node_src"] = self.node_src[:U].cpu().numpy()
         return out
 
 

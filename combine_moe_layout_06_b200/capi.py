@@ -65,7 +65,7 @@ class MoeConfig(ctypes.Structure):
 class MoeLayout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "expert_counts", "expert_offsets", "rank_offsets", "slot", "node_counts",
-        "node_offsets", "node_slot", "error_word", "workspace")]
+        "node_offsets", "node_slot", "error_word", "workspace", "node_src")]
 
 
 class MoeError(RuntimeError):
@@ -169,10 +169,11 @@ def moe_node_staging_rows(cfg: MoeConfig) -> int:
 
 
 def layout_struct(expert_counts, expert_offsets, rank_offsets, slot, error_word, workspace,
-                  node_counts=None, node_offsets=None, node_slot=None) -> MoeLayout:
+                  node_counts=None, node_offsets=None, node_slot=None,
+                  node_src=None) -> MoeLayout:
     return MoeLayout(_ptr(expert_counts), _ptr(expert_offsets), _ptr(rank_offsets), _ptr(slot),
                      _ptr(node_counts), _ptr(node_offsets), _ptr(node_slot), _ptr(error_word),
-                     _ptr(workspace))
+                     _ptr(workspace), _ptr(node_src))
 
 
 def moe_layout(cfg: MoeConfig, topk_idx, layout: MoeLayout, stream=None) -> None:

@@ -24,6 +24,7 @@
 // Every mbarrier wait is bounded; a wait that gives up records kErrTimeout,
 // stops issuing work, drains what it started and returns.  No load uses
 // cluster multicast.  Requires 16-byte aligned rows and base addresses.
+#include <climits>
 #include <initializer_list>
 
 #include "moe_kernels.h"
@@ -51,7 +52,7 @@ constexpr uint32_t kDispChunk = MOE_BULK_DISP_CHUNK;
 constexpr int kCombStages = MOE_BULK_COMB_STAGES;
 constexpr uint32_t kCombStageBytes = MOE_BULK_COMB_STAGE_BYTES;  // k row chunks per stage
 
-enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2 };
+enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2, kNodeRows = 3 };
 
 struct BulkArgs {
     const char* src;
@@ -61,6 +62,7 @@ struct BulkArgs {
     const int* node_slot;
     const int* node_offsets;
     const int* rank_offsets;
+    const int* node_src;      // [U] staging row -> token (kNodeRows)
     int64_t T;
     int k, N, ranks_per_node;
     int64_t row_bytes;
@@ -94,18 +96,31 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
     __syncwarp();
     // Flat and node-pack sources are x rows, which need no layout data: with
     // early inputs the first stages are loaded while the layout still runs.
-    const bool early = a.early != 0 && MODE != kNodeExpand;
+    const bool early = a.early != 0 && (MODE == kFlat || MODE == kNodePack);
     pdl_trigger();
     if (!early) pdl_wait();
 
-    const int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
+    int errbits = 0;
+    int64_t rows = MODE == kNodeExpand ? a.T * a.N : a.T;
+    // node-rows: lane n < N holds node n's first staging row and receive-row
+    // range; the rows to move are the node_offsets[N] the layout filled
+    int n_first = INT_MAX, n_lo = 0, n_hi = 0;
+    if (MODE == kNodeRows) {
+        if (lane < a.N) {
+            n_first = ld_dep(a.node_offsets + lane);
+            n_lo = ld_dep(a.rank_offsets + lane * a.ranks_per_node);
+            n_hi = ld_dep(a.rank_offsets + (lane + 1) * a.ranks_per_node);
+        }
+        const int64_t U = ld_dep(a.node_offsets + a.N);
+        rows = U < 0 ? 0 : (U > a.src_rows ? a.src_rows : U);
+        if (rows != U) errbits |= kErrBadLayout;
+    }
     const int64_t items = rows * a.cpr;
     // a contiguous, row-major range of items per warp
     const int64_t nwarps = (int64_t)gridDim.x * kBulkWarps;
     const int64_t gw = (int64_t)blockIdx.x * kBulkWarps + warp;
     const int64_t first = items * gw / nwarps;
     const int64_t mine = items * (gw + 1) / nwarps - first;
-    int errbits = 0;
 
     // Source row of an item (-1: nothing to move), and the chunk geometry.
     auto source = [&](int64_t item, int64_t& row, int64_t& base, uint32_t& bytes) -> int64_t {
@@ -113,12 +128,12 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
         base = (item - row * a.cpr) * (int64_t)a.chunk;
         const int64_t left = a.row_bytes - base;
         bytes = left < (int64_t)a.chunk ? (uint32_t)left : a.chunk;
-        if (MODE != kNodeExpand) return row;
+        if (MODE != kNodeExpand) return row;  // node-rows: the staging row itself
         const int n = (int)(row / a.T);
         const int64_t t = row - (int64_t)n * a.T;
-        const int ns = __ldg(a.node_slot + t * a.N + n);
+        const int ns = ld_dep(a.node_slot + t * a.N + n);
         if (ns < 0) return -1;
-        const int64_t r = (int64_t)__ldg(a.node_offsets + n) + ns;
+        const int64_t r = (int64_t)ld_dep(a.node_offsets + n) + ns;
         return (r >= 0 && r < a.src_rows) ? r : -2;
     };
     auto issue = [&](int64_t q) {
@@ -160,26 +175,38 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
         if (src_row >= 0) {
             if (MODE == kFlat) {
                 if (lane < a.k) {
-                    const int sl = __ldg(a.slot + row * a.k + lane);
+                    const int sl = ld_dep(a.slot + row * a.k + lane);
                     if (sl >= 0 && sl < a.dst_rows) dst = sl;
                     else if (sl != -1) errbits |= kErrBadLayout;
                 }
             } else if (MODE == kNodePack) {
                 if (lane < a.N) {
-                    const int ns = __ldg(a.node_slot + row * a.N + lane);
+                    const int ns = ld_dep(a.node_slot + row * a.N + lane);
                     if (ns >= 0) {
-                        const int64_t d = (int64_t)__ldg(a.node_offsets + lane) + ns;
+                        const int64_t d = (int64_t)ld_dep(a.node_offsets + lane) + ns;
                         if (d >= 0 && d < a.dst_rows) dst = d;
                         else errbits |= kErrBadLayout;
                     }
                 }
+            } else if (MODE == kNodeRows) {
+                // the node of staging row `row`: the last node starting at or before it
+                const int n = __popc(__ballot_sync(kFullMask, n_first <= row)) - 1;
+                const int lo = __shfl_sync(kFullMask, n_lo, n & 31);
+                const int hi = __shfl_sync(kFullMask, n_hi, n & 31);
+                const int t = ld_dep(a.node_src + row);
+                if (n < 0 || t < 0 || t >= a.T) {
+                    errbits |= kErrBadLayout;
+                } else if (lane < a.k) {
+                    const int sl = ld_dep(a.slot + (int64_t)t * a.k + lane);
+                    if (sl >= lo && sl < hi && sl < a.dst_rows) dst = sl;
+                }
             } else {
                 const int n = (int)(row / a.T);
                 const int64_t t = row - (int64_t)n * a.T;
-                const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
-                const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
+                const int lo = ld_dep(a.rank_offsets + n * a.ranks_per_node);
+                const int hi = ld_dep(a.rank_offsets + (n + 1) * a.ranks_per_node);
                 if (lane < a.k) {
-                    const int sl = __ldg(a.slot + t * a.k + lane);
+                    const int sl = ld_dep(a.slot + t * a.k + lane);
                     if (sl >= lo && sl < hi && sl < a.dst_rows) dst = sl;
                 }
             }
@@ -232,7 +259,7 @@ __global__ void __launch_bounds__(kBulkThreads) combine_bulk_kernel(BulkArgs a) 
     auto row_of = [&](int64_t t) -> int {
         int s = -1;
         if (lane < a.k) {
-            s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
+            s = a.slot ? ld_dep(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
             if (s < 0 || s >= eo_rows) {
                 if (s != -1) errbits |= kErrBadLayout;
                 s = -1;
@@ -274,7 +301,7 @@ __global__ void __launch_bounds__(kBulkThreads) combine_bulk_kernel(BulkArgs a) 
         geometry(first + q, t, base, bytes);
         const int s = row_of(t);
         const unsigned valid = __ballot_sync(kFullMask, s >= 0);
-        const float wl = lane < a.k ? __ldg(a.w + t * a.k + lane) : 0.f;
+        const float wl = lane < a.k ? ld_dep(a.w + t * a.k + lane) : 0.f;
         const unsigned char* stage = stage0 + (size_t)st * stage_bytes;
         char* yrow = a.dst + t * a.row_bytes + base;
         const int nvec = (int)(bytes >> 4);
@@ -326,6 +353,7 @@ BulkArgs bulk_args(const RowMoveParams& p, const void* src, void* dst, int64_t s
     a.node_slot = p.node_slot;
     a.node_offsets = p.node_offsets;
     a.rank_offsets = p.rank_offsets;
+    a.node_src = p.node_src;
     a.T = p.T;
     a.k = p.k;
     a.N = p.N;
@@ -369,6 +397,7 @@ cudaError_t launch_node_pack_bulk(const RowMoveParams& p, const void* x, void* s
 cudaError_t launch_node_expand_bulk(const RowMoveParams& p, const void* staging,
                                     int64_t staging_rows, void* recv, cudaStream_t stream) {
     const BulkArgs a = bulk_args(p, staging, recv, staging_rows, p.T * p.k, kDispChunk);
+    if (p.node_src != nullptr) return launch_disp_bulk<kNodeRows>(a, staging_rows, stream);
     return launch_disp_bulk<kNodeExpand>(a, p.T * p.N, stream);
 }
 

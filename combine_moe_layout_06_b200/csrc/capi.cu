@@ -49,6 +49,7 @@ moe::RowMoveParams move_params(const moe_config_t* c, const moe_layout_t* L) {
     p.node_slot = L->node_slot;
     p.node_offsets = L->node_offsets;
     p.rank_offsets = L->rank_offsets;
+    p.node_src = L->node_src;
     p.err = L->error_word;
     p.engine = engine_of(c->flags);
     return p;
@@ -168,6 +169,7 @@ moe_status_t moe_layout(const moe_config_t* c, const int32_t* topk_idx, const mo
     p.node_counts = L->node_counts;
     p.node_offsets = L->node_offsets;
     p.node_slot = L->node_slot;
+    p.node_src = L->node_src;
     p.err = L->error_word;
     p.workspace = L->workspace;
     return cuda_status(moe::launch_layout(p, static_cast<cudaStream_t>(stream)));

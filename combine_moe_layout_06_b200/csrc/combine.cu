@@ -53,8 +53,8 @@ __device__ __forceinline__ void load_route(const CombArgs& a, int64_t t, int lan
     s = -1;
     w = 0.f;
     if (lane < a.k) {
-        s = a.slot ? __ldg(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
-        w = __ldg(a.w + t * a.k + lane);
+        s = a.slot ? ld_dep(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
+        w = ld_dep(a.w + t * a.k + lane);
     }
     const bool ok = s >= 0 && s < a.eo_rows;
     bad |= (!ok && s != -1) ? kErrBadLayout : 0;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) rank_partial_kernel(RankArgs ra) {
         const int64_t base = (item - row * cpr) * 32;
         const int r = (int)(row / a.T);
         const int64_t t = row - (int64_t)r * a.T;
-        const int lo = __ldg(ra.rank_offsets + r), hi = __ldg(ra.rank_offsets + r + 1);
+        const int lo = ld_dep(ra.rank_offsets + r), hi = ld_dep(ra.rank_offsets + r + 1);
         int s = -1;
         float wl = 0.f;
         load_route(a, t, lane, s, wl, errbits);

@@ -15,6 +15,7 @@
 // to what is resident.  Lanes hold the destination rows (k <= 32 slots, or
 // N <= 32 nodes); the chunk is loaded once with streaming loads and stored
 // to every destination with evict-first stores.
+#include <climits>
 #include <initializer_list>
 
 #include "moe_kernels.h"
@@ -39,7 +40,7 @@ namespace {
 constexpr int kWarpsPerCta = 8;
 constexpr int kThreads = kWarpsPerCta * 32;
 
-enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2, kAllGather = 3, kRankSelect = 4 };
+enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2, kAllGather = 3, kRankSelect = 4, kNodeRows = 5 };
 
 struct FanArgs {
     const void* src;
@@ -48,6 +49,7 @@ struct FanArgs {
     const int* node_slot;
     const int* node_offsets;
     const int* rank_offsets;
+    const int* node_src;  // [U] staging row -> token (kNodeRows)
     int64_t T;
     int k, N, ranks_per_node;
     int64_t rv;        // vectors per row
@@ -57,7 +59,9 @@ struct FanArgs {
 };
 
 // Flat and node-pack rows are tokens; node-expand rows are (node, token)
-// pairs, node-major, so each node's forwarder work is one contiguous run.
+// pairs, node-major, so each node's forwarder work is one contiguous run;
+// node-rows rows are staging rows, so every warp gets the same number of
+// staging rows whatever the nodes' loads (load-aware forwarding).
 //
 // Where row r's data comes from and goes to: the source row (-1 = nothing to
 // move) and, per lane, one destination row (-1 = none).  Computed without
@@ -69,21 +73,44 @@ struct RowPlan {
     int bad;
 };
 
+// Per-lane node table of the node-rows mode, loaded once per warp: lane
+// n < N holds node n's first staging row and its receive-row range.
+struct NodeTable {
+    int first;
+    int lo, hi;
+};
+
+__device__ __forceinline__ NodeTable load_node_table(const FanArgs& a, int lane) {
+    NodeTable nt;
+    const bool on = lane < a.N;
+    nt.first = on ? ld_dep(a.node_offsets + lane) : INT_MAX;
+    nt.lo = on ? ld_dep(a.rank_offsets + lane * a.ranks_per_node) : 0;
+    nt.hi = on ? ld_dep(a.rank_offsets + (lane + 1) * a.ranks_per_node) : 0;
+    return nt;
+}
+
+// Node of staging row u: the last node whose first row is <= u (node
+// offsets ascend; an empty node shares its first row with the next one).
+__device__ __forceinline__ int node_of_row(const NodeTable& nt, int64_t u) {
+    return __popc(__ballot_sync(kFullMask, nt.first <= u)) - 1;
+}
+
 template <int MODE>
-__device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int lane) {
+__device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int lane,
+                                            const NodeTable& nt) {
     RowPlan p;
     p.dst = -1;
     p.bad = 0;
     if (MODE == kFlat) {
         p.src = row;
-        const int s = lane < a.k ? __ldg(a.slot + row * a.k + lane) : -1;
+        const int s = lane < a.k ? ld_dep(a.slot + row * a.k + lane) : -1;
         const bool ok = s >= 0 && s < a.dst_rows;
         p.dst = ok ? s : -1;
         p.bad = (!ok && s != -1) ? kErrBadLayout : 0;
     } else if (MODE == kNodePack) {
         p.src = row;
-        const int ns = lane < a.N ? __ldg(a.node_slot + row * a.N + lane) : -1;
-        const int64_t off = lane < a.N ? (int64_t)__ldg(a.node_offsets + lane) : 0;
+        const int ns = lane < a.N ? ld_dep(a.node_slot + row * a.N + lane) : -1;
+        const int64_t off = lane < a.N ? (int64_t)ld_dep(a.node_offsets + lane) : 0;
         const int64_t d = off + ns;
         const bool ok = ns >= 0 && d >= 0 && d < a.dst_rows;
         p.dst = ok ? d : -1;
@@ -96,19 +123,30 @@ __device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int l
         // rank r keeps, from its gathered copy, the token's rows on its experts
         const int r = (int)(row / a.T);
         const int64_t t = row - (int64_t)r * a.T;
-        const int lo = __ldg(a.rank_offsets + r);
-        const int hi = __ldg(a.rank_offsets + r + 1);
-        const int s = lane < a.k ? __ldg(a.slot + t * a.k + lane) : -1;
+        const int lo = ld_dep(a.rank_offsets + r);
+        const int hi = ld_dep(a.rank_offsets + r + 1);
+        const int s = lane < a.k ? ld_dep(a.slot + t * a.k + lane) : -1;
         p.src = row;
+        p.dst = (s >= lo && s < hi && s < a.dst_rows) ? s : -1;
+    } else if (MODE == kNodeRows) {
+        // staging row `row` holds token node_src[row] for node n
+        const int n = node_of_row(nt, row);
+        const int lo = __shfl_sync(kFullMask, nt.lo, n & 31);
+        const int hi = __shfl_sync(kFullMask, nt.hi, n & 31);
+        const int t = ld_dep(a.node_src + row);  // same for all lanes
+        const bool src_ok = n >= 0 && t >= 0 && t < a.T;
+        const int s = (src_ok && lane < a.k) ? ld_dep(a.slot + (int64_t)t * a.k + lane) : -1;
+        p.src = src_ok ? row : -1;
+        p.bad = src_ok ? 0 : kErrBadLayout;
         p.dst = (s >= lo && s < hi && s < a.dst_rows) ? s : -1;
     } else {
         const int n = (int)(row / a.T);
         const int64_t t = row - (int64_t)n * a.T;
-        const int ns = __ldg(a.node_slot + t * a.N + n);  // same for all lanes
-        const int64_t srow = (int64_t)__ldg(a.node_offsets + n) + ns;
-        const int lo = __ldg(a.rank_offsets + n * a.ranks_per_node);
-        const int hi = __ldg(a.rank_offsets + (n + 1) * a.ranks_per_node);
-        const int s = lane < a.k ? __ldg(a.slot + t * a.k + lane) : -1;
+        const int ns = ld_dep(a.node_slot + t * a.N + n);  // same for all lanes
+        const int64_t srow = (int64_t)ld_dep(a.node_offsets + n) + ns;
+        const int lo = ld_dep(a.rank_offsets + n * a.ranks_per_node);
+        const int hi = ld_dep(a.rank_offsets + (n + 1) * a.ranks_per_node);
+        const int s = lane < a.k ? ld_dep(a.slot + t * a.k + lane) : -1;
         const bool src_ok = ns >= 0 && srow >= 0 && srow < a.src_rows;
         p.src = src_ok ? srow : -1;
         p.bad = (ns >= 0 && !src_ok) ? kErrBadLayout : 0;
@@ -126,21 +164,29 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t rows = (MODE == kNodeExpand || MODE == kRankSelect) ? a.T * a.N : a.T;
+    int errbits = 0;
+    int64_t rows = (MODE == kNodeExpand || MODE == kRankSelect) ? a.T * a.N : a.T;
+    NodeTable nt = {INT_MAX, 0, 0};
+    if (MODE == kNodeRows) {
+        // the staging rows the layout filled: node_offsets[N], read here
+        nt = load_node_table(a, lane);
+        const int64_t U = ld_dep(a.node_offsets + a.N);
+        rows = U < 0 ? 0 : (U > a.src_rows ? a.src_rows : U);
+        if (rows != U) errbits |= kErrBadLayout;
+    }
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = rows * cpr;
     const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
     const int64_t gw = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
     const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
-    int errbits = 0;
     if (ib < ie) {
         int64_t row = ib / cpr;
         int64_t c = ib - row * cpr;
-        RowPlan cur = plan_row<MODE>(a, row, lane);
+        RowPlan cur = plan_row<MODE>(a, row, lane, nt);
         RowPlan nxt = cur;
         for (int64_t item = ib; item < ie; ++item) {
             const bool last_chunk = c + 1 == cpr;
-            if (last_chunk && item + 1 < ie) nxt = plan_row<MODE>(a, row + 1, lane);
+            if (last_chunk && item + 1 < ie) nxt = plan_row<MODE>(a, row + 1, lane, nt);
             if (cur.src >= 0) {
                 const int64_t base = c * CHUNK;
                 const V* src = static_cast<const V*>(a.src) + cur.src * a.rv + base;
@@ -191,7 +237,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(FanArgs a) {
     for (int64_t item = ib; item < ie; ++item) {
         const int64_t drow = item / cpr;
         const int64_t base = (item - drow * cpr) * CHUNK;
-        const int s = __ldg(a.slot + drow);   // same for all lanes
+        const int s = ld_dep(a.slot + drow);   // same for all lanes
         if (s < 0 || s >= a.src_rows) {
             if (s != -1) errbits |= kErrBadLayout;
             continue;
@@ -212,14 +258,14 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(FanArgs a) {
 // Contiguous copy of `rows` rows; the row count may live in device memory
 // (the decoupled path's transfer size is known only on the device).
 template <typename V>
-__global__ void __launch_bounds__(kThreads) copy_kernel(const V* __restrict__ src, V* __restrict__ dst,
+__global__ void __launch_bounds__(kThreads) copy_kernel(const V* src, V* dst,
                                                         const int* rows_dev, int64_t max_rows,
                                                         int64_t rv) {
     pdl_trigger();
     pdl_wait();
     int64_t rows = max_rows;
     if (rows_dev != nullptr) {
-        const int64_t r = *rows_dev;
+        const int64_t r = ld_dep(rows_dev);
         rows = r < 0 ? 0 : (r < max_rows ? r : max_rows);
     }
     const int64_t n = rows * rv;
@@ -286,6 +332,7 @@ FanArgs fan_args(const RowMoveParams& p, const void* src, void* dst, int64_t src
     a.node_slot = p.node_slot;
     a.node_offsets = p.node_offsets;
     a.rank_offsets = p.rank_offsets;
+    a.node_src = p.node_src;
     a.T = p.T;
     a.k = p.k;
     a.N = p.N;
@@ -324,6 +371,7 @@ cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging, int6
     if (use_bulk(p, {staging, recv}))
         return launch_node_expand_bulk(p, staging, staging_rows, recv, stream);
     FanArgs a = fan_args(p, staging, recv, staging_rows, p.T * p.k);
+    if (p.node_src != nullptr) return launch_fan<kNodeRows>(a, staging_rows, stream);
     return launch_fan<kNodeExpand>(a, p.T * p.N, stream);
 }
 

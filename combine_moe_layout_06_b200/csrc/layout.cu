@@ -70,6 +70,7 @@ struct LayoutArgs {
     int* node_counts;
     int* node_offsets;
     int* node_slot;
+    int* node_src;  // [U] staging row -> token, or nullptr
     int* err;
 };
 
@@ -90,7 +91,7 @@ __device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t 
     for (int j = 0; j < KMAX; ++j) {
         int v = -1;
         if (j < k) {
-            v = __ldg(row + j);
+            v = ld_dep(row + j);
             if (v < 0 || v >= E) {
                 bits |= kErrExpertOob;
                 v = -1;
@@ -99,7 +100,7 @@ __device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t 
                 if (seen & bit) {
                     bool repeat = false;
 #pragma unroll 1
-                    for (int i = 0; i < j; ++i) repeat |= __ldg(row + i) == v;
+                    for (int i = 0; i < j; ++i) repeat |= ld_dep(row + i) == v;
                     if (repeat) {
                         bits |= kErrDupExpert;
                         v = -1;
@@ -317,11 +318,17 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs
         }
     }
     if (a.nodes) {
+        // lane n: first staging row of node n (the scanned node histogram)
+        const int noff = (a.node_src && lane < a.N) ? a.ncnt[(int64_t)lane * a.C] : 0;
         for (int n = 0; n < a.N; ++n) {
             const bool touched = (nm >> n) & 1u;
             const unsigned b = __ballot_sync(kFullMask, touched);
-            if (t < a.T)
-                a.node_slot[t * a.N + n] = touched ? s_wn[warp * a.N + n] + __popc(b & lt) : -1;
+            const int ns = touched ? s_wn[warp * a.N + n] + __popc(b & lt) : -1;
+            const int off = __shfl_sync(kFullMask, noff, n);
+            if (t < a.T) {
+                a.node_slot[t * a.N + n] = ns;
+                if (a.node_src && touched) a.node_src[off + ns] = (int)t;
+            }
         }
     }
 }
@@ -533,7 +540,11 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
         for (int n = 0; n < N; ++n) {
             const bool touched = (nm >> n) & 1u;
             const unsigned b = __ballot_sync(kFullMask, touched);
-            if (t < a.T) a.node_slot[t * N + n] = touched ? s_wn[warp * N + n] + __popc(b & lt) : -1;
+            const int ns = touched ? s_wn[warp * N + n] + __popc(b & lt) : -1;
+            if (t < a.T) {
+                a.node_slot[t * N + n] = ns;
+                if (a.node_src && touched) a.node_src[tot[E + n] + ns] = (int)t;
+            }
         }
     }
 }
@@ -707,7 +718,11 @@ __global__ void __launch_bounds__(1024) layout_cluster_kernel(LayoutArgs a, int6
         for (int n = 0; n < N; ++n) {
             const bool touched = (nm >> n) & 1u;
             const unsigned bal = __ballot_sync(kFullMask, touched);
-            if (t < t1) a.node_slot[t * N + n] = touched ? wn[warp * N + n] + __popc(bal & lt) : -1;
+            const int ns = touched ? wn[warp * N + n] + __popc(bal & lt) : -1;
+            if (t < t1) {
+                a.node_slot[t * N + n] = ns;
+                if (a.node_src && touched) a.node_src[tot[E + n] + ns] = (int)t;
+            }
         }
         __syncthreads();
     }
@@ -859,6 +874,7 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     a.node_counts = p.node_counts;
     a.node_offsets = p.node_offsets;
     a.node_slot = p.node_slot;
+    a.node_src = p.nodes ? p.node_src : nullptr;
     a.err = p.err;
     if (p.cluster && p.T <= kClusterMaxTokens)
         return p.k <= 8 ? launch_layout_cluster<8>(a, stream) : launch_layout_cluster<32>(a, stream);

@@ -58,6 +58,26 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 
 // ---- cache-hinted global access -----------------------------------------
+// Every kernel here may start before its predecessor on the stream has
+// finished (programmatic dependent launch), so whatever a predecessor wrote
+// (layout arrays, staging rows, receive rows, partial sums, scales) is read
+// only after pdl_wait(), with coherent loads issued from volatile asm so that
+// the compiler keeps them below the wait.  The non-coherent path
+// (ld.global.nc, __ldg) is not used for such data: it assumes the data stays
+// unchanged while the reading kernel is resident, and a reading kernel that
+// is already resident while its predecessor writes breaks that assumption
+// (the compiler may also hoist such a load above the wait).
+__device__ __forceinline__ int ld_dep(const int* p) {
+    int v;
+    asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_dep(const float* p) {
+    float v;
+    asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
 // Streaming loads of rows read exactly once (no L1 allocation) and
 // evict-first stores of rows written once.
 template <typename V>
@@ -65,7 +85,7 @@ __device__ __forceinline__ V ld_stream(const V* p);
 template <>
 __device__ __forceinline__ uint4 ld_stream<uint4>(const uint4* p) {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
@@ -73,7 +93,7 @@ __device__ __forceinline__ uint4 ld_stream<uint4>(const uint4* p) {
 template <>
 __device__ __forceinline__ uint2 ld_stream<uint2>(const uint2* p) {
     uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+    asm volatile("ld.global.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
                  : "=r"(v.x), "=r"(v.y)
                  : "l"(p));
     return v;
@@ -81,13 +101,13 @@ __device__ __forceinline__ uint2 ld_stream<uint2>(const uint2* p) {
 template <>
 __device__ __forceinline__ uint32_t ld_stream<uint32_t>(const uint32_t* p) {
     uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    asm volatile("ld.global.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 template <>
 __device__ __forceinline__ uint16_t ld_stream<uint16_t>(const uint16_t* p) {
     uint16_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    asm volatile("ld.global.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
     return v;
 }
 

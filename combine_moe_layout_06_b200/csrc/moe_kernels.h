@@ -29,6 +29,7 @@ struct LayoutParams {
     int* node_counts;       // [N]    (nodes)
     int* node_offsets;      // [N+1]  (nodes)
     int* node_slot;         // [T*N]  (nodes)
+    int* node_src = nullptr;  // [U]  staging row -> token (nodes, optional)
     int* err;               // [1]
     void* workspace;        // layout_workspace_bytes()
 };
@@ -46,6 +47,10 @@ struct RowMoveParams {
     const int* node_slot;     // [T*N]
     const int* node_offsets;  // [N+1]
     const int* rank_offsets;  // [R+1]
+    // [U] staging row -> token; when given, the node expansion walks staging
+    // rows (work divided by rows, whatever each node's load), else (node,
+    // token) pairs
+    const int* node_src = nullptr;
     int* err;
     CopyEngine engine;
     // The source rows (x) were complete before the layout began and the

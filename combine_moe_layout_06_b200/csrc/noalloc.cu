@@ -80,6 +80,7 @@ extern "C" moe_status_t moe_layout_noalloc(const moe_config_t* c, const int32_t*
     p.node_counts = L->node_counts;
     p.node_offsets = L->node_offsets;
     p.node_slot = L->node_slot;
+    p.node_src = L->node_src;
     p.err = L->error_word;
     p.workspace = scratch;
     return moe::launch_layout(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK

@@ -174,6 +174,21 @@ def make_random(T: int, H: int, E: int, k: int, seed: int, renorm: bool = True,
     return {"x": x_bf16_bits(x), "topk_idx": idx, "topk_w": w}
 
 
+def make_node_skewed(T: int, H: int, E: int, k: int, N: int, hot_frac: float, seed: int) -> dict:
+    """Routing with one hot node: each token, with probability hot_frac,
+    sends all k choices to the first E//N experts (which sit on node 0 under
+    a contiguous expert partition); the others route uniformly.  Node 0 then
+    stages far more rows than the rest (the load imbalance a load-aware
+    forwarder is meant to absorb)."""
+    xrng, rng = _streams(seed)
+    x = xrng.standard_normal((T, H), dtype=np.float32)
+    logits = rng.standard_normal((T, E))
+    hot = rng.random(T) < hot_frac
+    logits[np.ix_(hot, np.arange(E) < E // N)] += 50.0
+    idx, w = route(logits, k, True)
+    return {"x": x_bf16_bits(x), "topk_idx": idx, "topk_w": w}
+
+
 def random_bf16(shape, seed: int, scale: float = 1.0) -> np.ndarray:
     """N(0, scale^2) values as bf16 bit patterns (e.g. stand-in expert outputs)."""
     rng = _rng(seed)

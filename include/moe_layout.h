@@ -121,6 +121,18 @@ typedef struct moe_config {
  *                          moe_get_error() reads and clears it
  *   workspace      moe_layout_workspace_bytes() bytes, 16-byte aligned,
  *                          scratch for moe_layout only
+ *   node_src       [moe_node_staging_rows()]  token held by each staging row:
+ *                          node_src[node_offsets[n] + node_slot[t][n]] = t
+ *                          (TWO_LEVEL, optional).  When it is given,
+ *                          moe_layout writes it and the second phase of a
+ *                          two-level dispatch divides its work by staging
+ *                          rows, so a node that receives many more tokens
+ *                          than the others is spread over the whole GPU
+ *                          (the load-aware forwarding of the FUSCO article,
+ *                          section "FUSCO 的核心创新"); when it is NULL the
+ *                          second phase walks (node, token) pairs, whose
+ *                          work per node follows that node's load.  Only
+ *                          entries below node_offsets[N] are written.
  * Node arrays may be NULL when MOE_FLAG_TWO_LEVEL is not set. */
 typedef struct moe_layout {
     int32_t *expert_counts;
@@ -132,6 +144,7 @@ typedef struct moe_layout {
     int32_t *node_slot;
     int32_t *error_word;
     void *workspace;
+    int32_t *node_src;
 } moe_layout_t;
 
 /* Text of a status code (static storage, never NULL). */

@@ -77,6 +77,8 @@ def _bind(path: str):
     lib.oracle_validate_topk.restype = ctypes.c_int
     lib.oracle_layout.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p]
     lib.oracle_layout.restype = ctypes.c_int
+    lib.oracle_node_sources.argtypes = [i64, i32, p, p, p]
+    lib.oracle_node_sources.restype = None
     lib.oracle_dispatch_flat.argtypes = [i64, i32, i32, p, p, p]
     lib.oracle_dispatch_flat.restype = None
     lib.oracle_dispatch_two_level.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p]
@@ -161,7 +163,8 @@ def validate_topk(topk: np.ndarray, E: int) -> int:
 # ---------------------------------------------------------------- layout
 
 def layout(topk: np.ndarray, E: int, R: int, N: int = 1, nodes: bool = False) -> dict:
-    """Layout metadata.  ``nodes`` also computes the node staging map."""
+    """Layout metadata.  ``nodes`` also computes the node staging map and its
+    inverse ``node_src`` (staging row -> token)."""
     topk = _c(topk, np.int32)
     T, k = topk.shape
     out = {
@@ -184,6 +187,10 @@ def layout(topk: np.ndarray, E: int, R: int, N: int = 1, nodes: bool = False) ->
                                _ptr(out["rank_offsets"]), _ptr(out["slot"]), nc, no, ns)
     if st != OK:
         raise OracleError(st)
+    if nodes:
+        out["node_src"] = np.zeros(int(out["node_offsets"][N]), np.int32)
+        _load().oracle_node_sources(T, N, _ptr(out["node_offsets"]), _ptr(out["node_slot"]),
+                                    _ptr(out["node_src"]))
     return out
 
 

@@ -282,6 +282,22 @@ int oracle_layout(int64_t T, int32_t k, int32_t E, int32_t R, int32_t N,
     return ORC_OK;
 }
 
+/* Inverse of the node staging map: staging row node_offsets[n] +
+ * node_slot[t][n] holds token t, for every (t, n) with node_slot[t][n] >= 0.
+ * node_src has node_offsets[N] entries.  (FUSCO article, section "FUSCO 的
+ * 核心创新": a forwarder handles the rows staged for its node; listing them
+ * row by row lets the forwarding work be divided by rows.) */
+void oracle_node_sources(int64_t T, int32_t N, const int32_t *node_offsets,
+                         const int32_t *node_slot, int32_t *node_src)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t n = 0; n < N; ++n) {
+            int32_t ns = node_slot[t * N + n];
+            if (ns >= 0)
+                node_src[(int64_t)node_offsets[n] + ns] = (int32_t)t;
+        }
+}
+
 /* ------------------------------------------------------------------ */
 /* Dispatch                                                            */
 /* ------------------------------------------------------------------ */

@@ -21,10 +21,11 @@ def cfg_of(T, H, E, k, R, N=1, flags=0):
     return capi.config(T, H, E, k, R, N, flags)
 
 
-def gpu_layout(cfg, topk_np):
-    """Run moe_layout; returns (DeviceLayout, device topk)."""
+def gpu_layout(cfg, topk_np, node_src=True):
+    """Run moe_layout; returns (DeviceLayout, device topk).  node_src=False
+    leaves the staging-row map out (pair-walking node expansion)."""
     ensure_lib()
-    lay = buffers.DeviceLayout(cfg)
+    lay = buffers.DeviceLayout(cfg, node_src=node_src)
     topk = torch.from_numpy(np.ascontiguousarray(topk_np, np.int32)).cuda()
     capi.moe_layout(cfg, topk, lay.struct)
     return lay, topk

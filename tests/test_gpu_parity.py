@@ -63,12 +63,18 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
     eo = inputs.random_bf16_bits((T * k, H), seed=T * k + H)
     y_ref = oracle_mod.combine(eo, w, ref["slot"])
     x_dev = M.to_dev(x)
-    for flags in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK):
+    runs = [(f, True) for f in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK)]
+    runs += [(f, False) for f in (TWO, TWO | VEC, TWO | BULK)]   # pair-walking expansion
+    for flags, node_src in runs:
         cfg = M.cfg_of(T, H, E, k, R, N, flags)
-        lay, _ = M.gpu_layout(cfg, topk)
+        lay, _ = M.gpu_layout(cfg, topk, node_src=node_src)
+        want = ref if flags & TWO else {k_: v for k_, v in ref.items() if not k_.startswith("node")}
+        if not node_src:
+            want = {k_: v for k_, v in want.items() if k_ != "node_src"}
+        M.assert_layout_equal(lay.host(), want)
         recv, staging = M.gpu_dispatch(cfg, lay, x_dev, fill=0x7F81)
         assert np.array_equal(M.bits(recv), recv_ref)
-        lay2 = M.buffers.DeviceLayout(cfg)
+        lay2 = M.buffers.DeviceLayout(cfg, node_src=node_src)
         recv2 = torch.empty_like(recv)
         st2 = M.staging_buffer(cfg) if flags & TWO else None
         capi.moe_layout_dispatch(cfg, torch.from_numpy(topk).cuda(), lay2.struct, x_dev, recv2, st2)
@@ -101,6 +107,32 @@ def test_large_batch_multi_kernel_layout(oracle_mod, T):
         assert np.array_equal(M.bits(recv), oracle_mod.dispatch_flat(x, ref["slot"]))
         y = M.gpu_combine(cfg, lay, recv, w)
         assert np.array_equal(M.bits(y), oracle_mod.combine(M.bits(recv), w, ref["slot"]))
+        assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+@pytest.mark.parametrize("engine", [0, VEC, BULK])
+@pytest.mark.parametrize("hot_frac", [0.0, 0.9, 1.0])
+def test_skewed_node_loads(oracle_mod, engine, hot_frac):
+    """One hot node (up to every token on node 0, the other nodes empty):
+    the row-balanced and the pair-walking expansions both reproduce the
+    oracle's staging and receive buffers bit for bit."""
+    T, H, E, k, R, N = 5000, 264, 64, 6, 8, 4
+    d = inputs.make_node_skewed(T, H, E, k, N, hot_frac, seed=int(hot_frac * 10) + 3)
+    x, topk = d["x"], d["topk_idx"]
+    ref = oracle_mod.layout(topk, E, R, N, nodes=True)
+    staging_ref, recv_ref = oracle_mod.dispatch_two_level(x, ref, R, N)
+    if hot_frac == 1.0:
+        assert ref["node_counts"][1:].sum() == 0 and ref["node_counts"][0] == T
+    x_dev = M.to_dev(x)
+    cfg = M.cfg_of(T, H, E, k, R, N, TWO | engine)
+    for node_src in (True, False):
+        lay, _ = M.gpu_layout(cfg, topk, node_src=node_src)
+        want = ref if node_src else {k_: v for k_, v in ref.items() if k_ != "node_src"}
+        M.assert_layout_equal(lay.host(), want)
+        recv, staging = M.gpu_dispatch(cfg, lay, x_dev, fill=0x7F81)
+        U = int(ref["node_offsets"][-1])
+        assert np.array_equal(M.bits(staging)[:U], staging_ref)
+        assert np.array_equal(M.bits(recv), recv_ref)
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 

@@ -35,15 +35,18 @@ def _brute_layout(topk, E, R, N):
     node_of = rank_of // (R // N)
     node_slot = np.full((T, N), -1, np.int64)
     node_counts = np.zeros(N, np.int64)
+    node_src = []
     for n in range(N):
         toks = [t for t in range(T) if any(node_of[topk[t, j]] == n for j in range(k))]
         for i, t in enumerate(toks):
             node_slot[t, n] = i
         node_counts[n] = len(toks)
+        node_src += toks                     # staging rows of node n, in token order
     node_offsets = np.concatenate([[0], np.cumsum(node_counts)])
     return dict(slot=slot, expert_counts=counts, expert_offsets=offsets,
                 rank_offsets=rank_offsets, node_slot=node_slot,
-                node_counts=node_counts, node_offsets=node_offsets)
+                node_counts=node_counts, node_offsets=node_offsets,
+                node_src=np.array(node_src, np.int64))
 
 
 def _random_topk(rng, T, E, k):
@@ -169,5 +172,5 @@ def test_exhaustive_tiny(oracle_mod):
             topk = np.array([a, b], np.int32)
             got = oracle_mod.layout(topk, 4, 2, 2, nodes=True)
             ref = _brute_layout(topk, 4, 2, 2)
-            for key in ("slot", "expert_offsets", "rank_offsets", "node_slot"):
+            for key in ("slot", "expert_offsets", "rank_offsets", "node_slot", "node_src"):
                 assert np.array_equal(np.asarray(got[key], np.int64), ref[key])

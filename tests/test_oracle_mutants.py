@@ -63,6 +63,9 @@ MUTANTS = {
     "fp8_combine_drops_scale": (
         "float coef = w[t * k + j] * eo_scale[row];",
         "float coef = w[t * k + j];"),
+    "node_src_ignores_node_offset": (
+        "node_src[(int64_t)node_offsets[n] + ns] = (int32_t)t;",
+        "node_src[ns] = (int32_t)t;"),
     "widening_drops_low_bit": (
         "    uint32_t u = ((uint32_t)h) << 16;",
         "    uint32_t u = ((uint32_t)(h & 0xFFFEu)) << 16;"),

@@ -26,7 +26,8 @@ def _both(cfg, topk_np):
     got = buffers.DeviceLayout(cfg)
     got_struct = capi.layout_struct(got.expert_counts, got.expert_offsets, got.rank_offsets,
                                     got.slot, got.error_word, None, got.node_counts,
-                                    got.node_offsets, got.node_slot)   # no workspace at all
+                                    got.node_offsets, got.node_slot,
+                                    got.node_src)   # no workspace at all
     capi.moe_layout_noalloc(cfg, topk, got_struct)
     torch.cuda.synchronize()
     assert capi.moe_get_error(ref.struct) == capi.MOE_OK
