@@ -7,14 +7,21 @@
 // rounded to nearest even and saturated to +-448 (cvt.rn.satfinite).  The
 // receive buffer then carries H bytes plus 4 per row instead of 2H.
 //
-//  quantize_fp8_kernel: one warp per source row; the first pass finds amax,
-//    the second converts 16-byte vectors of 8 bf16 values into 8 codes and
-//    stores them to every destination row: the row itself (row-wise
-//    quantization of expert outputs) or the token's k receive rows (fp8
-//    dispatch: quantize once, write k copies).
-//  combine_fp8_kernel: the fused combine on codes, coef_j = w[t][j] *
-//    scale[slot[t][j]] and acc = fma(coef_j, decode(code), acc) for j = 0 ..
-//    k-1 from +0, one RNE bf16 store.
+//  quantize_rows16_kernel (rows of up to 8192 values, H % 16 == 0): one
+//    warp per source row, the row held in registers (lane l owns the
+//    16-value groups l, l+32, ...), amax by a warp reduction, then every
+//    group's 16 codes go out as one 16-byte store to every destination row:
+//    the row itself (row-wise quantization of expert outputs) or the
+//    token's k receive rows (fp8 dispatch: quantize once, write k copies).
+//  quantize_fp8_kernel (any H % 8 == 0): the same with two passes over the
+//    row (amax, then convert) and 8-byte code stores.
+//  combine_ring_fp8_kernel (H % 16 == 0, k <= 8) and combine_fp8_kernel
+//    (any H % 8 == 0, k <= 32): the fused combine on codes, coef_j = w[t][j]
+//    * scale[slot[t][j]] and acc = fma(coef_j, decode(code), acc) for j = 0
+//    .. k-1 from +0, one RNE bf16 store.  The ring kernel stages the rows in
+//    shared memory with cp.async, so more bytes are in flight per warp than
+//    registers would hold; the code widening (e4m3 -> f16 -> f32 conversions)
+//    then bounds it.
 #include <cuda_fp8.h>
 
 #include "moe_kernels.h"
@@ -35,7 +42,8 @@ __device__ __forceinline__ uint2 to_e4m3x8(const float (&f)[8]) {
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
-// 8 e4m3 codes -> 8 floats (exact).
+// 8 e4m3 codes -> 8 floats (exact): the hardware conversion of code pairs to
+// f16x2, then each half widened to f32.
 __device__ __forceinline__ void from_e4m3x8(uint2 c, float (&f)[8]) {
     const uint32_t w[2] = {c.x, c.y};
 #pragma unroll
@@ -70,7 +78,7 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
         if (a.slot == nullptr) {
             dst = lane == 0 ? r : -1;
         } else if (lane < a.k) {
-            const int s = __ldg(a.slot + r * a.k + lane);
+            const int s = ld_dep(a.slot + r * a.k + lane);
             if (s >= 0 && s < a.dst_rows) dst = s;
             else if (s != -1) errbits |= kErrBadLayout;
         }
@@ -93,7 +101,9 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
             const int64_t v = v0 + lane;
             const bool active = v < a.rv;
             float f[8];
-            unpack_bf16<uint4>(active ? __ldg(src + v) : make_uint4(0, 0, 0, 0), f);
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (active) raw = ld_stream(src + v);
+            unpack_bf16<uint4>(raw, f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
             const uint2 code = to_e4m3x8(f);
@@ -103,6 +113,81 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
                 m &= m - 1;
                 const int64_t d = __shfl_sync(kFullMask, dst, j);
                 if (active) a.q[d * a.rv + v] = code;
+            }
+        }
+    }
+    warp_report(a.err, errbits);
+}
+
+// Register-resident row: NG 16-value groups per lane (H <= 512 * NG).
+template <int NG>
+__global__ void __launch_bounds__(kThreads) quantize_rows16_kernel(Fp8Args a) {
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t G = a.rv / 2;  // 16-value groups per row
+    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    int errbits = 0;
+    for (int64_t r = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); r < a.rows; r += nw) {
+        int64_t dst = -1;
+        if (a.slot == nullptr) {
+            dst = lane == 0 ? r : -1;
+        } else if (lane < a.k) {
+            const int s = ld_dep(a.slot + r * a.k + lane);
+            if (s >= 0 && s < a.dst_rows) dst = s;
+            else if (s != -1) errbits |= kErrBadLayout;
+        }
+        const uint4* src = a.src + r * a.rv;
+        uint4 raw[NG][2];
+#pragma unroll
+        for (int i = 0; i < NG; ++i) {
+            const int64_t g = lane + 32 * i;
+            raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
+            if (g < G) {
+                raw[i][0] = ld_stream(src + 2 * g);
+                raw[i][1] = ld_stream(src + 2 * g + 1);
+            }
+        }
+        uint32_t amax_bits = 0;
+#pragma unroll
+        for (int i = 0; i < NG; ++i)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float f[8];
+                unpack_bf16<uint4>(raw[i][h], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax_bits = max(amax_bits, __float_as_uint(fabsf(f[e])));
+            }
+        amax_bits = __reduce_max_sync(kFullMask, amax_bits);
+        const float amax = __uint_as_float(amax_bits);
+        const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
+        const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+        uint4 code[NG];
+#pragma unroll
+        for (int i = 0; i < NG; ++i) {
+            uint2 c[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float f[8];
+                unpack_bf16<uint4>(raw[i][h], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
+                c[h] = to_e4m3x8(f);
+            }
+            code[i] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+        }
+        if (dst >= 0) a.scale[dst] = scale;
+        unsigned m = __ballot_sync(kFullMask, dst >= 0);
+        uint4* q = reinterpret_cast<uint4*>(a.q);
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            const int64_t d = __shfl_sync(kFullMask, dst, j);
+            uint4* qrow = q + d * G;
+#pragma unroll
+            for (int i = 0; i < NG; ++i) {
+                const int64_t g = lane + 32 * i;
+                if (g < G) st_stream(qrow + g, code[i]);
             }
         }
     }
@@ -148,8 +233,8 @@ __global__ void __launch_bounds__(kThreads) combine_fp8_kernel(Fp8CombArgs a) {
             s = -1;
             coef = 0.f;
             if (lane < a.k) {
-                s = __ldg(a.slot + t * a.k + lane);
-                if (s >= 0 && s < a.q_rows) coef = __ldg(a.w + t * a.k + lane) * __ldg(a.scale + s);
+                s = ld_dep(a.slot + t * a.k + lane);
+                if (s >= 0 && s < a.q_rows) coef = ld_dep(a.w + t * a.k + lane) * ld_dep(a.scale + s);
                 else {
                     if (s != -1) errbits |= kErrBadLayout;
                     s = -1;
@@ -203,6 +288,127 @@ __global__ void __launch_bounds__(kThreads) combine_fp8_kernel(Fp8CombArgs a) {
     warp_report(a.err, errbits);
 }
 
+// Shared-memory staged combine (H % 16 == 0, k <= 8): each warp keeps a
+// ring of kRing stages, a stage holding one item's (token, 512-code chunk)
+// rows -- lane l copies group l of every expert row with cp.async -- plus
+// the rows' weights and scales.  The data in flight lives in shared memory,
+// not registers, so kRing - 1 items per warp stay in flight while one is
+// summed.  Items are a contiguous token-major range per warp; rows are
+// summed in column order j = 0 .. k-1 exactly as in the register kernels.
+#ifndef MOE_FP8_RING
+#define MOE_FP8_RING 3
+#endif
+#ifndef MOE_FP8_RING_WARPS
+#define MOE_FP8_RING_WARPS 8
+#endif
+constexpr int kRing = MOE_FP8_RING;
+constexpr int kRingWarps = MOE_FP8_RING_WARPS;
+constexpr int kRingThreads = kRingWarps * 32;
+constexpr int kRingRows = 8;
+struct RingStage {
+    uint4 code[kRingRows][32];  // [row j][lane]
+    float w[kRingRows];
+    float scale[kRingRows];
+    unsigned valid;             // bit j: row j is summed
+    unsigned pad[3];
+};
+
+__global__ void __launch_bounds__(kRingThreads) combine_ring_fp8_kernel(Fp8CombArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    RingStage* ring = reinterpret_cast<RingStage*>(smem) + warp * kRing;
+    pdl_trigger();
+    pdl_wait();
+    const int64_t G = a.rv / 2;   // 16-code groups per row
+    const int64_t cpr = (G + 31) / 32;
+    const int64_t items = a.T * cpr;
+    const int64_t nw = (int64_t)gridDim.x * kRingWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kRingWarps + warp;
+    const int64_t ib = items * gw / nw, ie = items * (gw + 1) / nw;
+    const uint4* q = reinterpret_cast<const uint4*>(a.q);
+    int errbits = 0;
+
+    // issue side: lane j < k holds the expert row of (token ti, j)
+    int64_t ti = -1;
+    int s_issue = -1;
+    auto issue = [&](int64_t item, RingStage& st) {
+        const int64_t t = item / cpr;
+        const int64_t g = (item - t * cpr) * 32 + lane;
+        if (t != ti) {
+            s_issue = -1;
+            if (lane < a.k) {
+                const int s = ld_dep(a.slot + t * a.k + lane);
+                if (s >= 0 && s < a.q_rows) s_issue = s;
+                else if (s != -1) errbits |= kErrBadLayout;
+            }
+            ti = t;
+        }
+        const unsigned valid = __ballot_sync(kFullMask, s_issue >= 0);
+        if (lane == 0) st.valid = valid;
+        if (s_issue >= 0) {
+            async_copy4(&st.w[lane], a.w + t * a.k + lane);
+            async_copy4(&st.scale[lane], a.scale + s_issue);
+        }
+        unsigned m = valid;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            const int sj = __shfl_sync(kFullMask, s_issue, j);
+            if (g < G) async_copy16(&st.code[j][lane], q + (int64_t)sj * G + g);
+        }
+        async_commit();
+    };
+
+    const int64_t mine = ie - ib;
+    for (int64_t i = 0; i < kRing - 1; ++i) {
+        if (i < mine) issue(ib + i, ring[i]);
+        else async_commit();   // keep one group per stage
+    }
+    for (int64_t i = 0; i < mine; ++i) {
+        // refill the stage freed last iteration, then wait for item i
+        if (i + kRing - 1 < mine) issue(ib + i + kRing - 1, ring[(i + kRing - 1) % kRing]);
+        else async_commit();
+        async_wait<kRing - 1>();
+        __syncwarp();
+        RingStage& st = ring[i % kRing];
+        const int64_t item = ib + i;
+        const int64_t t = item / cpr;
+        const int64_t g = (item - t * cpr) * 32 + lane;
+        const unsigned valid = st.valid;
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kRingRows; ++j) {
+            if (!((valid >> j) & 1u)) continue;
+            const float coef = st.w[j] * st.scale[j];
+            const uint4 c = st.code[j][lane];
+            float f[8];
+            from_e4m3x8(make_uint2(c.x, c.y), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(coef, f[e], acc[e]);
+            from_e4m3x8(make_uint2(c.z, c.w), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[8 + e] = __fmaf_rn(coef, f[e], acc[8 + e]);
+        }
+        if (g < G) {
+            float lo[8], hi[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                lo[e] = acc[e];
+                hi[e] = acc[8 + e];
+            }
+            uint4* yrow = a.y + t * a.rv;
+            st_stream(yrow + 2 * g, pack_bf16<uint4>(lo));
+            st_stream(yrow + 2 * g + 1, pack_bf16<uint4>(hi));
+        }
+        // every lane has read this stage before it is refilled
+        __syncwarp();
+    }
+    async_wait<0>();
+    warp_report(a.err, errbits);
+}
+
 }  // namespace
 
 bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
@@ -214,6 +420,15 @@ bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
         if (reinterpret_cast<uintptr_t>(p) % 8) return false;
     return true;
 }
+
+namespace {
+template <int NG>
+cudaError_t launch_rows16(const Fp8Args& a, cudaStream_t stream) {
+    constexpr auto kern = quantize_rows16_kernel<NG>;
+    const int grid = persistent_grid<kern>(a.rows, kThreads);
+    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+}  // namespace
 
 cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
                                 int64_t dst_rows, void* q, float* scale, int* err,
@@ -229,6 +444,12 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, c
     a.rv = hidden / 8;
     a.dst_rows = dst_rows;
     a.err = err;
+    // register-resident rows when the row splits into 16-value groups, at
+    // most 8 per lane, and the codes take 16-byte stores
+    const bool wide = hidden % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 16 == 0;
+    if (wide && hidden <= 512 * 2) return launch_rows16<2>(a, stream);
+    if (wide && hidden <= 512 * 4) return launch_rows16<4>(a, stream);
+    if (wide && hidden <= 512 * 8) return launch_rows16<8>(a, stream);
     constexpr auto kern = quantize_fp8_kernel;
     const int grid = persistent_grid<kern>(rows, kThreads);
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
@@ -248,6 +469,16 @@ cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const floa
     a.rv = (int64_t)(p.row_bytes / 16);
     a.q_rows = p.T * p.k;
     a.err = p.err;
+    const bool wide = (p.row_bytes / 2) % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 16 == 0;
+    if (wide && p.k <= kRingRows) {
+        constexpr auto kr = combine_ring_fp8_kernel;
+        const size_t smem = sizeof(RingStage) * kRing * kRingWarps;
+        cudaError_t e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const int64_t cprr = (a.rv / 2 + 31) / 32;
+        const int gridr = persistent_grid<kr>(a.T * cprr, kRingThreads, smem);
+        return launch_pdl(kr, dim3(gridr), dim3(kRingThreads), smem, stream, a);
+    }
     constexpr auto kern = combine_fp8_kernel<2>;
     const int64_t cpr = (a.rv + 63) / 64;
     const int grid = persistent_grid<kern>(a.T * cpr, kThreads);

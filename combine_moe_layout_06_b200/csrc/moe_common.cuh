@@ -279,6 +279,25 @@ __device__ __forceinline__ void bulk_wait_read() {
 // Wait until all of this thread's bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// ---- per-thread async copies (cp.async, global -> shared) -----------------
+// Each thread tracks its own copies in commit groups; a copy's bytes may be
+// read by the copying thread after cp.async.wait_group, by other threads of
+// the warp after that and a __syncwarp().
+__device__ __forceinline__ void async_copy16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void async_copy4(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+                 : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---- launching ------------------------------------------------------------
 // Launch with programmatic stream serialization allowed, so the kernel may
 // start while its predecessor drains; each kernel calls pdl_wait() before

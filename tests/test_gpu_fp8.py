@@ -20,6 +20,9 @@ CASES = [
     (257, 72, 64, 8, 4),
     (300, 16, 32, 16, 8),      # k > 8, rows shorter than a warp's vectors
     (1000, 2048, 60, 4, 7),
+    (64, 3088, 32, 6, 4),      # 193 16-value groups: a ragged last group per row
+    (40, 4096, 16, 4, 2),      # 8 groups per lane, the most held in registers
+    (24, 8208, 16, 4, 2),      # beyond the register-resident kernels
 ]
 
 
