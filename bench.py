@@ -563,6 +563,30 @@ def main():
         barrier()
         return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
+    # One step at a time after writing a scratch buffer of twice the L2
+    # outside the timed region (the cold variant of the back-to-back
+    # measurement); per-step times, median and mean.
+    scratch = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4,
+                          dtype=torch.float32, device=dev)
+
+    def flushed_steps(K):
+        single = graphs["step"][1]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            scratch.fill_(1.0)
+            e0.record()
+            single.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+        return {"median_ms": round(max_over_ranks(statistics.median(ts), world, dev), 5),
+                "mean_ms": round(max_over_ranks(statistics.fmean(ts), world, dev), 5),
+                "steps": K, "flush_bytes": scratch.numel() * 4}
+
     K = args.steps
     with ClockSampler(local) as clocks:
         total_ms = timed("step", K)
@@ -572,6 +596,7 @@ def main():
         agrs_ms = timed("agrs", K) if with_agrs else None
         fp8_ms = timed("fp8", K) if with_fp8 else None
         fp8_ld = timed("fp8_LD", K) / K if with_fp8 else None
+        flushed = flushed_steps(K)
     ms_per_step = total_ms / K
     t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
     for b in sets:
@@ -699,6 +724,8 @@ def main():
             "peak_gbs": peak, "peak_source": peak_src,
             "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
             "tokens_per_s": round(wl.T * world * K / (total_ms * 1e-3), 1),
+            "tokens_per_s_dispatch_combine": round(wl.T * world / ((t_dispatch + t_combine) * 1e-3), 1),
+            "flushed_step": flushed,
             "dispatch_combine_only_gbs": round(step_bytes / ((t_dispatch + t_combine) * 1e-3) / 1e9, 2),
             "kernels_ms": {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
                            "combine": round(t_combine, 5)},
