@@ -79,6 +79,8 @@ def _bind(path: str):
     lib.oracle_layout.restype = ctypes.c_int
     lib.oracle_node_sources.argtypes = [i64, i32, p, p, p]
     lib.oracle_node_sources.restype = None
+    lib.oracle_ep_layout.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p]
+    lib.oracle_ep_layout.restype = ctypes.c_int
     lib.oracle_dispatch_flat.argtypes = [i64, i32, i32, p, p, p]
     lib.oracle_dispatch_flat.restype = None
     lib.oracle_dispatch_two_level.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p]
@@ -191,6 +193,29 @@ def layout(topk: np.ndarray, E: int, R: int, N: int = 1, nodes: bool = False) ->
         out["node_src"] = np.zeros(int(out["node_offsets"][N]), np.int32)
         _load().oracle_node_sources(T, N, _ptr(out["node_offsets"]), _ptr(out["node_slot"]),
                                     _ptr(out["node_src"]))
+    return out
+
+
+def ep_layout(topk: np.ndarray, E: int, R: int, shard_begin) -> dict:
+    """Layout with the tokens sharded over source ranks (shard g = tokens
+    [shard_begin[g], shard_begin[g+1])): per-source counts [G, E], expert and
+    rank offsets, and slot [T, k] as rows of the concatenated receive
+    buffers."""
+    topk = _c(topk, np.int32)
+    T, k = topk.shape
+    sb = _c(shard_begin, np.int64)
+    G = sb.size - 1
+    out = {
+        "counts": np.zeros((G, E), np.int32),
+        "expert_offsets": np.zeros(E + 1, np.int32),
+        "rank_offsets": np.zeros(R + 1, np.int32),
+        "slot": np.zeros((T, k), np.int32),
+    }
+    st = _load().oracle_ep_layout(T, k, E, R, G, _ptr(sb), _ptr(topk), _ptr(out["counts"]),
+                                  _ptr(out["expert_offsets"]), _ptr(out["rank_offsets"]),
+                                  _ptr(out["slot"]))
+    if st != OK:
+        raise OracleError(st)
     return out
 
 

@@ -282,6 +282,88 @@ int oracle_layout(int64_t T, int32_t k, int32_t E, int32_t R, int32_t N,
     return ORC_OK;
 }
 
+/* Layout with the source tokens sharded over G ranks (expert parallelism
+ * over real GPUs; "[None][feat] support non-divisible EP in MoE alltoall and
+ * slurm benchmark", TensorRT-LLM PR #13888, the NVLinkOneSided one-sided
+ * dispatch of the commit adding the divisible fast path, and the FUSCO
+ * article, section "FUSCO 的核心创新", rows written straight to their final
+ * position).  Source rank g holds tokens [shard_begin[g], shard_begin[g+1]).
+ * The pages give no receive order across sources; the reading taken is
+ * expert-major, then source rank, then the source's token order, each
+ * receiving rank's rows contiguous.  Steps, as a sharded system takes them:
+ *  1. every source counts its own routes per expert: counts[g][e];
+ *  2. the counts are exchanged, so every rank sees counts[*][e];
+ *  3. expert totals, their exclusive prefix (expert_offsets) and the rank
+ *     offsets of the ceil/floor partition;
+ *  4. the first row of source g inside expert e: expert_offsets[e] plus the
+ *     counts of the sources before g;
+ *  5. each source walks its tokens in order with one cursor per expert.
+ * slot[t][j] is the row in the concatenation of all ranks' receive buffers
+ * (rank r holds rows [rank_offsets[r], rank_offsets[r+1])). */
+int oracle_ep_layout(int64_t T, int32_t k, int32_t E, int32_t R, int32_t G,
+                     const int64_t *shard_begin, const int32_t *topk,
+                     int32_t *counts, int32_t *expert_offsets,
+                     int32_t *rank_offsets, int32_t *slot)
+{
+    int st = oracle_validate_config(T, 1, E, k, R, 1);
+    if (st != ORC_OK)
+        return st;
+    st = oracle_validate_topk(T, k, E, topk);
+    if (st != ORC_OK)
+        return st;
+    if (G < 1 || shard_begin[0] != 0 || shard_begin[G] != T)
+        return ORC_INVALID_ARG;
+    for (int32_t g = 0; g < G; ++g)
+        if (shard_begin[g + 1] < shard_begin[g])
+            return ORC_INVALID_ARG;
+
+    /* 1. per-source histograms */
+    for (int64_t i = 0; i < (int64_t)G * E; ++i)
+        counts[i] = 0;
+    for (int32_t g = 0; g < G; ++g)
+        for (int64_t t = shard_begin[g]; t < shard_begin[g + 1]; ++t)
+            for (int32_t j = 0; j < k; ++j)
+                counts[(int64_t)g * E + topk[t * k + j]] += 1;
+
+    /* 2-3. totals over sources, expert offsets, rank offsets */
+    int64_t run = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        expert_offsets[e] = (int32_t)run;
+        for (int32_t g = 0; g < G; ++g)
+            run += counts[(int64_t)g * E + e];
+    }
+    expert_offsets[E] = (int32_t)run;
+    int32_t *first = (int32_t *)malloc(sizeof(int32_t) * (size_t)(R + 1));
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (first == NULL || cursor == NULL) {
+        free(first);
+        free(cursor);
+        return ORC_INVALID_ARG;
+    }
+    oracle_partition(E, R, first);
+    for (int32_t r = 0; r <= R; ++r)
+        rank_offsets[r] = expert_offsets[first[r]];
+
+    /* 4-5. each source's first row per expert, then its tokens in order */
+    for (int32_t g = 0; g < G; ++g) {
+        for (int32_t e = 0; e < E; ++e) {
+            int64_t before = 0;
+            for (int32_t h = 0; h < g; ++h)
+                before += counts[(int64_t)h * E + e];
+            cursor[e] = (int32_t)(expert_offsets[e] + before);
+        }
+        for (int64_t t = shard_begin[g]; t < shard_begin[g + 1]; ++t)
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t e = topk[t * k + j];
+                slot[t * k + j] = cursor[e];
+                cursor[e] += 1;
+            }
+    }
+    free(first);
+    free(cursor);
+    return ORC_OK;
+}
+
 /* Inverse of the node staging map: staging row node_offsets[n] +
  * node_slot[t][n] holds token t, for every (t, n) with node_slot[t][n] >= 0.
  * node_src has node_offsets[N] entries.  (FUSCO article, section "FUSCO 的

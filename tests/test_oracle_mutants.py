@@ -66,6 +66,12 @@ MUTANTS = {
     "node_src_ignores_node_offset": (
         "node_src[(int64_t)node_offsets[n] + ns] = (int32_t)t;",
         "node_src[ns] = (int32_t)t;"),
+    "ep_counts_later_sources": (
+        "for (int32_t h = 0; h < g; ++h)",
+        "for (int32_t h = g + 1; h < G; ++h)"),
+    "ep_cursor_ignores_source_offset": (
+        "cursor[e] = (int32_t)(expert_offsets[e] + before);",
+        "cursor[e] = (int32_t)(expert_offsets[e]);"),
     "widening_drops_low_bit": (
         "    uint32_t u = ((uint32_t)h) << 16;",
         "    uint32_t u = ((uint32_t)(h & 0xFFFEu)) << 16;"),
@@ -88,7 +94,8 @@ def test_pins_catch_mutant(name, tmp_path):
            os.path.join(ROOT, "tests", "test_oracle_partition.py"),
            os.path.join(ROOT, "tests", "test_oracle_layout.py"),
            os.path.join(ROOT, "tests", "test_oracle_dispatch_combine.py"),
-           os.path.join(ROOT, "tests", "test_oracle_fp8.py")]
+           os.path.join(ROOT, "tests", "test_oracle_fp8.py"),
+           os.path.join(ROOT, "tests", "test_oracle_ep.py")]
     res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode == 1, (
         f"mutant {name} passed every pin:\n{res.stdout[-2000:]}\n{res.stderr[-2000:]}")
