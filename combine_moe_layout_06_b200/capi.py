@@ -43,13 +43,14 @@ STATUS_NAMES = {
     MOE_ERR_BAD_LAYOUT: "BAD_LAYOUT",
 }
 
-# Every entry point the header declares, in declaration order.
+# Every entry point the header declares.
 ENTRY_POINTS = (
     "moe_status_string", "moe_check_config", "moe_expert_partition",
     "moe_layout_workspace_bytes", "moe_node_staging_rows", "moe_layout", "moe_dispatch",
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
     "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
     "moe_combine_reducescatter", "moe_quantize_rows_fp8", "moe_dispatch_fp8", "moe_combine_fp8",
+    "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -66,6 +67,10 @@ class MoeLayout(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "expert_counts", "expert_offsets", "rank_offsets", "slot", "node_counts",
         "node_offsets", "node_slot", "error_word", "workspace", "node_src")]
+
+
+class MoeEpLayout(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in ("expert_offsets", "rank_offsets", "slot")]
 
 
 class MoeError(RuntimeError):
@@ -109,6 +114,11 @@ def lib() -> ctypes.CDLL:
     L.moe_quantize_rows_fp8.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P]
     L.moe_dispatch_fp8.argtypes = [C, LP, P, P, P, P]
     L.moe_combine_fp8.argtypes = [C, LP, P, P, P, P, P]
+    EP = ctypes.POINTER(MoeEpLayout)
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    L.moe_ep_layout.argtypes = [C, ctypes.c_int32, ctypes.c_int32, P, P, LP, EP, P]
+    L.moe_ep_dispatch.argtypes = [C, LP, EP, P, PP, ctypes.c_int64, P]
+    L.moe_ep_combine.argtypes = [C, LP, EP, PP, ctypes.c_int64, P, P, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -224,6 +234,37 @@ def moe_layout_noalloc(cfg: MoeConfig, topk_idx, layout: MoeLayout, stream=None)
     layout.workspace (for callers that cannot allocate device memory)."""
     _check(lib().moe_layout_noalloc(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(layout),
                                     _stream(stream)), "moe_layout_noalloc")
+
+
+def ep_layout_struct(expert_offsets, rank_offsets, slot) -> MoeEpLayout:
+    return MoeEpLayout(_ptr(expert_offsets), _ptr(rank_offsets), _ptr(slot))
+
+
+def _ptr_array(bufs):
+    """Host array of device pointers (tensors or integers)."""
+    return (ctypes.c_void_p * len(bufs))(*[_ptr(b) for b in bufs])
+
+
+def moe_ep_layout(cfg: MoeConfig, source_rank: int, num_sources: int, topk_idx, counts_all,
+                  local: MoeLayout, ep: MoeEpLayout, stream=None) -> None:
+    _check(lib().moe_ep_layout(ctypes.byref(cfg), source_rank, num_sources, _ptr(topk_idx),
+                               _ptr(counts_all), ctypes.byref(local), ctypes.byref(ep),
+                               _stream(stream)), "moe_ep_layout")
+
+
+def moe_ep_dispatch(cfg: MoeConfig, local: MoeLayout, ep: MoeEpLayout, x, recv_bufs,
+                    capacity_rows: int, stream=None) -> None:
+    arr = _ptr_array(recv_bufs)
+    _check(lib().moe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(local), ctypes.byref(ep), _ptr(x),
+                                 arr, capacity_rows, _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_combine(cfg: MoeConfig, local: MoeLayout, ep: MoeEpLayout, expert_out_bufs,
+                   capacity_rows: int, topk_weights, y, stream=None) -> None:
+    arr = _ptr_array(expert_out_bufs)
+    _check(lib().moe_ep_combine(ctypes.byref(cfg), ctypes.byref(local), ctypes.byref(ep), arr,
+                                capacity_rows, _ptr(topk_weights), _ptr(y), _stream(stream)),
+           "moe_ep_combine")
 
 
 def moe_dispatch_allgather(cfg: MoeConfig, layout: MoeLayout, x, gathered, recv,

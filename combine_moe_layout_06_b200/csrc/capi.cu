@@ -320,6 +320,84 @@ moe_status_t moe_combine_reducescatter(const moe_config_t* c, const moe_layout_t
     return cuda_status(e);
 }
 
+namespace {
+
+moe_status_t check_ep(const moe_config_t* c, const moe_layout_t* L, const moe_ep_layout_t* ep) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (two_level(c) || c->num_ranks > moe::kMaxEpRanks) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (ep == nullptr || ep->expert_offsets == nullptr || ep->rank_offsets == nullptr ||
+        (c->num_tokens > 0 && ep->slot == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+moe_status_t moe_ep_layout(const moe_config_t* c, int32_t g, int32_t G, const int32_t* topk_idx,
+                           const int32_t* counts_all, const moe_layout_t* L,
+                           const moe_ep_layout_t* ep, void* stream) {
+    const moe_status_t st = check_ep(c, L, ep);
+    if (st != MOE_OK) return st;
+    if (G < 1 || g < 0 || g >= G || counts_all == nullptr || (c->num_tokens > 0 && topk_idx == nullptr))
+        return MOE_ERR_INVALID_ARG;
+    moe::EpParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.E = c->num_experts;
+    p.R = c->num_ranks;
+    p.G = G;
+    p.g = g;
+    p.topk = topk_idx;
+    p.counts_all = counts_all;
+    p.local_expert_offsets = L->expert_offsets;
+    p.local_slot = L->slot;
+    p.expert_offsets = ep->expert_offsets;
+    p.rank_offsets = ep->rank_offsets;
+    p.slot = ep->slot;
+    p.err = L->error_word;
+    return cuda_status(moe::launch_ep_layout(p, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_dispatch(const moe_config_t* c, const moe_layout_t* L, const moe_ep_layout_t* ep,
+                             const void* x, void* const* recv_bufs, int64_t capacity_rows,
+                             void* stream) {
+    const moe_status_t st = check_ep(c, L, ep);
+    if (st != MOE_OK || c->num_tokens == 0) return st;
+    if (x == nullptr || recv_bufs == nullptr || capacity_rows < 0) return MOE_ERR_INVALID_ARG;
+    for (int32_t r = 0; r < c->num_ranks; ++r)
+        if (recv_bufs[r] == nullptr) return MOE_ERR_INVALID_ARG;
+    moe::RowMoveParams p = move_params(c, L);
+    p.N = c->num_ranks;  // one lane per rank
+    p.slot = ep->slot;
+    p.rank_offsets = ep->rank_offsets;
+    return cuda_status(moe::launch_ep_dispatch(p, x, recv_bufs, capacity_rows,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_combine(const moe_config_t* c, const moe_layout_t* L, const moe_ep_layout_t* ep,
+                            const void* const* eo_bufs, int64_t capacity_rows,
+                            const float* topk_weights, void* y, void* stream) {
+    const moe_status_t st = check_ep(c, L, ep);
+    if (st != MOE_OK || c->num_tokens == 0) return st;
+    if (eo_bufs == nullptr || topk_weights == nullptr || y == nullptr || capacity_rows < 0)
+        return MOE_ERR_INVALID_ARG;
+    for (int32_t r = 0; r < c->num_ranks; ++r)
+        if (eo_bufs[r] == nullptr) return MOE_ERR_INVALID_ARG;
+    moe::CombineParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.row_bytes = (size_t)c->hidden * 2;
+    p.slot = ep->slot;
+    p.w = topk_weights;
+    p.err = L->error_word;
+    p.engine = engine_of(c->flags);
+    return cuda_status(moe::launch_ep_combine(p, c->num_ranks, ep->rank_offsets, eo_bufs,
+                                              capacity_rows, y, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_quantize_rows_fp8(const void* src, int64_t rows, int32_t hidden, void* q,
                                    float* scale, void* stream) {
     if (rows < 0 || hidden < 1) return MOE_ERR_INVALID_ARG;

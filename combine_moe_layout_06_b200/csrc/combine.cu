@@ -43,31 +43,67 @@ struct CombArgs {
     int64_t T;
     int k;
     int64_t rv;        // vectors per row
+    int64_t row_bytes;
     int64_t eo_rows;
     int* err;
+    // expert parallelism over sharded sources: the expert rows live in the
+    // buffers of ep_ranks ranks, rank r holding rows [rank_offsets[r],
+    // rank_offsets[r+1]) of the concatenation, at most ep_capacity each
+    const void* ep_bufs[kMaxEpRanks];
+    const int* rank_offsets;
+    int ep_ranks;
+    int64_t ep_capacity;
+};
+
+// Lane r < ep_ranks: rank r's rows [lo, hi) and its buffer (EP only).
+struct EpLane {
+    int lo, hi;
+    unsigned long long buf;
 };
 
 // Lane j < k: expert row and gate weight of (t, j); row -1 when invalid.
-__device__ __forceinline__ void load_route(const CombArgs& a, int64_t t, int lane, int& s, float& w,
-                                           int& bad) {
+// EP: also the address of the row, in the buffer of the rank holding it.
+template <bool EP>
+__device__ __forceinline__ void load_route(const CombArgs& a, int64_t t, int lane, const EpLane& el,
+                                           int& s, float& w, unsigned long long& rowp, int& bad) {
     s = -1;
     w = 0.f;
     if (lane < a.k) {
         s = a.slot ? ld_dep(a.slot + t * a.k + lane) : (int)(t * a.k + lane);
         w = ld_dep(a.w + t * a.k + lane);
     }
-    const bool ok = s >= 0 && s < a.eo_rows;
-    bad |= (!ok && s != -1) ? kErrBadLayout : 0;
-    s = ok ? s : -1;
+    if constexpr (EP) {
+        int r = 0;
+        for (int q = 1; q < a.ep_ranks; ++q) r += s >= __shfl_sync(kFullMask, el.lo, q) ? 1 : 0;
+        const int lo = __shfl_sync(kFullMask, el.lo, r);
+        const int hi = __shfl_sync(kFullMask, el.hi, r);
+        const unsigned long long buf = __shfl_sync(kFullMask, el.buf, r);
+        const int64_t local = (int64_t)s - lo;
+        const bool ok = s >= 0 && s < hi && local < a.ep_capacity && buf != 0ull;
+        bad |= (!ok && s != -1) ? kErrBadLayout : 0;
+        s = ok ? s : -1;
+        rowp = ok ? buf + (unsigned long long)local * (unsigned long long)a.row_bytes : 0ull;
+    } else {
+        const bool ok = s >= 0 && s < a.eo_rows;
+        bad |= (!ok && s != -1) ? kErrBadLayout : 0;
+        s = ok ? s : -1;
+        rowp = 0ull;
+    }
 }
 
-template <typename V, int VPL, int KB>
+template <typename V, int VPL, int KB, bool EP = false>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     constexpr int EPV = VecInfo<V>::kElems;
     constexpr int CHUNK = 32 * VPL;
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
+    EpLane el = {0, 0, 0ull};
+    if (EP && lane < a.ep_ranks) {
+        el.lo = ld_dep(a.rank_offsets + lane);
+        el.hi = ld_dep(a.rank_offsets + lane + 1);
+        el.buf = reinterpret_cast<unsigned long long>(a.ep_bufs[lane]);
+    }
     const int64_t cpr = (a.rv + CHUNK - 1) / CHUNK;
     const int64_t items = a.T * cpr;
     const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
@@ -81,10 +117,11 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
         int64_t c = ib - t * cpr;
         int s, s_next = -1;
         float wl, w_next = 0.f;
-        load_route(a, t, lane, s, wl, errbits);
+        unsigned long long rp, rp_next = 0ull;
+        load_route<EP>(a, t, lane, el, s, wl, rp, errbits);
         for (int64_t item = ib; item < ie; ++item) {
             const bool last_chunk = c + 1 == cpr;
-            if (last_chunk && item + 1 < ie) load_route(a, t + 1, lane, s_next, w_next, errbits);
+            if (last_chunk && item + 1 < ie) load_route<EP>(a, t + 1, lane, el, s_next, w_next, rp_next, errbits);
             const int64_t base = c * CHUNK;
             float acc[VPL][EPV];
 #pragma unroll
@@ -101,8 +138,10 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
                     const int sj = __shfl_sync(kFullMask, s, j & 31);
                     wq[q] = __shfl_sync(kFullMask, wl, j & 31);
                     ok[q] = j < a.k && sj >= 0;
+                    const unsigned long long rj = EP ? __shfl_sync(kFullMask, rp, j & 31) : 0ull;
                     if (ok[q]) {
-                        const V* row = eo + (int64_t)sj * a.rv + base;
+                        const V* row = EP ? reinterpret_cast<const V*>(rj) + base
+                                          : eo + (int64_t)sj * a.rv + base;
 #pragma unroll
                         for (int i = 0; i < VPL; ++i)
                             if (base + i * 32 + lane < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
@@ -129,6 +168,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
             if (last_chunk) {
                 s = s_next;
                 wl = w_next;
+                rp = rp_next;
                 ++t;
                 c = 0;
             } else {
@@ -139,18 +179,33 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     warp_report(a.err, errbits);
 }
 
-template <typename V, int VPL, int KB>
+template <typename V, int VPL, int KB, bool EP>
 cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
-    constexpr auto kern = combine_kernel<V, VPL, KB>;
+    constexpr auto kern = combine_kernel<V, VPL, KB, EP>;
     const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
     const int grid = persistent_grid<kern>(a.T * cpr, kThreads);
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
 }
 
-template <typename V, int VPL>
+template <typename V, int VPL, bool EP = false>
 cudaError_t launch_combine_k(CombArgs a, cudaStream_t stream) {
-    if (a.k <= 4) return launch_combine_v<V, VPL, 4>(a, stream);
-    return launch_combine_v<V, VPL, (MOE_COMBINE_KB > 4 ? MOE_COMBINE_KB : 4)>(a, stream);
+    if (a.k <= 4) return launch_combine_v<V, VPL, 4, EP>(a, stream);
+    return launch_combine_v<V, VPL, (MOE_COMBINE_KB > 4 ? MOE_COMBINE_KB : 4), EP>(a, stream);
+}
+
+CombArgs comb_args(const CombineParams& p, const void* expert_out, void* y) {
+    CombArgs a = {};
+    a.eo = expert_out;
+    a.w = p.w;
+    a.slot = p.slot;
+    a.y = y;
+    a.T = p.T;
+    a.k = p.k;
+    a.row_bytes = (int64_t)p.row_bytes;
+    a.eo_rows = p.T * p.k;
+    a.err = p.err;
+    a.rv = 0;
+    return a;
 }
 
 // ---- reduce-scatter formulation (comparison path) -------------------------
@@ -215,7 +270,8 @@ __global__ void __launch_bounds__(kThreads) rank_partial_kernel(RankArgs ra) {
         const int lo = ld_dep(ra.rank_offsets + r), hi = ld_dep(ra.rank_offsets + r + 1);
         int s = -1;
         float wl = 0.f;
-        load_route(a, t, lane, s, wl, errbits);
+        unsigned long long unused;
+        load_route<false>(a, t, lane, EpLane{0, 0, 0ull}, s, wl, unused, errbits);
         float acc[EPV];
 #pragma unroll
         for (int e = 0; e < EPV; ++e) acc[e] = 0.f;
@@ -273,15 +329,7 @@ cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void*
     // register engine unless the bulk engine is asked for
     if (p.engine == CopyEngine::kBulk && bulk_eligible(p.row_bytes, {expert_out, y}))
         return launch_combine_bulk(p, expert_out, y, stream);
-    CombArgs a;
-    a.eo = expert_out;
-    a.w = p.w;
-    a.slot = p.slot;
-    a.y = y;
-    a.T = p.T;
-    a.k = p.k;
-    a.eo_rows = p.T * p.k;
-    a.err = p.err;
+    CombArgs a = comb_args(p, expert_out, y);
     switch (vec_bytes(p.row_bytes, expert_out, y)) {
         case 16:
             a.rv = (int64_t)(p.row_bytes / 16);
@@ -295,18 +343,29 @@ cudaError_t launch_combine(const CombineParams& p, const void* expert_out, void*
     }
 }
 
-static CombArgs comb_args(const CombineParams& p, const void* expert_out, void* y) {
-    CombArgs a;
-    a.eo = expert_out;
-    a.w = p.w;
-    a.slot = p.slot;
-    a.y = y;
-    a.T = p.T;
-    a.k = p.k;
-    a.eo_rows = p.T * p.k;
-    a.err = p.err;
-    a.rv = 0;
-    return a;
+cudaError_t launch_ep_combine(const CombineParams& p, int R, const int* rank_offsets,
+                              const void* const* bufs, int64_t capacity_rows, void* y,
+                              cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    CombArgs a = comb_args(p, nullptr, y);
+    a.rank_offsets = rank_offsets;
+    a.ep_ranks = R;
+    a.ep_capacity = capacity_rows;
+    uintptr_t bits = (uintptr_t)p.row_bytes | reinterpret_cast<uintptr_t>(y);
+    for (int r = 0; r < R; ++r) {
+        a.ep_bufs[r] = bufs[r];
+        bits |= reinterpret_cast<uintptr_t>(bufs[r]);
+    }
+    if (bits % 16 == 0) {
+        a.rv = (int64_t)(p.row_bytes / 16);
+        return launch_combine_k<uint4, MOE_COMBINE_VPL, true>(a, stream);
+    }
+    if (bits % 4 == 0) {
+        a.rv = (int64_t)(p.row_bytes / 4);
+        return launch_combine_k<uint32_t, 4, true>(a, stream);
+    }
+    a.rv = (int64_t)(p.row_bytes / 2);
+    return launch_combine_k<uint16_t, 4, true>(a, stream);
 }
 
 cudaError_t launch_combine_rank_partials(const CombineParams& p, int R, const int* rank_offsets,

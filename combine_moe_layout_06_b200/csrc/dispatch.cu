@@ -40,7 +40,10 @@ namespace {
 constexpr int kWarpsPerCta = 8;
 constexpr int kThreads = kWarpsPerCta * 32;
 
-enum FanMode { kFlat = 0, kNodePack = 1, kNodeExpand = 2, kAllGather = 3, kRankSelect = 4, kNodeRows = 5 };
+enum FanMode {
+    kFlat = 0, kNodePack = 1, kNodeExpand = 2, kAllGather = 3, kRankSelect = 4, kNodeRows = 5,
+    kEpFlat = 6
+};
 
 struct FanArgs {
     const void* src;
@@ -50,8 +53,11 @@ struct FanArgs {
     const int* node_offsets;
     const int* rank_offsets;
     const int* node_src;  // [U] staging row -> token (kNodeRows)
+    void* ep_bufs[kMaxEpRanks];  // receive buffer of each rank (kEpFlat)
+    int64_t ep_capacity;         // rows per receive buffer (kEpFlat)
     int64_t T;
     int k, N, ranks_per_node;
+    int64_t row_bytes;
     int64_t rv;        // vectors per row
     int64_t src_rows;  // rows in src (bounds check)
     int64_t dst_rows;  // rows in dst (bounds check)
@@ -73,15 +79,29 @@ struct RowPlan {
     int bad;
 };
 
-// Per-lane node table of the node-rows mode, loaded once per warp: lane
-// n < N holds node n's first staging row and its receive-row range.
+// Per-lane table, loaded once per warp.  Node-rows mode: lane n < N holds
+// node n's first staging row and its receive-row range [lo, hi).  EP mode:
+// lane r < N holds rank r's rows [lo, hi) of the concatenated receive
+// buffers and the base of its buffer.
 struct NodeTable {
     int first;
     int lo, hi;
+    unsigned long long buf;
 };
+
+__device__ __forceinline__ NodeTable load_ep_table(const FanArgs& a, int lane) {
+    NodeTable nt = {INT_MAX, 0, 0, 0ull};
+    if (lane < a.N) {
+        nt.lo = ld_dep(a.rank_offsets + lane);
+        nt.hi = ld_dep(a.rank_offsets + lane + 1);
+        nt.buf = reinterpret_cast<unsigned long long>(a.ep_bufs[lane]);
+    }
+    return nt;
+}
 
 __device__ __forceinline__ NodeTable load_node_table(const FanArgs& a, int lane) {
     NodeTable nt;
+    nt.buf = 0ull;
     const bool on = lane < a.N;
     nt.first = on ? ld_dep(a.node_offsets + lane) : INT_MAX;
     nt.lo = on ? ld_dep(a.rank_offsets + lane * a.ranks_per_node) : 0;
@@ -128,6 +148,19 @@ __device__ __forceinline__ RowPlan plan_row(const FanArgs& a, int64_t row, int l
         const int s = lane < a.k ? ld_dep(a.slot + t * a.k + lane) : -1;
         p.src = row;
         p.dst = (s >= lo && s < hi && s < a.dst_rows) ? s : -1;
+    } else if (MODE == kEpFlat) {
+        // the rank whose rows [lo, hi) hold slot s, and the row in its buffer
+        const int s = lane < a.k ? ld_dep(a.slot + row * a.k + lane) : -1;
+        int r = 0;
+        for (int q = 1; q < a.N; ++q) r += s >= __shfl_sync(kFullMask, nt.lo, q) ? 1 : 0;
+        const int lo = __shfl_sync(kFullMask, nt.lo, r);
+        const int hi = __shfl_sync(kFullMask, nt.hi, r);
+        const unsigned long long buf = __shfl_sync(kFullMask, nt.buf, r);
+        const int64_t local = (int64_t)s - lo;
+        const bool ok = s >= 0 && s < hi && local >= 0 && local < a.ep_capacity && buf != 0ull;
+        p.src = row;
+        p.dst = ok ? (int64_t)(buf + (unsigned long long)local * (unsigned long long)a.row_bytes) : -1;
+        p.bad = (s != -1 && !ok) ? kErrBadLayout : 0;
     } else if (MODE == kNodeRows) {
         // staging row `row` holds token node_src[row] for node n
         const int n = node_of_row(nt, row);
@@ -166,7 +199,8 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
     const int lane = threadIdx.x & 31;
     int errbits = 0;
     int64_t rows = (MODE == kNodeExpand || MODE == kRankSelect) ? a.T * a.N : a.T;
-    NodeTable nt = {INT_MAX, 0, 0};
+    NodeTable nt = {INT_MAX, 0, 0, 0ull};
+    if (MODE == kEpFlat) nt = load_ep_table(a, lane);
     if (MODE == kNodeRows) {
         // the staging rows the layout filled: node_offsets[N], read here
         nt = load_node_table(a, lane);
@@ -200,7 +234,7 @@ __global__ void __launch_bounds__(kThreads) fanout_kernel(FanArgs a) {
                     const int j = __ffs(m) - 1;
                     m &= m - 1;
                     const int64_t d = __shfl_sync(kFullMask, cur.dst, j);
-                    V* drow = dbase + d * a.rv;
+                    V* drow = MODE == kEpFlat ? reinterpret_cast<V*>(d) + base : dbase + d * a.rv;
 #pragma unroll
                     for (int i = 0; i < VPL; ++i)
                         if (base + i * 32 + lane < a.rv) st_stream(drow + i * 32 + lane, v[i]);
@@ -337,7 +371,10 @@ FanArgs fan_args(const RowMoveParams& p, const void* src, void* dst, int64_t src
     a.k = p.k;
     a.N = p.N;
     a.ranks_per_node = p.ranks_per_node;
+    a.row_bytes = (int64_t)p.row_bytes;
     a.rv = (int64_t)p.row_bytes;  // bytes until the vector width is chosen
+    for (int r = 0; r < kMaxEpRanks; ++r) a.ep_bufs[r] = nullptr;
+    a.ep_capacity = 0;
     a.src_rows = src_rows;
     a.dst_rows = dst_rows;
     a.err = p.err;
@@ -373,6 +410,21 @@ cudaError_t launch_node_expand(const RowMoveParams& p, const void* staging, int6
     FanArgs a = fan_args(p, staging, recv, staging_rows, p.T * p.k);
     if (p.node_src != nullptr) return launch_fan<kNodeRows>(a, staging_rows, stream);
     return launch_fan<kNodeExpand>(a, p.T * p.N, stream);
+}
+
+cudaError_t launch_ep_dispatch(const RowMoveParams& p, const void* x, void* const* bufs,
+                               int64_t capacity_rows, cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    FanArgs a = fan_args(p, x, nullptr, p.T, INT64_MAX);
+    uintptr_t bits = (uintptr_t)p.row_bytes | reinterpret_cast<uintptr_t>(x);
+    for (int r = 0; r < p.N; ++r) {
+        a.ep_bufs[r] = bufs[r];
+        bits |= reinterpret_cast<uintptr_t>(bufs[r]);
+    }
+    a.ep_capacity = capacity_rows;
+    if (bits % 16 == 0) return launch_fan_v<kEpFlat, uint4>(a, p.T, stream);
+    if (bits % 4 == 0) return launch_fan_v<kEpFlat, uint32_t>(a, p.T, stream);
+    return launch_fan_v<kEpFlat, uint16_t>(a, p.T, stream);
 }
 
 cudaError_t launch_allgather_rows(const RowMoveParams& p, const void* x, void* gathered,

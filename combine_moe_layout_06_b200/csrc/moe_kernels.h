@@ -118,6 +118,32 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, c
 cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,
                                cudaStream_t stream);
 
+// ---- expert parallelism over sharded sources (ep.cu) ----------------------------
+// Receive buffers of at most kMaxEpRanks ranks, passed by value to kernels.
+constexpr int kMaxEpRanks = 32;
+struct EpParams {
+    int64_t T;                        // this source's tokens
+    int k, E, R, G, g;                // experts, expert ranks, sources, this source
+    const int* topk;                  // [T*k] local routes
+    const int* counts_all;            // [G*E] every source's expert counts
+    const int* local_expert_offsets;  // [E+1] from the local layout
+    const int* local_slot;            // [T*k] from the local layout
+    int* expert_offsets;              // [E+1] out: rows of each expert, concatenated buffers
+    int* rank_offsets;                // [R+1] out: first row of each rank's buffer
+    int* slot;                        // [T*k] out: row of (t, j) in the concatenation
+    int* err;
+};
+cudaError_t launch_ep_layout(const EpParams& p, cudaStream_t stream);
+// bufs[r][slot[t][j] - rank_offsets[r]] = x[t] for the rank r holding the
+// row (p.slot / p.rank_offsets are the sharded-source arrays, p.N = R);
+// rows at or beyond capacity_rows of a buffer are refused (error bit).
+cudaError_t launch_ep_dispatch(const RowMoveParams& p, const void* x, void* const* bufs,
+                               int64_t capacity_rows, cudaStream_t stream);
+// y[t] = bf16_rne(sum_j fma(w[t][j], bufs[r_j][slot[t][j] - rank_offsets[r_j]], .))
+cudaError_t launch_ep_combine(const CombineParams& p, int R, const int* rank_offsets,
+                              const void* const* bufs, int64_t capacity_rows, void* y,
+                              cudaStream_t stream);
+
 // ---- bulk-copy (TMA) engine (bulk.cu) ------------------------------------------
 // Usable when the row size and every base address are multiples of 16 bytes.
 bool bulk_eligible(size_t row_bytes, std::initializer_list<const void*> ptrs);

@@ -1,0 +1,100 @@
+"""Expert parallelism over sharded sources: the host side of one rank.
+
+With one rank per GPU, rank g routes only its own tokens and every rank's
+receive buffer holds its own experts' rows ("[None][feat] support
+non-divisible EP in MoE alltoall and slurm benchmark", TensorRT-LLM PR #13888:
+the NVLinkOneSided dispatch writes straight into peer receive buffers).  The
+one exchange on the data path is an all-gather of the per-expert counts;
+dispatch and combine are this library's kernels writing to, and reading
+from, the ranks' buffers through peer-mapped pointers.  This module holds
+only plumbing: the count exchange and receive sizes (torch.distributed), and
+the mapping of every rank's buffer into this process (CUDA IPC handles of
+torch storages).  Every step on the data runs in libmoe_layout.so.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from . import buffers, capi
+
+
+def gather_counts(local_counts: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather of every rank's int32 [E] expert counts -> [G, E], source
+    rank order.  The tensors live where the group's backend wants them (CPU
+    for gloo, the GPU for NCCL)."""
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(local_counts) for _ in range(world)]
+    dist.all_gather(parts, local_counts.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def receive_rows(counts_all: np.ndarray, num_ranks: int) -> np.ndarray:
+    """Rows each rank receives: the experts of rank r (ceil/floor partition,
+    the first E mod R ranks holding one more) summed over all sources."""
+    counts_all = np.asarray(counts_all)
+    E = counts_all.shape[1]
+    base, rem = divmod(E, num_ranks)
+    sizes = [base + (1 if r < rem else 0) for r in range(num_ranks)]
+    per_expert = counts_all.sum(axis=0)
+    out, e0 = [], 0
+    for n in sizes:
+        out.append(int(per_expert[e0:e0 + n].sum()))
+        e0 += n
+    return np.array(out, np.int64)
+
+
+def share_buffer(t: torch.Tensor, group=None) -> list:
+    """Device addresses of every rank's `t` (same shape on every rank), as
+    usable from this process: this rank's own address, and the peers'
+    through CUDA IPC mappings of their storages.  The returned list keeps the
+    mapped storages alive (second element of each pair)."""
+    storage = t.untyped_storage()
+    handle = storage._share_cuda_()
+    offset = t.storage_offset() * t.element_size()
+    handles = [None] * dist.get_world_size(group)
+    dist.all_gather_object(handles, (handle, offset), group=group)
+    me = dist.get_rank(group)
+    out = []
+    for r, (h, off) in enumerate(handles):
+        if r == me:
+            out.append((t.data_ptr(), t))
+        else:
+            peer = torch.UntypedStorage._new_shared_cuda(*h)
+            out.append((peer.data_ptr() + off, peer))
+    return out
+
+
+class ExpertParallelRank:
+    """One rank's step: local layout, count exchange, sharded-source layout,
+    dispatch into every rank's receive buffer, combine from every rank's
+    expert outputs.  `cfg` describes this rank's shard (num_tokens = its
+    tokens, num_ranks = the number of ranks, flat)."""
+
+    def __init__(self, cfg: capi.MoeConfig, rank: int, world: int, device="cuda", group=None):
+        self.cfg, self.rank, self.world, self.group = cfg, rank, world, group
+        self.local = buffers.DeviceLayout(cfg, device)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.expert_offsets = torch.zeros(cfg.num_experts + 1, **i32)
+        self.rank_offsets = torch.zeros(cfg.num_ranks + 1, **i32)
+        self.slot = torch.zeros(max(cfg.num_tokens * cfg.top_k, 1), **i32)
+        self.ep = capi.ep_layout_struct(self.expert_offsets, self.rank_offsets, self.slot)
+        self.counts_all = None
+
+    def layout(self, topk: torch.Tensor, exchange_device="cpu") -> np.ndarray:
+        """Local layout, count exchange, sharded-source layout.  Returns the
+        rows every rank receives (host int64 [R])."""
+        capi.moe_layout(self.cfg, topk, self.local.struct)
+        counts = self.local.expert_counts.to(exchange_device)
+        counts_all = gather_counts(counts, self.group)
+        self.counts_all = counts_all.to(self.local.expert_counts.device)
+        capi.moe_ep_layout(self.cfg, self.rank, self.world, topk, self.counts_all,
+                           self.local.struct, self.ep)
+        return receive_rows(counts_all.cpu().numpy(), self.cfg.num_ranks)
+
+    def dispatch(self, x: torch.Tensor, recv_bufs, capacity_rows: int) -> None:
+        capi.moe_ep_dispatch(self.cfg, self.local.struct, self.ep, x, recv_bufs, capacity_rows)
+
+    def combine(self, expert_out_bufs, capacity_rows: int, w: torch.Tensor, y: torch.Tensor) -> None:
+        capi.moe_ep_combine(self.cfg, self.local.struct, self.ep, expert_out_bufs, capacity_rows, w, y)

@@ -278,6 +278,69 @@ moe_status_t moe_combine_reducescatter(const moe_config_t *cfg, const moe_layout
                                        const void *expert_out, const float *topk_weights,
                                        float *partial, void *y, void *stream);
 
+/* ---- expert parallelism over sharded sources ----
+ * With one rank per GPU, rank g routes only its own T_g tokens and every
+ * rank's receive buffer holds its own experts' rows ("[None][feat] support
+ * non-divisible EP in MoE alltoall and slurm benchmark", TensorRT-LLM PR
+ * #13888: the NVLinkOneSided dispatch writes straight into peer receive
+ * buffers; FUSCO article, "FUSCO 的核心创新": every row goes straight to its
+ * final position).  Order inside rank r's buffer: expert-major, then source
+ * rank, then the source's token order.  When the sources are contiguous token
+ * ranges of one batch in rank order, the rows equal moe_layout()'s on the
+ * whole batch.  One step on rank g:
+ *   1. moe_layout(cfg_g, topk_g, local) over its own tokens (cfg_g.num_tokens
+ *      = T_g, flat, num_ranks = R): local->expert_counts are its counts;
+ *   2. the caller gathers every rank's expert_counts into counts_all
+ *      ([G][E], device, source-major), e.g. with an NCCL all-gather;
+ *   3. moe_ep_layout(): the rows of the concatenated receive buffers;
+ *   4. moe_ep_dispatch() into the R receive buffers (peer-mapped pointers),
+ *      then a barrier across ranks, the experts, another barrier, and
+ *   5. moe_ep_combine() from the R expert-output buffers.
+ * No entry point synchronises ranks; barriers and buffer mapping are the
+ * caller's.  num_ranks <= MOE_MAX_NODES, and MOE_FLAG_TWO_LEVEL is refused. */
+
+/* Rows in the concatenation of all ranks' receive buffers (device int32,
+ * caller-owned):
+ *   expert_offsets [E+1]   first row of each expert (last = total rows)
+ *   rank_offsets   [R+1]   rank r's buffer holds rows [rank_offsets[r],
+ *                          rank_offsets[r+1]); its local row is the
+ *                          difference from rank_offsets[r]
+ *   slot           [T_g*k] row of this rank's (t, j), -1 if the route was
+ *                          invalid */
+typedef struct moe_ep_layout {
+    int32_t *expert_offsets;
+    int32_t *rank_offsets;
+    int32_t *slot;
+} moe_ep_layout_t;
+
+/* Step 3.  cfg: this rank's shard (as in step 1); source_rank g in
+ * [0, num_sources); counts_all: device int32 [num_sources][E] with row g equal
+ * to local->expert_counts; topk_idx: the shard's routes; local: the layout of
+ * step 1 (its expert_offsets, slot and error_word are read).  Every rank
+ * computes the same expert_offsets and rank_offsets. */
+moe_status_t moe_ep_layout(const moe_config_t *cfg, int32_t source_rank, int32_t num_sources,
+                           const int32_t *topk_idx, const int32_t *counts_all,
+                           const moe_layout_t *local, const moe_ep_layout_t *ep, void *stream);
+
+/* Step 4: bufs[r][slot[t][j] - rank_offsets[r]] = x[t] for every (t, j).
+ *   recv_bufs     HOST array of num_ranks device pointers (this GPU's or
+ *                 peers', e.g. CUDA IPC mappings), each bf16 rows of `hidden`
+ *   capacity_rows rows each buffer holds; a row at or beyond it is skipped
+ *                 and reported (MOE_ERR_BAD_LAYOUT) */
+moe_status_t moe_ep_dispatch(const moe_config_t *cfg, const moe_layout_t *local,
+                             const moe_ep_layout_t *ep, const void *x, void *const *recv_bufs,
+                             int64_t capacity_rows, void *stream);
+
+/* Step 5: y[t] = bf16_rne( sum_{j=0..k-1} w[t][j] * eo_r[slot[t][j] -
+ * rank_offsets[r]] ), r the rank holding the row, fp32 FMA in column order
+ * as in moe_combine().
+ *   expert_out_bufs  HOST array of num_ranks device pointers, bf16 rows laid
+ *                    out like the receive buffers */
+moe_status_t moe_ep_combine(const moe_config_t *cfg, const moe_layout_t *local,
+                            const moe_ep_layout_t *ep, const void *const *expert_out_bufs,
+                            int64_t capacity_rows, const float *topk_weights, void *y,
+                            void *stream);
+
 /* ---- fp8 (e4m3) payload ----
  * TensorRT-LLM PR #13888 (ConfigurableMoE commit) validates an fp8
  * low-precision combine at rtol 0.02 / atol 0.15.  Rows are carried as OCP
