@@ -383,6 +383,8 @@ def main():
                    help="skip timing the all-gather / reduce-scatter comparison path")
     p.add_argument("--no-node-balance", action="store_true",
                    help="skip timing the two node expansions on a hot-node routing")
+    p.add_argument("--no-ep", action="store_true",
+                   help="skip timing expert parallelism over sharded sources (virtual ranks)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--ref-tokens", type=int, default=0)
@@ -426,10 +428,39 @@ def main():
     eo_bits = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
     bf16 = dict(dtype=torch.bfloat16, device=dev)
 
+    # Expert parallelism over sharded sources with every rank on this GPU:
+    # rank g routes tokens [sb[g], sb[g+1]); its receive and expert-output
+    # buffers are the rank's rows of the set's recv / eo (pointer tables).
+    G = wl.R
+    sb = (np.arange(G + 1, dtype=np.int64) * wl.T) // G
+    from combine_moe_layout_06_b200 import ep as epmod
+    shard_counts = np.stack([np.bincount(d["topk_idx"][sb[g]:sb[g + 1]].ravel(), minlength=wl.E)
+                             for g in range(G)])
+    ep_rows = epmod.receive_rows(shard_counts, wl.R)
+    ep_first = np.concatenate([[0], np.cumsum(ep_rows)])
+    ep_cfgs = [capi.config(int(sb[g + 1] - sb[g]), wl.H, wl.E, wl.k, wl.R, 1,
+                           flags & (capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK))
+               for g in range(G)]
+
+    class EpShards:
+        """Per-rank layouts and sharded-source arrays of one buffer set."""
+
+        def __init__(self, b):
+            i32 = dict(dtype=torch.int32, device=dev)
+            self.lays = [buffers.DeviceLayout(c, dev) for c in ep_cfgs]
+            self.counts_all = torch.zeros((G, wl.E), **i32)
+            self.arrays = [(torch.zeros(wl.E + 1, **i32), torch.zeros(wl.R + 1, **i32),
+                            torch.zeros(max(c.num_tokens * wl.k, 1), **i32)) for c in ep_cfgs]
+            self.structs = [capi.ep_layout_struct(*a) for a in self.arrays]
+            row = wl.H * 2
+            self.recv_bufs = [b.recv.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
+            self.eo_bufs = [b.eo.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
+            self.cap = int(ep_rows.max())
+
     class BufferSet:
         """One independent set of the step's inputs and outputs."""
 
-        def __init__(self, decoupled=False, agrs=False, fp8=False):
+        def __init__(self, decoupled=False, agrs=False, fp8=False, ep=False):
             self.lay = buffers.DeviceLayout(cfg, dev)
             self.x = buffers.bf16_from_bits(d["x"], dev)
             self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
@@ -458,11 +489,13 @@ def main():
             if agrs:
                 self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
                 self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
+            self.ep = EpShards(self) if ep else None
 
     with_decoupled = not args.no_decoupled
     with_agrs = not args.no_agrs and wl.R <= capi.MOE_MAX_NODES
     with_fp8 = not args.no_fp8 and wl.H % 8 == 0 and not wl.two_level
-    sets = [BufferSet(with_decoupled, with_agrs, with_fp8), BufferSet(with_decoupled, with_agrs, with_fp8)]
+    with_ep = not args.no_ep and wl.R <= capi.MOE_MAX_NODES and not wl.two_level
+    sets = [BufferSet(with_decoupled, with_agrs, with_fp8, with_ep) for _ in range(2)]
 
     def layout(b):
         capi.moe_layout(cfg, b.topk, b.lay.struct)
@@ -491,6 +524,43 @@ def main():
         fp8_layout_dispatch(b)
         capi.moe_combine_fp8(cfg, b.lay.struct, b.eo_q, b.eo_s, b.w, b.y)
 
+    ep_streams = [torch.cuda.Stream(dev) for _ in range(G)] if wl.R <= capi.MOE_MAX_NODES else []
+
+    def ep_phase(fn):
+        """Run fn(g) for every rank on its own stream, all after the work
+        enqueued so far and before anything enqueued later (the ranks of a
+        multi-GPU system run concurrently; the joins stand for its barriers)."""
+        cur = torch.cuda.current_stream()
+        for st in ep_streams:
+            st.wait_stream(cur)
+        for g, st in enumerate(ep_streams):
+            with torch.cuda.stream(st):
+                fn(g)
+        for st in ep_streams:
+            cur.wait_stream(st)
+
+    def ep_step(b):
+        e = b.ep
+        sh = lambda t, g: t[int(sb[g]):int(sb[g + 1])]
+
+        def local(g):
+            capi.moe_layout(ep_cfgs[g], sh(b.topk, g), e.lays[g].struct)
+            e.counts_all[g].copy_(e.lays[g].expert_counts)   # the count all-gather
+
+        def send(g):
+            capi.moe_ep_layout(ep_cfgs[g], g, G, sh(b.topk, g), e.counts_all, e.lays[g].struct,
+                               e.structs[g])
+            capi.moe_ep_dispatch(ep_cfgs[g], e.lays[g].struct, e.structs[g], sh(b.x, g),
+                                 e.recv_bufs, e.cap)
+
+        def gather(g):
+            capi.moe_ep_combine(ep_cfgs[g], e.lays[g].struct, e.structs[g], e.eo_bufs, e.cap,
+                                sh(b.w, g), sh(b.y, g))
+
+        ep_phase(local)
+        ep_phase(send)
+        ep_phase(gather)
+
     def agrs_step(b):
         layout(b)
         capi.moe_dispatch_allgather(cfg, b.lay.struct, b.x, b.gathered, b.recv)
@@ -509,9 +579,11 @@ def main():
             agrs_step(sets[i % 2])
         if with_fp8:
             fp8_step(sets[i % 2])
+        if with_ep:
+            ep_step(sets[i % 2])
     torch.cuda.synchronize()
     for b in sets:
-        for lay in [b.lay] + ([b.dlay] if with_decoupled else []):
+        for lay in [b.lay] + ([b.dlay] if with_decoupled else []) + (b.ep.lays if with_ep else []):
             st = capi.moe_get_error(lay.struct)
             if st != capi.MOE_OK:
                 raise SystemExit(f"device error after warm-up: {capi.moe_status_string(st)}")
@@ -542,6 +614,8 @@ def main():
         graphs["fp8"] = (capture(lambda: (fp8_step(A), fp8_step(B))), capture(lambda: fp8_step(A)))
         graphs["fp8_LD"] = (capture(lambda: (fp8_layout_dispatch(A), fp8_layout_dispatch(B))),
                             capture(lambda: fp8_layout_dispatch(A)))
+    if with_ep:
+        graphs["ep"] = (capture(lambda: (ep_step(A), ep_step(B))), capture(lambda: ep_step(A)))
     for pair, single in graphs.values():
         pair.replay()
         single.replay()
@@ -596,6 +670,7 @@ def main():
         agrs_ms = timed("agrs", K) if with_agrs else None
         fp8_ms = timed("fp8", K) if with_fp8 else None
         fp8_ld = timed("fp8_LD", K) / K if with_fp8 else None
+        ep_ms = timed("ep", K) if with_ep else None
         flushed = flushed_steps(K)
     ms_per_step = total_ms / K
     t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
@@ -648,6 +723,22 @@ def main():
         with ClockSampler(local) as nb_clocks:
             balance = node_balance(args, dev, world, barrier, flags)
         balance["clocks"] = nb_clocks.summary()
+
+    ep_line = None
+    if ep_ms is not None:
+        for b in sets:
+            for lay in b.ep.lays:
+                st = capi.moe_get_error(lay.struct)
+                if st != capi.MOE_OK:
+                    raise SystemExit(f"device error in the sharded-source run: {capi.moe_status_string(st)}")
+        ep_value = job_gbs(step_bytes, world, K, ep_ms * 1e-3)
+        ep_line = {"value": round(ep_value, 2), "unit": "GB/s", "ms_per_step": round(ep_ms / K, 5),
+                   "ranks": G, "vs_single_source": round(ep_value / value, 3),
+                   "receive_rows": [int(r) for r in ep_rows],
+                   "path": f"{G} source ranks on this GPU, one stream each, joined between "
+                           "phases: layout of its shard and the count all-gather (device copies); "
+                           "sharded-source layout and dispatch into every rank's receive buffer; "
+                           "combine from every rank's expert outputs (pointer tables)"}
 
     # End to end through the C ABI from pinned host buffers, pipelined over
     # the two buffer sets: step i's inputs go up on a copy stream while step
@@ -737,6 +828,7 @@ def main():
             "allgather_reducescatter": agrs,
             "fp8_payload": fp8,
             "node_balance": balance,
+            "expert_parallel_virtual_ranks": ep_line,
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
