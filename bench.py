@@ -486,6 +486,10 @@ def main():
                 self.eo_s = torch.empty(rows, dtype=torch.float32, device=dev)
                 # expert outputs as an fp8 producer would emit them
                 capi.moe_quantize_rows_fp8(self.eo, rows, wl.H, self.eo_q, self.eo_s)
+                if wl.two_level:
+                    srows = capi.moe_node_staging_rows(cfg)
+                    self.st_q = torch.empty((srows, wl.H), dtype=torch.uint8, device=dev)
+                    self.st_s = torch.empty(srows, dtype=torch.float32, device=dev)
             if agrs:
                 self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
                 self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
@@ -493,7 +497,7 @@ def main():
 
     with_decoupled = not args.no_decoupled
     with_agrs = not args.no_agrs and wl.R <= capi.MOE_MAX_NODES
-    with_fp8 = not args.no_fp8 and wl.H % 8 == 0 and not wl.two_level
+    with_fp8 = not args.no_fp8 and wl.H % 8 == 0
     with_ep = not args.no_ep and wl.R <= capi.MOE_MAX_NODES and not wl.two_level
     sets = [BufferSet(with_decoupled, with_agrs, with_fp8, with_ep) for _ in range(2)]
 
@@ -518,7 +522,10 @@ def main():
 
     def fp8_layout_dispatch(b):
         layout(b)
-        capi.moe_dispatch_fp8(cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
+        if wl.two_level:
+            capi.moe_dispatch_fp8_two_level(cfg, b.lay.struct, b.x, b.st_q, b.st_s, b.recv_q, b.recv_s)
+        else:
+            capi.moe_dispatch_fp8(cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
 
     def fp8_step(b):
         fp8_layout_dispatch(b)
@@ -714,8 +721,10 @@ def main():
                "kernels_ms": {"dispatch": round(fp8_ld - t_l, 5),
                               "combine": round(fp8_ms / K - fp8_ld, 5)},
                "bytes_per_step": fp8_bytes,
-               "path": "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + "
-                       "fp8 combine (expert rows already e4m3)"}
+               "path": ("layout + fp8 two-level dispatch (quantize once into node staging, "
+                        "expand codes and scales; staging not credited) + " if wl.two_level else
+                        "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + ")
+                       + "fp8 combine (expert rows already e4m3)"}
 
     graphs.clear()
     balance = None

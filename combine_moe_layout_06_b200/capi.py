@@ -50,7 +50,7 @@ ENTRY_POINTS = (
     "moe_combine", "moe_get_error", "moe_dispatch_decoupled", "moe_combine_decoupled",
     "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
     "moe_combine_reducescatter", "moe_quantize_rows_fp8", "moe_dispatch_fp8", "moe_combine_fp8",
-    "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine",
+    "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine", "moe_dispatch_fp8_two_level",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -114,6 +114,7 @@ def lib() -> ctypes.CDLL:
     L.moe_quantize_rows_fp8.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, P]
     L.moe_dispatch_fp8.argtypes = [C, LP, P, P, P, P]
     L.moe_combine_fp8.argtypes = [C, LP, P, P, P, P, P]
+    L.moe_dispatch_fp8_two_level.argtypes = [C, LP, P, P, P, P, P, P]
     EP = ctypes.POINTER(MoeEpLayout)
     PP = ctypes.POINTER(ctypes.c_void_p)
     L.moe_ep_layout.argtypes = [C, ctypes.c_int32, ctypes.c_int32, P, P, LP, EP, P]
@@ -292,6 +293,14 @@ def moe_dispatch_fp8(cfg: MoeConfig, layout: MoeLayout, x, recv_q, recv_scale,
                      stream=None) -> None:
     _check(lib().moe_dispatch_fp8(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x), _ptr(recv_q),
                                   _ptr(recv_scale), _stream(stream)), "moe_dispatch_fp8")
+
+
+def moe_dispatch_fp8_two_level(cfg: MoeConfig, layout: MoeLayout, x, staging_q, staging_scale,
+                               recv_q, recv_scale, stream=None) -> None:
+    _check(lib().moe_dispatch_fp8_two_level(ctypes.byref(cfg), ctypes.byref(layout), _ptr(x),
+                                            _ptr(staging_q), _ptr(staging_scale), _ptr(recv_q),
+                                            _ptr(recv_scale), _stream(stream)),
+           "moe_dispatch_fp8_two_level")
 
 
 def moe_combine_fp8(cfg: MoeConfig, layout: MoeLayout, eo_q, eo_scale, topk_weights, y,

@@ -424,6 +424,38 @@ moe_status_t moe_dispatch_fp8(const moe_config_t* c, const moe_layout_t* L, cons
                                                 static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_dispatch_fp8_two_level(const moe_config_t* c, const moe_layout_t* L, const void* x,
+                                        void* staging_q, float* staging_scale, void* recv_q,
+                                        float* recv_scale, void* stream) {
+    moe_status_t st = moe_check_config(c);
+    if (st != MOE_OK) return st;
+    if (!two_level(c)) return MOE_ERR_INVALID_ARG;
+    st = check_layout_ptrs(c, L);
+    if (st != MOE_OK) return st;
+    if (c->num_tokens == 0) return MOE_OK;
+    if (x == nullptr || staging_q == nullptr || staging_scale == nullptr || recv_q == nullptr ||
+        recv_scale == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (!moe::fp8_eligible(c->hidden, {x}, {staging_q, recv_q})) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t rows = staging_rows(c);
+    // phase 1: each token quantized once, into the staging row of every node it touches
+    cudaError_t e = moe::launch_quantize_fp8(x, c->num_tokens, c->hidden, L->node_slot, c->num_nodes,
+                                             rows, staging_q, staging_scale, L->error_word, s,
+                                             L->node_offsets);
+    // phase 2: the node expansion, once over the codes and once over the scales
+    moe::RowMoveParams p = move_params(c, L);
+    if (e == cudaSuccess) {
+        p.row_bytes = (size_t)c->hidden;
+        e = moe::launch_node_expand(p, staging_q, rows, recv_q, s);
+    }
+    if (e == cudaSuccess) {
+        p.row_bytes = sizeof(float);
+        e = moe::launch_node_expand(p, staging_scale, rows, recv_scale, s);
+    }
+    return cuda_status(e);
+}
+
 moe_status_t moe_combine_fp8(const moe_config_t* c, const moe_layout_t* L, const void* eo_q,
                              const float* eo_scale, const float* topk_weights, void* y,
                              void* stream) {

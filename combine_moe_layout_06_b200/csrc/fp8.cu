@@ -60,12 +60,29 @@ struct Fp8Args {
     uint2* q;             // e4m3 rows, 8 codes per vector
     float* scale;         // one per destination row
     const int* slot;      // nullptr: the destination of row r is row r
+    const int* dst_base;  // nullptr, or per-column first rows (node staging)
     int64_t rows;         // source rows
     int k;                // destinations per source row (slot mode)
     int64_t rv;           // vectors per row (H / 8)
     int64_t dst_rows;
     int* err;
 };
+
+// Lane j's destination row of source row r (-1: none): row r itself, or
+// dst_base[j] + slot[r][j] for j < k (a receive row, or a node's staging row).
+__device__ __forceinline__ int64_t quant_dst(const Fp8Args& a, int64_t r, int lane, int& errbits) {
+    if (a.slot == nullptr) return lane == 0 ? r : -1;
+    if (lane >= a.k) return -1;
+    const int s = ld_dep(a.slot + r * a.k + lane);
+    if (s < 0) {
+        if (s != -1) errbits |= kErrBadLayout;
+        return -1;
+    }
+    const int64_t d = (a.dst_base ? (int64_t)ld_dep(a.dst_base + lane) : 0) + s;
+    if (d < a.dst_rows) return d;
+    errbits |= kErrBadLayout;
+    return -1;
+}
 
 __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
     pdl_trigger();
@@ -74,14 +91,7 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
     const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
     int errbits = 0;
     for (int64_t r = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); r < a.rows; r += nw) {
-        int64_t dst = -1;
-        if (a.slot == nullptr) {
-            dst = lane == 0 ? r : -1;
-        } else if (lane < a.k) {
-            const int s = ld_dep(a.slot + r * a.k + lane);
-            if (s >= 0 && s < a.dst_rows) dst = s;
-            else if (s != -1) errbits |= kErrBadLayout;
-        }
+        const int64_t dst = quant_dst(a, r, lane, errbits);
         const uint4* src = a.src + r * a.rv;
         uint32_t amax_bits = 0;
         for (int64_t v = lane; v < a.rv; v += 32) {
@@ -129,14 +139,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows16_kernel(Fp8Args a) {
     const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
     int errbits = 0;
     for (int64_t r = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); r < a.rows; r += nw) {
-        int64_t dst = -1;
-        if (a.slot == nullptr) {
-            dst = lane == 0 ? r : -1;
-        } else if (lane < a.k) {
-            const int s = ld_dep(a.slot + r * a.k + lane);
-            if (s >= 0 && s < a.dst_rows) dst = s;
-            else if (s != -1) errbits |= kErrBadLayout;
-        }
+        const int64_t dst = quant_dst(a, r, lane, errbits);
         const uint4* src = a.src + r * a.rv;
         uint4 raw[NG][2];
 #pragma unroll
@@ -432,13 +435,14 @@ cudaError_t launch_rows16(const Fp8Args& a, cudaStream_t stream) {
 
 cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
                                 int64_t dst_rows, void* q, float* scale, int* err,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const int* dst_base) {
     if (rows <= 0) return cudaSuccess;
     Fp8Args a;
     a.src = static_cast<const uint4*>(src);
     a.q = static_cast<uint2*>(q);
     a.scale = scale;
     a.slot = slot;
+    a.dst_base = dst_base;
     a.rows = rows;
     a.k = k;
     a.rv = hidden / 8;

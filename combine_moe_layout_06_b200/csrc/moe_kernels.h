@@ -110,10 +110,11 @@ cudaError_t launch_reduce_rank_partials(const CombineParams& p, int R, const flo
 bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
                   std::initializer_list<const void*> q_ptrs);
 // Quantize `rows` bf16 rows (amax scale per row).  slot == nullptr: row r ->
-// q row r; else row r goes to q rows slot[r*k + j] (j < k), bounded by dst_rows.
+// q row r; else row r goes to q rows dst_base[j] + slot[r*k + j] (j < k,
+// slot >= 0; dst_base nullptr = 0), bounded by dst_rows.
 cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
                                 int64_t dst_rows, void* q, float* scale, int* err,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const int* dst_base = nullptr);
 // y[t] = bf16_rne(sum_j fma(w[t][j] * scale[slot], decode(q[slot]), .))
 cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,
                                cudaStream_t stream);

@@ -365,6 +365,18 @@ moe_status_t moe_quantize_rows_fp8(const void *src, int64_t rows, int32_t hidden
 moe_status_t moe_dispatch_fp8(const moe_config_t *cfg, const moe_layout_t *layout, const void *x,
                               void *recv_q, float *recv_scale, void *stream);
 
+/* Two-level dispatch with an fp8 payload (MOE_FLAG_TWO_LEVEL required):
+ * each x row is quantized once, into the staging row of every node it
+ * touches (codes and scale, as moe_dispatch() stages bf16 rows), and the
+ * node expansion then copies codes and scales to the receive rows.  Results
+ * equal moe_dispatch_fp8() on the same layout bit for bit.
+ *   staging_q      device uint8 [moe_node_staging_rows()][H]
+ *   staging_scale  device fp32 [moe_node_staging_rows()]
+ *   recv_q, recv_scale  as for moe_dispatch_fp8() */
+moe_status_t moe_dispatch_fp8_two_level(const moe_config_t *cfg, const moe_layout_t *layout,
+                                        const void *x, void *staging_q, float *staging_scale,
+                                        void *recv_q, float *recv_scale, void *stream);
+
 /* Fused combine of fp8 expert rows: coef_j = w[t][j] * scale[slot[t][j]]
  * (fp32), acc = fma(coef_j, decode(code), acc) for j = 0..k-1 from +0, one
  * bf16 round-to-nearest-even store.

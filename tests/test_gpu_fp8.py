@@ -123,6 +123,36 @@ def test_fp8_workload_olmoe(oracle_mod):
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
+@pytest.mark.parametrize("node_src", [True, False])
+@pytest.mark.parametrize("T,H,E,k,R,N", [
+    (33, 136, 13, 4, 5, 5),
+    (257, 2048, 64, 8, 4, 2),
+    (600, 7168, 32, 8, 8, 4),       # beyond the register-resident quantizer
+])
+def test_fp8_two_level(oracle_mod, T, H, E, k, R, N, node_src):
+    d = inputs.make_random(T, H, E, k, seed=T + N)
+    x, topk = d["x"], d["topk_idx"]
+    ref = oracle_mod.layout(topk, E, R, N, nodes=True)
+    cfg = M.cfg_of(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL)
+    lay, _ = M.gpu_layout(cfg, topk, node_src=node_src)
+    rows = capi.moe_node_staging_rows(cfg)
+    st_q = torch.full((rows, H), 0x55, dtype=torch.uint8, device="cuda")
+    st_s = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    recv_q = torch.empty((T * k, H), dtype=torch.uint8, device="cuda")
+    recv_s = torch.empty(T * k, dtype=torch.float32, device="cuda")
+    capi.moe_dispatch_fp8_two_level(cfg, lay.struct, M.to_dev(x), st_q, st_s, recv_q, recv_s)
+    rq, rs = oracle_mod.dispatch_fp8(x, ref["slot"])
+    assert np.array_equal(_u8(recv_q), rq)
+    assert np.array_equal(recv_s.cpu().numpy(), rs)
+    # staging row u holds the codes of token node_src[u]; rows beyond U untouched
+    xq, xs = oracle_mod.quantize_rows_fp8(x)
+    U = int(ref["node_offsets"][-1])
+    assert np.array_equal(_u8(st_q)[:U], xq[ref["node_src"]])
+    assert np.array_equal(st_s.cpu().numpy()[:U], xs[ref["node_src"]])
+    assert np.all(_u8(st_q)[U:] == 0x55)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
 def test_fp8_refusals():
     cfg = M.cfg_of(4, 12, 8, 2, 2)                       # hidden % 8 != 0
     lay, _ = M.gpu_layout(cfg, np.array([[0, 1], [2, 3], [4, 5], [6, 7]], np.int32))
@@ -135,4 +165,8 @@ def test_fp8_refusals():
     two = M.cfg_of(4, 16, 8, 2, 2, 2, capi.MOE_FLAG_TWO_LEVEL)
     with pytest.raises(capi.MoeError) as ei:
         capi.moe_dispatch_fp8(two, lay.struct, x, q, s)
+    assert ei.value.status == capi.MOE_ERR_INVALID_ARG
+    flat = M.cfg_of(4, 16, 8, 2, 2)
+    with pytest.raises(capi.MoeError) as ei:                 # the staged form needs node staging
+        capi.moe_dispatch_fp8_two_level(flat, lay.struct, x, q, s, q, s)
     assert ei.value.status == capi.MOE_ERR_INVALID_ARG
