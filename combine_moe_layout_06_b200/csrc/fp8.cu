@@ -98,7 +98,10 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
             float f[8];
             unpack_bf16<uint4>(ld_stream(src + v), f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) amax_bits = max(amax_bits, __float_as_uint(fabsf(f[e])));
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t b = __float_as_uint(fabsf(f[e]));
+                if (b <= 0x7F800000u) amax_bits = max(amax_bits, b);   // NaNs have no magnitude
+            }
         }
         amax_bits = __reduce_max_sync(kFullMask, amax_bits);
         const float amax = __uint_as_float(amax_bits);
@@ -129,16 +132,18 @@ __global__ void __launch_bounds__(kThreads) quantize_fp8_kernel(Fp8Args a) {
     warp_report(a.err, errbits);
 }
 
-// Register-resident row: NG 16-value groups per lane (H <= 512 * NG).
-template <int NG>
-__global__ void __launch_bounds__(kThreads) quantize_rows16_kernel(Fp8Args a) {
+// Register-resident row: NG 16-value groups per lane (H <= 512 * NG), W
+// warps per CTA.  Codes are made one group at a time and stored to every
+// destination at once, so only the raw row stays in registers.
+template <int NG, int W>
+__global__ void __launch_bounds__(W * 32) quantize_rows16_kernel(Fp8Args a) {
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t G = a.rv / 2;  // 16-value groups per row
-    const int64_t nw = (int64_t)gridDim.x * kWarpsPerCta;
+    const int64_t nw = (int64_t)gridDim.x * W;
     int errbits = 0;
-    for (int64_t r = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5); r < a.rows; r += nw) {
+    for (int64_t r = (int64_t)blockIdx.x * W + (threadIdx.x >> 5); r < a.rows; r += nw) {
         const int64_t dst = quant_dst(a, r, lane, errbits);
         const uint4* src = a.src + r * a.rv;
         uint4 raw[NG][2];
@@ -151,21 +156,31 @@ __global__ void __launch_bounds__(kThreads) quantize_rows16_kernel(Fp8Args a) {
                 raw[i][1] = ld_stream(src + 2 * g + 1);
             }
         }
-        uint32_t amax_bits = 0;
+        // |v| of a bf16 orders like its low 15 bits (infinity above every
+        // finite value): a per-halfword integer max finds amax's bits; NaNs
+        // (above 0x7F80) have no magnitude and are masked out
+        uint32_t m2 = 0;
+        auto fold = [&](uint32_t w) {
+            const uint32_t x = w & 0x7FFF7FFFu;
+            m2 = __vmaxu2(m2, x & ~__vcmpgtu2(x, 0x7F807F80u));
+        };
 #pragma unroll
         for (int i = 0; i < NG; ++i)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                float f[8];
-                unpack_bf16<uint4>(raw[i][h], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) amax_bits = max(amax_bits, __float_as_uint(fabsf(f[e])));
+                fold(raw[i][h].x);
+                fold(raw[i][h].y);
+                fold(raw[i][h].z);
+                fold(raw[i][h].w);
             }
+        uint32_t amax_bits = max(m2 & 0xFFFFu, m2 >> 16) << 16;
         amax_bits = __reduce_max_sync(kFullMask, amax_bits);
         const float amax = __uint_as_float(amax_bits);
         const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
         const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
-        uint4 code[NG];
+        if (dst >= 0) a.scale[dst] = scale;
+        const unsigned dmask = __ballot_sync(kFullMask, dst >= 0);
+        uint4* q = reinterpret_cast<uint4*>(a.q);
 #pragma unroll
         for (int i = 0; i < NG; ++i) {
             uint2 c[2];
@@ -177,20 +192,14 @@ __global__ void __launch_bounds__(kThreads) quantize_rows16_kernel(Fp8Args a) {
                 for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
                 c[h] = to_e4m3x8(f);
             }
-            code[i] = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
-        }
-        if (dst >= 0) a.scale[dst] = scale;
-        unsigned m = __ballot_sync(kFullMask, dst >= 0);
-        uint4* q = reinterpret_cast<uint4*>(a.q);
-        while (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1;
-            const int64_t d = __shfl_sync(kFullMask, dst, j);
-            uint4* qrow = q + d * G;
-#pragma unroll
-            for (int i = 0; i < NG; ++i) {
-                const int64_t g = lane + 32 * i;
-                if (g < G) st_stream(qrow + g, code[i]);
+            const uint4 code = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+            const int64_t g = lane + 32 * i;
+            unsigned m = dmask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int64_t d = __shfl_sync(kFullMask, dst, j);
+                if (g < G) st_stream(q + d * G + g, code);
             }
         }
     }
@@ -425,11 +434,11 @@ bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
 }
 
 namespace {
-template <int NG>
+template <int NG, int W>
 cudaError_t launch_rows16(const Fp8Args& a, cudaStream_t stream) {
-    constexpr auto kern = quantize_rows16_kernel<NG>;
-    const int grid = persistent_grid<kern>(a.rows, kThreads);
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+    constexpr auto kern = quantize_rows16_kernel<NG, W>;
+    const int grid = persistent_grid<kern>(a.rows, W * 32);
+    return launch_pdl(kern, dim3(grid), dim3(W * 32), 0, stream, a);
 }
 }  // namespace
 
@@ -451,9 +460,10 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, c
     // register-resident rows when the row splits into 16-value groups, at
     // most 8 per lane, and the codes take 16-byte stores
     const bool wide = hidden % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 16 == 0;
-    if (wide && hidden <= 512 * 2) return launch_rows16<2>(a, stream);
-    if (wide && hidden <= 512 * 4) return launch_rows16<4>(a, stream);
-    if (wide && hidden <= 512 * 8) return launch_rows16<8>(a, stream);
+    if (wide && hidden <= 512 * 2) return launch_rows16<2, 8>(a, stream);
+    if (wide && hidden <= 512 * 4) return launch_rows16<4, 8>(a, stream);
+    if (wide && hidden <= 512 * 8) return launch_rows16<8, 8>(a, stream);
+    if (wide && hidden <= 512 * 16) return launch_rows16<16, 4>(a, stream);
     constexpr auto kern = quantize_fp8_kernel;
     const int grid = persistent_grid<kern>(rows, kThreads);
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);

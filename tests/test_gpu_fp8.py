@@ -90,6 +90,9 @@ def test_fp8_zero_and_extreme_rows(oracle_mod):
     x[3] = 0                                     # zero row: scale 1, codes 0
     x[5, 7] = 0x7F7F                             # bf16 max: scale huge
     x[6] = 0x0001                                # a bf16 subnormal row
+    x[8, 3] = 0x7FC0                             # NaNs among finite values: no magnitude
+    x[8, 5] = 0xFFC0
+    x[9, 0] = 0x7F80                             # +infinity: scale inf, the rest code 0
     ref = oracle_mod.layout(d["topk_idx"], E, R)
     cfg = M.cfg_of(T, H, E, k, R)
     lay, _ = M.gpu_layout(cfg, d["topk_idx"])

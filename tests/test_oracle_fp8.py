@@ -71,6 +71,21 @@ def test_quantize_rows_closed_forms(oracle_mod):
     assert np.all(err <= 2.0 ** -4 * np.abs(xf) + scale[:, None] * 2.0 ** -10 + 1e-30)
 
 
+def test_quantize_rows_nan_has_no_magnitude(oracle_mod):
+    x = inputs.random_bf16((3, 40), seed=8, scale=2.0)
+    x[0, 3] = 0x7FC0                      # quiet NaN
+    x[0, 9] = 0xFFC0                      # negative quiet NaN
+    clean = x.copy()
+    clean[0, [3, 9]] = 0                  # the same row with zeros where the NaNs are
+    q, s = oracle_mod.quantize_rows_fp8(x)
+    qc, sc = oracle_mod.quantize_rows_fp8(clean)
+    assert s[0] == sc[0], "the scale comes from the finite values"
+    assert q[0, 3] == 0x7F and q[0, 9] == 0x7F
+    keep = np.ones(40, bool)
+    keep[[3, 9]] = False
+    assert np.array_equal(q[0, keep], qc[0, keep])
+
+
 def test_dispatch_fp8_rows_are_copies(oracle_mod):
     d = inputs.make_random(60, 32, 12, 4, seed=9)
     lay = oracle_mod.layout(d["topk_idx"], 12, 3)
