@@ -136,6 +136,29 @@ def test_skewed_node_loads(oracle_mod, engine, hot_frac):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
+def test_combine_nan_and_infinity_propagate(oracle_mod):
+    """Non-finite expert outputs: NaN where the oracle has NaN (any payload;
+    the GPU stores bf16 NaNs in canonical form), every other value bit for
+    bit, infinities included."""
+    T, H, E, k, R = 300, 64, 16, 4, 4
+    d = inputs.make_random(T, H, E, k, seed=12)
+    ref = oracle_mod.layout(d["topk_idx"], E, R)
+    eo = inputs.random_bf16_bits((T * k, H), seed=13)
+    eo[5, 3] = 0x7FC0                                  # NaN
+    eo[9, 0] = 0xFFC1                                  # negative NaN, odd payload
+    eo[20, 7] = 0x7F80                                 # +inf
+    eo[21, 7] = 0xFF80                                 # -inf (inf - inf where both meet)
+    eo[40, 2] = 0x7F80
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, d["topk_idx"])
+    y = M.bits(M.gpu_combine(cfg, lay, M.to_dev(eo), d["topk_w"]))
+    want = oracle_mod.combine(eo, d["topk_w"], ref["slot"])
+    nan = lambda b: (b & 0x7FFF) > 0x7F80
+    assert np.array_equal(nan(y), nan(want)) and nan(want).any()
+    assert np.array_equal(y[~nan(want)], want[~nan(want)])
+    assert ((want & 0x7FFF) == 0x7F80).any(), "an infinity reaches the output"
+
+
 def test_empty_batch(oracle_mod):
     cfg = M.cfg_of(0, 64, 8, 2, 2, 2, TWO)
     lay, _ = M.gpu_layout(cfg, np.zeros((0, 2), np.int32))
