@@ -95,7 +95,8 @@ def test_pins_catch_mutant(name, tmp_path):
            os.path.join(ROOT, "tests", "test_oracle_layout.py"),
            os.path.join(ROOT, "tests", "test_oracle_dispatch_combine.py"),
            os.path.join(ROOT, "tests", "test_oracle_fp8.py"),
-           os.path.join(ROOT, "tests", "test_oracle_ep.py")]
+           os.path.join(ROOT, "tests", "test_oracle_ep.py"),
+           os.path.join(ROOT, "tests", "test_oracle_properties.py")]
     res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert res.returncode == 1, (
         f"mutant {name} passed every pin:\n{res.stdout[-2000:]}\n{res.stderr[-2000:]}")
