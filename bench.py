@@ -764,33 +764,41 @@ def main():
     s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev = lambda: torch.cuda.Event()
     inputs_up, computed, result_down = [ev() for _ in sets], [ev() for _ in sets], [ev() for _ in sets]
-    torch.cuda.synchronize()
-    barrier()
-    t0 = time.perf_counter()
-    for i in range(e2e_steps):
-        j = i % 2
-        b = sets[j]
-        if i >= 2:
-            s_in.wait_event(computed[j])        # step i-2 has read this set's inputs
-        with torch.cuda.stream(s_in):
-            b.x.copy_(x_h, non_blocking=True)
-            b.topk.copy_(topk_h, non_blocking=True)
-            b.w.copy_(w_h, non_blocking=True)
-            inputs_up[j].record(s_in)
-        s_comp.wait_event(inputs_up[j])
-        if i >= 2:
-            s_comp.wait_event(result_down[j])   # step i-2's result has left this set's y
-        with torch.cuda.stream(s_comp):
-            capi.moe_layout_dispatch(cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
-            capi.moe_combine(cfg, b.lay.struct, b.recv, b.w, b.y)   # identity expert
-            computed[j].record(s_comp)
-        s_out.wait_event(computed[j])
-        with torch.cuda.stream(s_out):
-            y_h[j].copy_(b.y, non_blocking=True)
-            result_down[j].record(s_out)
-    for s_ in (s_in, s_comp, s_out):
-        s_.synchronize()
-    e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
+
+    def e2e_run(compute: bool) -> float:
+        """Wall seconds for e2e_steps pipelined steps (max over ranks);
+        compute=False moves the same bytes with no kernels (the copy bound)."""
+        torch.cuda.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        for i in range(e2e_steps):
+            j = i % 2
+            b = sets[j]
+            if i >= 2:
+                s_in.wait_event(computed[j])        # step i-2 has read this set's inputs
+            with torch.cuda.stream(s_in):
+                b.x.copy_(x_h, non_blocking=True)
+                b.topk.copy_(topk_h, non_blocking=True)
+                b.w.copy_(w_h, non_blocking=True)
+                inputs_up[j].record(s_in)
+            s_comp.wait_event(inputs_up[j])
+            if i >= 2:
+                s_comp.wait_event(result_down[j])   # step i-2's result has left this set's y
+            with torch.cuda.stream(s_comp):
+                if compute:
+                    capi.moe_layout_dispatch(cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
+                    capi.moe_combine(cfg, b.lay.struct, b.recv, b.w, b.y)   # identity expert
+                computed[j].record(s_comp)
+            s_out.wait_event(computed[j])
+            with torch.cuda.stream(s_out):
+                y_h[j].copy_(b.y, non_blocking=True)
+                result_down[j].record(s_out)
+        for s_ in (s_in, s_comp, s_out):
+            s_.synchronize()
+        return max_over_ranks(time.perf_counter() - t0, world, dev)
+
+    copies_s = e2e_run(False)
+    e2e_s = e2e_run(True)
     e2e_value = job_gbs(step_bytes, world, e2e_steps, e2e_s)
 
     cpu = None
@@ -841,6 +849,7 @@ def main():
             "clocks": clocks.summary(),
             "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "copies_only_value": round(job_gbs(step_bytes, world, e2e_steps, copies_s), 3),
                     "mode": "moe_layout_dispatch + moe_combine per step, host copies pipelined "
                             "on two copy streams over two buffer sets (wall clock)"},
             "gpu_launches": launches_per_step * K,
