@@ -63,6 +63,7 @@ def measured_peak():
 KERNEL_SOURCES = {
     "combine": ["combine.cu", "moe_common.cuh"],
     "dispatch": ["bulk.cu", "dispatch.cu", "moe_common.cuh"],
+    "layout_dispatch": ["fused.cu", "layout_common.cuh", "moe_common.cuh"],
 }
 
 
@@ -371,7 +372,9 @@ def main():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="olmoe", choices=sorted(inputs.WORKLOADS))
     p.add_argument("--engine", default="auto", choices=["auto", "vector", "bulk"])
-    p.add_argument("--layout", default="kernels", choices=["kernels", "cluster"])
+    p.add_argument("--layout", default="kernels", choices=["kernels", "fused", "cluster"],
+                   help="kernels: layout kernels then the dispatch kernel; fused: a count kernel "
+                        "then an assign/dispatch kernel (flat); cluster: one-cluster layout")
     p.add_argument("--unfused", action="store_true",
                    help="moe_layout + moe_dispatch instead of moe_layout_dispatch")
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")
@@ -420,6 +423,8 @@ def main():
     flags |= {"auto": 0, "vector": capi.MOE_FLAG_COPY_VECTOR, "bulk": capi.MOE_FLAG_COPY_BULK}[args.engine]
     if args.layout == "cluster":
         flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
+    if args.layout == "fused":
+        flags |= capi.MOE_FLAG_LAYOUT_FUSED
     cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
     # the decoupled comparison path packs per rank: one "node" per rank
     dcfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R,
@@ -576,7 +581,12 @@ def main():
     cluster_layout = args.layout == "cluster" and wl.T <= 131072
     small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
     layout_launches = 1 if cluster_layout else (2 if small_layout else 3)
-    launches_per_step = layout_launches + (2 if wl.two_level else 1) + 1
+    # moe_layout_dispatch as the count + assign/dispatch pair (the library's
+    # rule: flat, 16-byte rows, at most 256 experts, no engine or layout
+    # override)
+    ld_pair = (not args.unfused and not wl.two_level and args.layout == "fused"
+               and (wl.H * 2) % 16 == 0 and wl.E <= 256)
+    launches_per_step = (2 if ld_pair else layout_launches + (2 if wl.two_level else 1)) + 1
 
     for i in range(args.warmup):
         step(sets[i % 2])
@@ -680,7 +690,14 @@ def main():
         ep_ms = timed("ep", K) if with_ep else None
         flushed = flushed_steps(K)
     ms_per_step = total_ms / K
-    t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
+    # Stage costs by subtraction.  With the count + assign/dispatch pair the
+    # assignment runs inside the dispatch kernel: the pair's whole cost
+    # counts as dispatch (the layout alone, moe_layout's kernels, is reported
+    # beside it).
+    if ld_pair:
+        t_layout, t_dispatch, t_combine = 0.0, t_ld, ms_per_step - t_ld
+    else:
+        t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
     for b in sets:
         st = capi.moe_get_error(b.lay.struct)
         if st != capi.MOE_OK:
@@ -691,6 +708,7 @@ def main():
     value = job_gbs(step_bytes, world, K, total_ms * 1e-3)
     peak, peak_src = measured_peak()
     dom = "dispatch" if t_dispatch >= t_combine else "combine"
+    dom_kernel = "layout_dispatch" if dom == "dispatch" and ld_pair else dom
     dom_bytes = disp_b if dom == "dispatch" else comb_b
     dom_ms = t_dispatch if dom == "dispatch" else t_combine
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
@@ -718,7 +736,7 @@ def main():
                "ms_per_step": round(fp8_ms / K, 5),
                "tokens_per_s": round(wl.T * world * K / (fp8_ms * 1e-3), 1),
                "speedup_vs_bf16_step": round(total_ms / fp8_ms, 3),
-               "kernels_ms": {"dispatch": round(fp8_ld - t_l, 5),
+               "kernels_ms": {"dispatch": round(fp8_ld - t_l, 5),  # fp8 path: layout kernels + dispatch
                               "combine": round(fp8_ms / K - fp8_ld, 5)},
                "bytes_per_step": fp8_bytes,
                "path": ("layout + fp8 two-level dispatch (quantize once into node staging, "
@@ -822,8 +840,10 @@ def main():
                                "buffer sets, each step moves %.0f MB (%.1fx L2)"
                                % (step_bytes / 1e6, step_bytes / torch.cuda.get_device_properties(dev).L2_cache_size)),
                            engine=args.engine,
-                           layout="one cluster launch" if cluster_layout else
-                           ("count + assign kernels" if small_layout else "count/scan/assign kernels"),
+                           layout=("count kernel + assign/dispatch kernel" if ld_pair
+                                   else "one cluster launch" if cluster_layout else
+                                   ("count + assign kernels" if small_layout
+                                    else "count/scan/assign kernels")),
                            entry="moe_layout + moe_dispatch" if args.unfused else "moe_layout_dispatch",
                            timing="K steps back to back (CUDA graphs of two steps) between two CUDA "
                                   "events on the launching stream; stage costs from graphs of "
@@ -835,11 +855,13 @@ def main():
             "tokens_per_s_dispatch_combine": round(wl.T * world / ((t_dispatch + t_combine) * 1e-3), 1),
             "flushed_step": flushed,
             "dispatch_combine_only_gbs": round(step_bytes / ((t_dispatch + t_combine) * 1e-3) / 1e9, 2),
-            "kernels_ms": {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
-                           "combine": round(t_combine, 5)},
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2),
+            "kernels_ms": ({"layout_dispatch": round(t_dispatch, 5), "combine": round(t_combine, 5),
+                            "layout_kernels_alone": round(t_l, 5)} if ld_pair else
+                           {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
+                            "combine": round(t_combine, 5)}),
+            "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": profiled_traffic(dom, wl.name),
+                         "traffic": profiled_traffic(dom_kernel, wl.name),
                          "peak_kind": f"{peak_src} copy bandwidth"},
             "decoupled_3pass": decoupled,
             "allgather_reducescatter": agrs,

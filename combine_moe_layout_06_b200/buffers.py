@@ -26,7 +26,9 @@ class DeviceLayout:
         self.slot = torch.zeros(T * k, **i32)
         self.error_word = torch.zeros(1, **i32)
         ws = capi.moe_layout_workspace_bytes(cfg)
-        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        # zeroed once: a counter of moe_layout_dispatch's kernels lives in it
+        # and must start at zero
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
         self.two_level = bool(cfg.flags & capi.MOE_FLAG_TWO_LEVEL)
         if self.two_level:
             self.node_counts = torch.zeros(N, **i32)

@@ -25,6 +25,7 @@ MOE_FLAG_TWO_LEVEL = 0x1
 MOE_FLAG_COPY_VECTOR = 0x2
 MOE_FLAG_COPY_BULK = 0x4
 MOE_FLAG_LAYOUT_CLUSTER = 0x8
+MOE_FLAG_LAYOUT_FUSED = 0x10
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1

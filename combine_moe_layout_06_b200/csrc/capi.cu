@@ -8,8 +8,8 @@ namespace {
 
 using moe::CopyEngine;
 
-constexpr uint32_t kKnownFlags =
-    MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK | MOE_FLAG_LAYOUT_CLUSTER;
+constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK |
+                                 MOE_FLAG_LAYOUT_CLUSTER | MOE_FLAG_LAYOUT_FUSED;
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -79,6 +79,30 @@ moe_status_t dispatch_impl(const moe_config_t* c, const moe_layout_t* L, const v
     p.early_inputs = false;  // expansion reads staging written by the pack
     if (e == cudaSuccess) e = moe::launch_node_expand(p, node_staging, rows, recv, s);
     return cuda_status(e);
+}
+
+moe::LayoutParams layout_params(const moe_config_t* c, const int32_t* topk_idx,
+                                const moe_layout_t* L) {
+    moe::LayoutParams p;
+    p.T = c->num_tokens;
+    p.k = c->top_k;
+    p.E = c->num_experts;
+    p.R = c->num_ranks;
+    p.N = c->num_nodes;
+    p.nodes = two_level(c);
+    p.cluster = (c->flags & MOE_FLAG_LAYOUT_CLUSTER) != 0;
+    p.topk = topk_idx;
+    p.expert_counts = L->expert_counts;
+    p.expert_offsets = L->expert_offsets;
+    p.rank_offsets = L->rank_offsets;
+    p.slot = L->slot;
+    p.node_counts = L->node_counts;
+    p.node_offsets = L->node_offsets;
+    p.node_slot = L->node_slot;
+    p.node_src = L->node_src;
+    p.err = L->error_word;
+    p.workspace = L->workspace;
+    return p;
 }
 
 }  // namespace
@@ -153,25 +177,7 @@ moe_status_t moe_layout(const moe_config_t* c, const int32_t* topk_idx, const mo
     if (st != MOE_OK) return st;
     if (L->workspace == nullptr || (c->num_tokens > 0 && topk_idx == nullptr))
         return MOE_ERR_INVALID_ARG;
-    moe::LayoutParams p;
-    p.T = c->num_tokens;
-    p.k = c->top_k;
-    p.E = c->num_experts;
-    p.R = c->num_ranks;
-    p.N = c->num_nodes;
-    p.nodes = two_level(c);
-    p.cluster = (c->flags & MOE_FLAG_LAYOUT_CLUSTER) != 0;
-    p.topk = topk_idx;
-    p.expert_counts = L->expert_counts;
-    p.expert_offsets = L->expert_offsets;
-    p.rank_offsets = L->rank_offsets;
-    p.slot = L->slot;
-    p.node_counts = L->node_counts;
-    p.node_offsets = L->node_offsets;
-    p.node_slot = L->node_slot;
-    p.node_src = L->node_src;
-    p.err = L->error_word;
-    p.workspace = L->workspace;
+    const moe::LayoutParams p = layout_params(c, topk_idx, L);
     return cuda_status(moe::launch_layout(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -187,6 +193,16 @@ moe_status_t moe_layout_dispatch(const moe_config_t* c, const int32_t* topk_idx,
                                  void* node_staging, void* stream) {
     moe_status_t st = check_dispatch_args(c, L, x, recv, node_staging);
     if (st != MOE_OK) return st;
+    const size_t row_bytes = (size_t)c->hidden * 2;
+    const bool pair =
+        (c->flags & MOE_FLAG_LAYOUT_FUSED) != 0 && !two_level(c) && c->num_tokens > 0 &&
+        L->workspace != nullptr && topk_idx != nullptr &&
+        moe::bulk_eligible(row_bytes, {x, recv, L->workspace}) &&
+        moe::layout_dispatch_fused_eligible(c->num_tokens, c->top_k, c->num_experts, row_bytes);
+    if (pair)
+        return cuda_status(moe::launch_layout_dispatch_fused(layout_params(c, topk_idx, L), x, recv,
+                                                             row_bytes,
+                                                             static_cast<cudaStream_t>(stream)));
     st = moe_layout(c, topk_idx, L, stream);
     if (st != MOE_OK || c->num_tokens == 0) return st;
     return dispatch_impl(c, L, x, recv, node_staging, static_cast<cudaStream_t>(stream), true);

@@ -43,6 +43,7 @@
 //            names an expert twice, this ordering is by token index.
 #include <cooperative_groups.h>
 
+#include "layout_common.cuh"
 #include "moe_kernels.h"
 
 namespace moe {
@@ -73,55 +74,6 @@ struct LayoutArgs {
     int* node_src;  // [U] staging row -> token, or nullptr
     int* err;
 };
-
-// Load token t's k expert ids.  Invalid entries become -1 and set error
-// bits: an id outside [0, E), or a repeat of an id earlier in the row (the
-// later copy is dropped).  Count and assign use the same rule, so the
-// histogram and the ranks always agree even on bad input.  Repeats are found
-// with a 64-bit mask of ids seen so far (id mod 64); only when the mask hits
-// are the earlier raw entries re-read (from cache) to confirm, which is exact
-// because a valid id equal to an earlier raw id is a repeat.
-template <int KMAX>
-__device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t t, int k, int E,
-                                          int (&e)[KMAX]) {
-    int bits = 0;
-    const int* row = topk + t * k;
-    uint64_t seen = 0;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        int v = -1;
-        if (j < k) {
-            v = ld_dep(row + j);
-            if (v < 0 || v >= E) {
-                bits |= kErrExpertOob;
-                v = -1;
-            } else {
-                const uint64_t bit = 1ull << (v & 63);
-                if (seen & bit) {
-                    bool repeat = false;
-#pragma unroll 1
-                    for (int i = 0; i < j; ++i) repeat |= ld_dep(row + i) == v;
-                    if (repeat) {
-                        bits |= kErrDupExpert;
-                        v = -1;
-                    }
-                }
-                seen |= bit;
-            }
-        }
-        e[j] = v;
-    }
-    return bits;
-}
-
-template <int KMAX>
-__device__ __forceinline__ uint32_t node_mask(const Partition& part, const int (&e)[KMAX]) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j)
-        if (e[j] >= 0) m |= 1u << part.node_of(e[j]);
-    return m;
-}
 
 template <int KMAX>
 __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs a) {
@@ -157,36 +109,6 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs 
     if (a.nodes)
         for (int i = threadIdx.x; i < a.N; i += blockDim.x)
             a.ncnt[(int64_t)i * a.C + blockIdx.x] = s_ncnt[i];
-}
-
-// Exclusive scan of one value per thread over the whole block; also returns
-// the block total.  s_warp holds 32 ints.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& total) {
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFullMask, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nwarps ? s_warp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFullMask, w, o);
-            if (lane >= o) w += y;
-        }
-        s_warp[lane] = w;
-    }
-    __syncthreads();
-    const int before = warp > 0 ? s_warp[warp - 1] : 0;
-    total = s_warp[nwarps - 1];
-    __syncthreads();
-    return before + x - v;
 }
 
 // In-place exclusive scan of data[0..L) by one block: each thread owns a
@@ -331,25 +253,6 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs
             }
         }
     }
-}
-
-// In-place exclusive scan of an int array in shared memory (length L) by
-// one block; returns the total.  s_warp holds 32 ints.
-__device__ int smem_exclusive_scan(int* data, int L, int* s_warp) {
-    const int span = (L + blockDim.x - 1) / blockDim.x;
-    const int beg = min(L, (int)threadIdx.x * span);
-    const int end = min(L, beg + span);
-    int sum = 0;
-    for (int i = beg; i < end; ++i) sum += data[i];
-    int total = 0;
-    int run = block_exclusive_scan(sum, s_warp, total);
-    for (int i = beg; i < end; ++i) {
-        const int v = data[i];
-        data[i] = run;
-        run += v;
-    }
-    __syncthreads();
-    return total;
 }
 
 // Assign with the scan folded in (up to kFusedScanMaxChunks chunks): each CTA
@@ -553,16 +456,6 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
 // (ints): hist[E+N] | tot[E+N] | base[E+N] | wbase[W][ES] wmask[W][ES] wn[W][N],
 // W = blockDim.x / 32, ES = E rounded to an odd stride (conflict-free columns).
 constexpr int kMaxCluster = 16;
-
-__device__ __forceinline__ int warp_inclusive_scan(int v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFullMask, v, o);
-        if (lane >= o) v += y;
-    }
-    return v;
-}
 
 template <int KMAX>
 __global__ void __launch_bounds__(1024) layout_cluster_kernel(LayoutArgs a, int64_t tokens_per_cta) {
@@ -847,10 +740,18 @@ cudaError_t launch_layout_cluster(const LayoutArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+size_t fused_workspace_offset(int64_t T, int E) {
+    const int64_t C = (T + kTokensPerCta - 1) / kTokensPerCta;
+    return round_up(sizeof(int) * (size_t)E * (size_t)C, 256);
+}
+
 size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes) {
     const int64_t C = (T + kTokensPerCta - 1) / kTokensPerCta;
     size_t b = round_up(sizeof(int) * (size_t)E * (size_t)C, 256);
-    if (nodes) b += round_up(sizeof(int) * (size_t)N * (size_t)C, 256);
+    if (nodes)
+        b += round_up(sizeof(int) * (size_t)N * (size_t)C, 256);
+    else
+        b += kFusedBarrierBytes + round_up(sizeof(int) * (size_t)E * kFusedMaxCtas, 256);
     return b < 256 ? 256 : b;
 }
 

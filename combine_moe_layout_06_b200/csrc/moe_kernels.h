@@ -33,8 +33,28 @@ struct LayoutParams {
     int* err;               // [1]
     void* workspace;        // layout_workspace_bytes()
 };
+// Workspace bytes: the layout kernels' chunk histograms and, for flat
+// layouts (no node maps), the region of the count + assign/dispatch pair
+// (fused.cu) after them: kFusedBarrierBytes holding a ticket counter, which
+// must be zero before the first launch and is left zero by every launch,
+// then an [E][kFusedMaxCtas] histogram matrix.
 size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes);
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
+
+// ---- layout and flat dispatch, assignment folded into the dispatch (fused.cu)
+constexpr int kFusedMaxCtas = 256;      // columns of the histogram matrix
+constexpr int kFusedMaxExperts = 256;   // shared-memory lane masks per expert
+constexpr int kFusedMaxTopk = 32;
+constexpr size_t kFusedBarrierBytes = 256;
+// Byte offset of the fused region inside the workspace (flat layouts).
+size_t fused_workspace_offset(int64_t T, int E);
+// Whether the count + assign/dispatch pair takes this problem (16-byte
+// aligned rows are checked by the caller).
+bool layout_dispatch_fused_eligible(int64_t T, int k, int E, size_t row_bytes);
+// moe_layout() (flat) + moe_dispatch() as the count + assign/dispatch pair;
+// lp.nodes must be false and lp.workspace must hold layout_workspace_bytes().
+cudaError_t launch_layout_dispatch_fused(const LayoutParams& lp, const void* x, void* recv,
+                                         size_t row_bytes, cudaStream_t stream);
 
 // ---- row movement ------------------------------------------------------------
 // Geometry shared by the dispatch-side kernels.  Row sizes are in bytes;

@@ -70,6 +70,10 @@ extern "C" {
 #define MOE_FLAG_LAYOUT_CLUSTER 0x8u /* layout in one thread-block-cluster
                                         launch (up to 131072 tokens) instead
                                         of the count/scan/assign kernels */
+#define MOE_FLAG_LAYOUT_FUSED 0x10u  /* moe_layout_dispatch(): a count kernel
+                                        and an assign/dispatch kernel instead
+                                        of the layout kernels and the
+                                        dispatch kernel (flat layouts) */
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -119,8 +123,14 @@ typedef struct moe_config {
  *                          or -1 when t touches no expert of n (TWO_LEVEL)
  *   error_word     [1]     device error bits; zero it once before first use,
  *                          moe_get_error() reads and clears it
- *   workspace      moe_layout_workspace_bytes() bytes, 16-byte aligned,
- *                          scratch for moe_layout only
+ *   workspace      moe_layout_workspace_bytes() bytes, 16-byte aligned.
+ *                          Scratch for moe_layout; without
+ *                          MOE_FLAG_TWO_LEVEL it also holds a counter used by
+ *                          moe_layout_dispatch with MOE_FLAG_LAYOUT_FUSED, so
+ *                          zero the whole workspace once before its first
+ *                          use (every call leaves the counter zero; calls
+ *                          that share a workspace must not overlap on the
+ *                          GPU)
  *   node_src       [moe_node_staging_rows()]  token held by each staging row:
  *                          node_src[node_offsets[n] + node_slot[t][n]] = t
  *                          (TWO_LEVEL, optional).  When it is given,
@@ -197,11 +207,21 @@ moe_status_t moe_dispatch(const moe_config_t *cfg, const moe_layout_t *layout,
 /* Layout and dispatch in one call, the layout transformation fused with
  * the data movement (FUSCO article, "FUSCO 的核心创新": the transfer itself
  * carries where each row comes from and goes to).  Same results as
- * moe_layout() followed by moe_dispatch() with the same arguments, but the
- * dispatch kernel starts loading x rows while the layout kernels still run
- * (bulk-copy engine), because x and topk_idx are known to be complete when
- * the layout starts.  Arguments as for moe_layout() and moe_dispatch(); all
- * are checked before anything is enqueued. */
+ * moe_layout() followed by moe_dispatch() with the same arguments.
+ *  - By default the layout kernels run first and the dispatch kernel starts
+ *    loading x rows while they still run (bulk-copy engine), because x and
+ *    topk_idx are complete when the layout starts.
+ *  - With MOE_FLAG_LAYOUT_FUSED, without MOE_FLAG_TWO_LEVEL, with 16-byte
+ *    aligned x, recv and workspace, H*2 a multiple of 16 and E <= 256, it is
+ *    two kernels over the same split of the tokens (one CTA per SM): a count
+ *    kernel whose last CTA turns the per-CTA histograms into prefixes and
+ *    offsets, and an assign/dispatch kernel that loads its x rows and routes
+ *    while the count kernel runs, then ranks its tokens and stores each row
+ *    straight to its receive rows.  A ticket counter lives in the workspace
+ *    (zero it once before first use).  Other configurations with this flag
+ *    take the default path.
+ * Arguments as for moe_layout() and moe_dispatch(); all are checked before
+ * anything is enqueued. */
 moe_status_t moe_layout_dispatch(const moe_config_t *cfg, const int32_t *topk_idx,
                                  const moe_layout_t *layout, const void *x, void *recv,
                                  void *node_staging, void *stream);
