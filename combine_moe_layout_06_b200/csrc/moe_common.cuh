@@ -336,14 +336,28 @@ inline int blocks_per_sm(int threads, size_t smem = 0) {
     return cached;
 }
 
-// Grid for a persistent warp-strided loop over `warp_items` items: enough
-// blocks to give every warp an item, capped at what is resident at once.
+// Grid for a warp-strided loop over `warp_items` items.  Small problems get
+// a persistent grid (each warp one contiguous range of items).  When a
+// resident grid would give each warp more than 2 * kItemsPerWarp items, the
+// grid becomes a whole number of resident waves (up to 16) of about
+// kItemsPerWarp items per warp: the block scheduler hands out the later
+// waves as earlier blocks finish, so the kernel ends with every SM busy
+// instead of a tail of slow warps, and no wave is left partly empty.
+#ifndef MOE_ITEMS_PER_WARP
+#define MOE_ITEMS_PER_WARP 4
+#endif
+constexpr int64_t kItemsPerWarp = MOE_ITEMS_PER_WARP;
 template <auto Kernel>
 inline int persistent_grid(int64_t warp_items, int threads, size_t smem = 0) {
     const int64_t warps_per_block = threads / 32;
     const int64_t resident = (int64_t)device_sm_count() * blocks_per_sm<Kernel>(threads, smem);
-    int64_t g = (warp_items + warps_per_block - 1) / warps_per_block;
-    if (g > resident) g = resident;
+    int64_t g = (warp_items + warps_per_block - 1) / warps_per_block;   // one item per warp
+    if (g > resident) {
+        int64_t waves = warp_items / (resident * warps_per_block * kItemsPerWarp);
+        if (waves < 1) waves = 1;
+        if (waves > 16) waves = 16;
+        g = waves * resident;
+    }
     return (int)(g < 1 ? 1 : g);
 }
 
