@@ -45,7 +45,10 @@ namespace {
 #ifndef MOE_BULK_COMB_STAGE_BYTES
 #define MOE_BULK_COMB_STAGE_BYTES 4096
 #endif
-constexpr int kBulkWarps = 4;
+#ifndef MOE_BULK_WARPS
+#define MOE_BULK_WARPS 4
+#endif
+constexpr int kBulkWarps = MOE_BULK_WARPS;
 constexpr int kBulkThreads = kBulkWarps * 32;
 constexpr int kDispStages = MOE_BULK_DISP_STAGES;
 constexpr uint32_t kDispChunk = MOE_BULK_DISP_CHUNK;
