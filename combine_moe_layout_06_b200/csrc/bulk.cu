@@ -34,10 +34,10 @@ namespace {
 
 // Pipeline shape (compile-time tunables).
 #ifndef MOE_BULK_DISP_STAGES
-#define MOE_BULK_DISP_STAGES 4
+#define MOE_BULK_DISP_STAGES 8
 #endif
 #ifndef MOE_BULK_DISP_CHUNK
-#define MOE_BULK_DISP_CHUNK 4096
+#define MOE_BULK_DISP_CHUNK 2048
 #endif
 #ifndef MOE_BULK_COMB_STAGES
 #define MOE_BULK_COMB_STAGES 3
