@@ -34,6 +34,10 @@ constexpr int kThreads = kWarpsPerCta * 32;
 #ifndef MOE_COMBINE_KB
 #define MOE_COMBINE_KB 8
 #endif
+// items per warp in each wave of a large combine (see persistent_grid)
+#ifndef MOE_COMBINE_IPW
+#define MOE_COMBINE_IPW 4
+#endif
 
 struct CombArgs {
     const void* eo;
@@ -183,7 +187,7 @@ template <typename V, int VPL, int KB, bool EP>
 cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
     constexpr auto kern = combine_kernel<V, VPL, KB, EP>;
     const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
-    const int grid = persistent_grid<kern>(a.T * cpr, kThreads);
+    const int grid = persistent_grid<kern>(a.T * cpr, kThreads, 0, MOE_COMBINE_IPW);
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
 }
 

@@ -338,9 +338,9 @@ inline int blocks_per_sm(int threads, size_t smem = 0) {
 
 // Grid for a warp-strided loop over `warp_items` items.  Small problems get
 // a persistent grid (each warp one contiguous range of items).  When a
-// resident grid would give each warp more than 2 * kItemsPerWarp items, the
+// resident grid would give each warp at least 2 * items_per_warp items, the
 // grid becomes a whole number of resident waves (up to 16) of about
-// kItemsPerWarp items per warp: the block scheduler hands out the later
+// items_per_warp items per warp: the block scheduler hands out the later
 // waves as earlier blocks finish, so the kernel ends with every SM busy
 // instead of a tail of slow warps, and no wave is left partly empty.
 #ifndef MOE_ITEMS_PER_WARP
@@ -348,12 +348,13 @@ inline int blocks_per_sm(int threads, size_t smem = 0) {
 #endif
 constexpr int64_t kItemsPerWarp = MOE_ITEMS_PER_WARP;
 template <auto Kernel>
-inline int persistent_grid(int64_t warp_items, int threads, size_t smem = 0) {
+inline int persistent_grid(int64_t warp_items, int threads, size_t smem = 0,
+                           int64_t items_per_warp = kItemsPerWarp) {
     const int64_t warps_per_block = threads / 32;
     const int64_t resident = (int64_t)device_sm_count() * blocks_per_sm<Kernel>(threads, smem);
     int64_t g = (warp_items + warps_per_block - 1) / warps_per_block;   // one item per warp
     if (g > resident) {
-        int64_t waves = warp_items / (resident * warps_per_block * kItemsPerWarp);
+        int64_t waves = warp_items / (resident * warps_per_block * items_per_warp);
         if (waves < 1) waves = 1;
         if (waves > 16) waves = 16;
         g = waves * resident;
