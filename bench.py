@@ -375,6 +375,8 @@ def main():
     p.add_argument("--layout", default="kernels", choices=["kernels", "fused", "cluster"],
                    help="kernels: layout kernels then the dispatch kernel; fused: a count kernel "
                         "then an assign/dispatch kernel (flat); cluster: one-cluster layout")
+    p.add_argument("--two-level-fused", action="store_true",
+                   help="two-level dispatch in one kernel (staging rows read back from L2)")
     p.add_argument("--unfused", action="store_true",
                    help="moe_layout + moe_dispatch instead of moe_layout_dispatch")
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")
@@ -425,6 +427,8 @@ def main():
         flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
     if args.layout == "fused":
         flags |= capi.MOE_FLAG_LAYOUT_FUSED
+    if args.two_level_fused:
+        flags |= capi.MOE_FLAG_TWO_LEVEL_FUSED
     cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
     # the decoupled comparison path packs per rank: one "node" per rank
     dcfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R,
@@ -586,7 +590,10 @@ def main():
     # override)
     ld_pair = (not args.unfused and not wl.two_level and args.layout == "fused"
                and (wl.H * 2) % 16 == 0 and wl.E <= 256)
-    launches_per_step = (2 if ld_pair else layout_launches + (2 if wl.two_level else 1)) + 1
+    # two-level: pack + expand, or one kernel with --two-level-fused (16-byte rows, N + k <= 32)
+    two_kernels = wl.two_level and (not args.two_level_fused or args.engine == "vector"
+                                    or (wl.H * 2) % 16 or wl.N + wl.k > 32)
+    launches_per_step = (2 if ld_pair else layout_launches + (2 if two_kernels else 1)) + 1
 
     for i in range(args.warmup):
         step(sets[i % 2])

@@ -74,6 +74,8 @@ struct BulkArgs {
     int64_t src_rows, dst_rows;
     int* err;
     int early;                // start source loads before waiting (see RowMoveParams)
+    char* staging = nullptr;  // node_dispatch_kernel: node staging rows
+    int64_t staging_rows = 0;
 };
 
 // Drain after a timeout: wait (bounded) for every stage this warp still
@@ -223,6 +225,173 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
             issue(q - 1 + kDispStages);
             inflight |= 1u << ((q - 1) % kDispStages);
         }
+    }
+    bulk_wait_all();
+    warp_report(a.err, errbits);
+}
+
+// Two-level dispatch in one kernel (FUSCO article, section "负载均衡与跨节点
+// 去重": a token crosses to a node once, into that node's forwarding region,
+// and is fanned out to the node's experts from there).  Per (token, chunk)
+// item a warp
+//   1. loads the x chunk into shared memory (double-buffered: the next
+//      item's chunk is loaded while this one is handled),
+//   2. stores it to the token's staging row of every node it touches (lane
+//      31 - n for node n),
+//   3. once those stores are complete, reads each node's staging row back
+//      into shared memory and stores it to the token's receive rows on that
+//      node (lane j < k for column j).
+// Step 3 reads the staging rows right after they were written, so the reads
+// are served by L2 instead of a second pass over HBM.  The staging buffer and
+// the receive rows end up exactly as with the two-kernel form (pack, then
+// expansion).  Needs N + k <= 32.  Opt-in (MOE_FLAG_TWO_LEVEL_FUSED): it
+// moves fewer bytes, but nearly all of them are writes, and measured right
+// before a combine the step is slower than with the two-kernel form, whose
+// expansion mixes the staging reads into its writes.  Waits are bounded; a wait that gives up
+// records kErrTimeout, drains what this warp started and stops.
+constexpr int kNfWarps = 8;
+constexpr int kNfThreads = kNfWarps * 32;
+
+
+__global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char* xbuf = smem + (size_t)warp * 3 * a.chunk;  // X[0], X[1]
+    unsigned char* rbuf = xbuf + 2 * (size_t)a.chunk;         // R
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kNfWarps * 3 * a.chunk) + warp * 3;
+    if (lane == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    const bool early = a.early != 0;
+    pdl_trigger();
+    if (!early) pdl_wait();
+
+    const int64_t items = a.T * a.cpr;
+    const int64_t nwarps = (int64_t)gridDim.x * kNfWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kNfWarps + warp;
+    const int64_t first = items * gw / nwarps;
+    const int64_t mine = items * (gw + 1) / nwarps - first;
+    auto geometry = [&](int64_t q, int64_t& t, int64_t& off, uint32_t& bytes) {
+        const int64_t it = first + q;
+        t = it / a.cpr;
+        off = (it - t * a.cpr) * (int64_t)a.chunk;
+        const int64_t left = a.row_bytes - off;
+        bytes = left < (int64_t)a.chunk ? (uint32_t)left : a.chunk;
+    };
+    auto issue_x = [&](int64_t q, int b) {
+        int64_t t, off;
+        uint32_t bytes;
+        geometry(q, t, off, bytes);
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bar[b], bytes);
+            bulk_load(xbuf + (size_t)b * a.chunk, a.src + t * a.row_bytes + off, bytes, &bar[b]);
+        }
+    };
+    uint32_t parity = 0, inflight = 0;  // bits 0, 1: X buffers; bit 2: R
+    if (mine > 0) {
+        issue_x(0, 0);
+        inflight |= 1u;
+    }
+    if (early) pdl_wait();
+
+    // node n: lane n holds its receive-row range [lo, hi); lane 31 - n its
+    // first staging row
+    const int N = a.N;
+    int n_lo = INT_MAX, n_hi = INT_MIN, n_first = 0;
+    if (lane < N) {
+        n_lo = ld_dep(a.rank_offsets + lane * a.ranks_per_node);
+        n_hi = ld_dep(a.rank_offsets + (lane + 1) * a.ranks_per_node);
+    }
+    const bool stager = lane >= 32 - N;
+    const int my_node = 31 - lane;
+    if (stager) n_first = ld_dep(a.node_offsets + my_node);
+
+    int errbits = 0;
+    int64_t t_cur = -1;
+    int sl = -1, nj = -1;
+    int64_t srow = -1;
+    bool failed = false;
+    for (int64_t q = 0; q < mine && !failed; ++q) {
+        const int b = (int)(q & 1);
+        int64_t t, off;
+        uint32_t bytes;
+        geometry(q, t, off, bytes);
+        if (t != t_cur) {
+            // column j's receive row and its node; node n's staging row
+            sl = -1;
+            nj = -1;
+            srow = -1;
+            if (lane < a.k) {
+                const int s = ld_dep(a.slot + t * a.k + lane);
+                if (s >= 0 && s < a.dst_rows) sl = s;
+                else if (s != -1) errbits |= kErrBadLayout;
+            }
+            for (int n = 0; n < N; ++n) {
+                const int lo = __shfl_sync(kFullMask, n_lo, n);
+                const int hi = __shfl_sync(kFullMask, n_hi, n);
+                if (sl >= lo && sl < hi) nj = n;
+            }
+            if (sl >= 0 && nj < 0) errbits |= kErrBadLayout;
+            if (stager) {
+                const int ns = ld_dep(a.node_slot + t * N + my_node);
+                if (ns >= 0) {
+                    const int64_t r = (int64_t)n_first + ns;
+                    if (r >= 0 && r < a.staging_rows) srow = r;
+                    else errbits |= kErrBadLayout;
+                }
+            }
+            t_cur = t;
+        }
+        if (!__all_sync(kFullMask, mbar_wait(&bar[b], (parity >> b) & 1u))) {
+            failed = true;
+            break;
+        }
+        parity ^= 1u << b;
+        inflight &= ~(1u << b);
+        // 2. one staging row per node touched
+        if (srow >= 0) bulk_store(a.staging + srow * a.row_bytes + off, xbuf + (size_t)b * a.chunk, bytes);
+        bulk_commit();
+        // the other X buffer was last read by the previous item's staging
+        // stores: free once all but the newest group have been read
+        bulk_wait_read<1>();
+        __syncwarp();
+        if (q + 1 < mine) {
+            issue_x(q + 1, b ^ 1);
+            inflight |= 1u << (b ^ 1);
+        }
+        // 3. the staging rows are complete before they are read back
+        if (stager) bulk_wait_all();
+        __syncwarp();
+        unsigned touched = __ballot_sync(kFullMask, srow >= 0);  // bit 31 - n: node n
+        while (touched) {
+            const int hb = 31 - __clz(touched);  // highest set bit: lowest node first
+            touched &= ~(1u << hb);
+            const int n = 31 - hb;
+            const int64_t row_n = __shfl_sync(kFullMask, srow, hb);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bar[2], bytes);
+                bulk_load(rbuf, a.staging + row_n * a.row_bytes + off, bytes, &bar[2]);
+            }
+            inflight |= 4u;
+            if (!__all_sync(kFullMask, mbar_wait(&bar[2], (parity >> 2) & 1u))) {
+                failed = true;
+                break;
+            }
+            parity ^= 4u;
+            inflight &= ~4u;
+            if (lane < a.k && sl >= 0 && nj == n)
+                bulk_store(a.dst + (int64_t)sl * a.row_bytes + off, rbuf, bytes);
+            bulk_commit();
+            bulk_wait_read<0>();  // R is free for the next node
+            __syncwarp();
+        }
+    }
+    if (failed) {
+        errbits |= kErrTimeout;
+        for (int i = 0; i < 3; ++i)
+            if (inflight & (1u << i)) (void)mbar_wait(&bar[i], (parity >> i) & 1u);
     }
     bulk_wait_all();
     warp_report(a.err, errbits);
@@ -402,6 +571,23 @@ cudaError_t launch_node_expand_bulk(const RowMoveParams& p, const void* staging,
     const BulkArgs a = bulk_args(p, staging, recv, staging_rows, p.T * p.k, kDispChunk);
     if (p.node_src != nullptr) return launch_disp_bulk<kNodeRows>(a, staging_rows, stream);
     return launch_disp_bulk<kNodeExpand>(a, p.T * p.N, stream);
+}
+
+bool node_dispatch_eligible(const RowMoveParams& p) { return p.N + p.k <= 32; }
+
+cudaError_t launch_node_dispatch_bulk(const RowMoveParams& p, const void* x, void* staging,
+                                      int64_t staging_rows, void* recv, cudaStream_t stream) {
+    BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kDispChunk);
+    a.staging = static_cast<char*>(staging);
+    a.staging_rows = staging_rows;
+    const int64_t items = p.T * a.cpr;
+    if (items <= 0) return cudaSuccess;
+    const size_t smem = (size_t)kNfWarps * 3 * (a.chunk + sizeof(uint64_t));
+    cudaError_t e = cudaFuncSetAttribute(node_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid<node_dispatch_kernel>(items, kNfThreads, smem);
+    return launch_pdl(node_dispatch_kernel, dim3(grid), dim3(kNfThreads), smem, stream, a);
 }
 
 cudaError_t launch_combine_bulk(const CombineParams& p, const void* expert_out, void* y,

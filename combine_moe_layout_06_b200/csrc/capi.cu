@@ -9,7 +9,8 @@ namespace {
 using moe::CopyEngine;
 
 constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK |
-                                 MOE_FLAG_LAYOUT_CLUSTER | MOE_FLAG_LAYOUT_FUSED;
+                                 MOE_FLAG_LAYOUT_CLUSTER | MOE_FLAG_LAYOUT_FUSED |
+                                 MOE_FLAG_TWO_LEVEL_FUSED;
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -75,6 +76,9 @@ moe_status_t dispatch_impl(const moe_config_t* c, const moe_layout_t* L, const v
     p.early_inputs = early;
     if (!two_level(c)) return cuda_status(moe::launch_dispatch_flat(p, x, recv, s));
     const int64_t rows = staging_rows(c);
+    if ((c->flags & MOE_FLAG_TWO_LEVEL_FUSED) != 0 && p.engine != CopyEngine::kVector &&
+        moe::bulk_eligible(p.row_bytes, {x, node_staging, recv}) && moe::node_dispatch_eligible(p))
+        return cuda_status(moe::launch_node_dispatch_bulk(p, x, node_staging, rows, recv, s));
     cudaError_t e = moe::launch_node_pack(p, x, node_staging, rows, s);
     p.early_inputs = false;  // expansion reads staging written by the pack
     if (e == cudaSuccess) e = moe::launch_node_expand(p, node_staging, rows, recv, s);

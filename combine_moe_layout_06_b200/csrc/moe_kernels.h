@@ -174,6 +174,13 @@ cudaError_t launch_node_pack_bulk(const RowMoveParams& p, const void* x, void* s
                                   int64_t staging_rows, cudaStream_t stream);
 cudaError_t launch_node_expand_bulk(const RowMoveParams& p, const void* staging,
                                     int64_t staging_rows, void* recv, cudaStream_t stream);
+// Two-level dispatch in one kernel: per (token, chunk), the x chunk goes to
+// the token's staging row of every node touched, and each staging row, once
+// written, is read back and goes to the token's receive rows on its node.
+// Needs N + k <= 32 (and 16-byte aligned rows, checked by the caller).
+bool node_dispatch_eligible(const RowMoveParams& p);
+cudaError_t launch_node_dispatch_bulk(const RowMoveParams& p, const void* x, void* staging,
+                                      int64_t staging_rows, void* recv, cudaStream_t stream);
 cudaError_t launch_combine_bulk(const CombineParams& p, const void* expert_out, void* y,
                                 cudaStream_t stream);
 

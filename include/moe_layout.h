@@ -74,6 +74,10 @@ extern "C" {
                                         and an assign/dispatch kernel instead
                                         of the layout kernels and the
                                         dispatch kernel (flat layouts) */
+#define MOE_FLAG_TWO_LEVEL_FUSED 0x20u /* two-level dispatch in one kernel
+                                          that reads each staging row back
+                                          right after writing it, instead of
+                                          a pack kernel then an expansion */
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -199,7 +203,12 @@ moe_status_t moe_layout(const moe_config_t *cfg, const int32_t *topk_idx,
  *                 written once per (token, node touched), node-major then
  *                 token order (FUSCO article, "负载均衡与跨节点去重"), then
  *                 expanded from staging to the expert rows of that node.
- *                 The final recv is identical in both modes. */
+ *                 The final recv is identical in both modes.
+ * Two-level engines: a pack kernel, then an expansion kernel.  With
+ * MOE_FLAG_TWO_LEVEL_FUSED, 16-byte aligned rows and N + k <= 32, one kernel
+ * does both phases, reading each staging row back right after writing it
+ * (the reads then come from L2); other configurations with the flag take the
+ * two kernels. */
 moe_status_t moe_dispatch(const moe_config_t *cfg, const moe_layout_t *layout,
                           const void *x, void *recv, void *node_staging,
                           void *stream);

@@ -19,6 +19,7 @@ TWO = capi.MOE_FLAG_TWO_LEVEL
 VEC = capi.MOE_FLAG_COPY_VECTOR
 BULK = capi.MOE_FLAG_COPY_BULK
 CL = capi.MOE_FLAG_LAYOUT_CLUSTER
+ONE = capi.MOE_FLAG_TWO_LEVEL_FUSED
 
 SMALL = [
     # T, H, E, k, R, N
@@ -63,7 +64,10 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
     eo = inputs.random_bf16_bits((T * k, H), seed=T * k + H)
     y_ref = oracle_mod.combine(eo, w, ref["slot"])
     x_dev = M.to_dev(x)
-    runs = [(f, True) for f in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK)]
+    # TWO: pack + expansion; TWO | ONE: one kernel (node staging, then the
+    # staging row read back) where N + k <= 32 and rows are 16-byte multiples
+    runs = [(f, True) for f in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK, TWO | ONE,
+                                TWO | ONE | BULK)]
     runs += [(f, False) for f in (TWO, TWO | VEC, TWO | BULK)]   # pair-walking expansion
     for flags, node_src in runs:
         cfg = M.cfg_of(T, H, E, k, R, N, flags)
@@ -110,12 +114,13 @@ def test_large_batch_multi_kernel_layout(oracle_mod, T):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
-@pytest.mark.parametrize("engine", [0, VEC, BULK])
+@pytest.mark.parametrize("engine", [0, VEC, BULK, ONE, ONE | BULK])
 @pytest.mark.parametrize("hot_frac", [0.0, 0.9, 1.0])
 def test_skewed_node_loads(oracle_mod, engine, hot_frac):
-    """One hot node (up to every token on node 0, the other nodes empty):
-    the row-balanced and the pair-walking expansions both reproduce the
-    oracle's staging and receive buffers bit for bit."""
+    """One hot node (up to every token on node 0, the other nodes empty): the
+    one-kernel two-level dispatch and, in the two-kernel form, the
+    row-balanced and the pair-walking expansions all reproduce the oracle's
+    staging and receive buffers bit for bit."""
     T, H, E, k, R, N = 5000, 264, 64, 6, 8, 4
     d = inputs.make_node_skewed(T, H, E, k, N, hot_frac, seed=int(hot_frac * 10) + 3)
     x, topk = d["x"], d["topk_idx"]
@@ -282,6 +287,31 @@ def test_workload_forced_engine(oracle_mod, name, engine):
     y = M.bits(M.gpu_combine(cfg, lay, M.to_dev(eo), w))
     assert np.array_equal(y, oracle_mod.combine(eo, w, ref["slot"]))
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+def test_workload_two_level_one_kernel(oracle_mod):
+    """The one-kernel two-level dispatch on the DeepSeek-V3-shaped workload
+    at full size: staging rows and receive rows as the oracle has them."""
+    d = inputs.make("dsv3")
+    wl = d["workload"]
+    x, topk = d["x"], d["topk_idx"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, TWO | ONE)
+    lay, _ = M.gpu_layout(cfg, topk)
+    x_dev = M.to_dev(x)
+    recv, staging = M.gpu_dispatch(cfg, lay, x_dev)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+    slot_dev = torch.from_numpy(ref["slot"].reshape(-1).astype(np.int64)).cuda()
+    tok_dev = torch.arange(wl.T, device="cuda").repeat_interleave(wl.k)
+    assert torch.equal(recv.view(torch.int16)[slot_dev], x_dev.view(torch.int16)[tok_dev])
+    del slot_dev, tok_dev, recv
+    U = int(ref["node_offsets"][-1])
+    node_tok = np.concatenate([np.flatnonzero(ref["node_slot"][:, n] >= 0) for n in range(wl.N)])
+    assert node_tok.size == U
+    assert torch.equal(staging[:U].view(torch.int16),
+                       x_dev.view(torch.int16)[torch.from_numpy(node_tok).cuda()])
+    del staging
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name", NAMES)
