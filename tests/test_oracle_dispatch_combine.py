@@ -231,7 +231,7 @@ def test_rank_partial_combine_order_is_rank_order(oracle_mod):
     vals = {0: 2.0 ** 20, 1: 2.0 ** -9, 2: -(2.0 ** 20)}
     eo = np.zeros((3, 1), np.uint16)
     for j, e in enumerate(topk[0]):
-        eo[lay["slot"][0, j], 0] = oracle_mod.f32_to_bf16(np.float32(vals[e]))
+        eo[lay["slot"][0, j], 0] = oracle_mod.f32_to_bf16(np.float32(vals[int(e)])).item()
     w = np.ones((1, 3), np.float32)
     y_rs = _bits_to_f64(oracle_mod.combine_rank_partials(eo, w, lay["slot"], lay["rank_offsets"]))
     y_col = _bits_to_f64(oracle_mod.combine(eo, w, lay["slot"]))
