@@ -187,24 +187,29 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle leg
 
-def oracle_step_time(d, tokens, reps, eo_bits):
+def oracle_step_time(d, tokens, reps, eo_bits, parallel=False):
     """Time the oracle (plain C loops, one thread) on the first `tokens`
-    tokens of the workload: layout, dispatch, combine.  Best of `reps`."""
+    tokens of the workload: layout, dispatch, combine.  Best of `reps`.
+    parallel: dispatch and combine through the oracle's OpenMP variants
+    (token loops over all host threads; the layout stays serial)."""
     import oracle
     wl = d["workload"]
     topk = np.ascontiguousarray(d["topk_idx"][:tokens])
     x = np.ascontiguousarray(d["x"][:tokens])
     w = np.ascontiguousarray(d["topk_w"][:tokens])
     eo = np.ascontiguousarray(eo_bits[: tokens * wl.k])
+    two = oracle.dispatch_two_level_par if parallel else oracle.dispatch_two_level
+    flat = oracle.dispatch_flat_par if parallel else oracle.dispatch_flat
+    comb = oracle.combine_par if parallel else oracle.combine
     best = float("inf")
     for _ in range(reps):
         t0 = time.perf_counter()
         lay = oracle.layout(topk, wl.E, wl.R, wl.N, nodes=wl.two_level)
         if wl.two_level:
-            oracle.dispatch_two_level(x, lay, wl.R, wl.N)
+            two(x, lay, wl.R, wl.N)
         else:
-            oracle.dispatch_flat(x, lay["slot"])
-        oracle.combine(eo, w, lay["slot"])
+            flat(x, lay["slot"])
+        comb(eo, w, lay["slot"])
         best = min(best, time.perf_counter() - t0)
     return best
 
@@ -826,7 +831,7 @@ def main():
     e2e_s = e2e_run(True)
     e2e_value = job_gbs(step_bytes, world, e2e_steps, e2e_s)
 
-    cpu = None
+    cpu = cpu_par = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         one = oracle_step_time(d, wl.T, 1, eo_bits)
         reps = max(1, min(30, int(args.cpu_seconds / max(one, 1e-3))))
@@ -835,6 +840,15 @@ def main():
                "kind": "oracle",
                "sample": f"full workload ({wl.T} tokens: layout+dispatch+combine), best of "
                          f"{reps + 1} runs, single thread on {os.cpu_count()} host cores"}
+        import oracle
+        threads = oracle.parallel_threads()
+        one = oracle_step_time(d, wl.T, 1, eo_bits, parallel=True)
+        reps = max(1, min(30, int(args.cpu_seconds / 2 / max(one, 1e-3))))
+        best = min(one, oracle_step_time(d, wl.T, reps, eo_bits, parallel=True))
+        cpu_par = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": threads,
+                   "kind": "oracle, dispatch and combine token loops over OpenMP threads "
+                           "(layout serial)",
+                   "sample": f"full workload ({wl.T} tokens), best of {reps + 1} runs"}
 
     if rank == 0:
         line = {
@@ -883,6 +897,7 @@ def main():
                             "on two copy streams over two buffer sets (wall clock)"},
             "gpu_launches": launches_per_step * K,
             "cpu_baseline": cpu,
+            "cpu_baseline_parallel": cpu_par,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -49,7 +49,7 @@ def build(force: bool = False) -> str:
         if fresh and not force:
             return _LIB
         tmp = _LIB + f".tmp{os.getpid()}"
-        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
                "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
@@ -87,6 +87,14 @@ def _bind(path: str):
     lib.oracle_dispatch_two_level.restype = None
     lib.oracle_combine.argtypes = [i64, i32, i32, p, p, p, p]
     lib.oracle_combine.restype = None
+    lib.oracle_parallel_threads.argtypes = []
+    lib.oracle_parallel_threads.restype = ctypes.c_int
+    lib.oracle_dispatch_flat_par.argtypes = [i64, i32, i32, p, p, p]
+    lib.oracle_dispatch_flat_par.restype = None
+    lib.oracle_dispatch_two_level_par.argtypes = [i64, i32, i32, i32, i32, p, p, p, p, p, p, p]
+    lib.oracle_dispatch_two_level_par.restype = None
+    lib.oracle_combine_par.argtypes = [i64, i32, i32, p, p, p, p]
+    lib.oracle_combine_par.restype = None
     lib.oracle_combine_tokens.argtypes = [i64, p, i32, i32, p, p, p, p]
     lib.oracle_combine_tokens.restype = None
     lib.oracle_combine_rank_partials.argtypes = [i64, i32, i32, i32, p, p, p, p, p]
@@ -259,6 +267,51 @@ def combine(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray) -> np.ndarray:
     H = eo_bits.shape[1]
     y = np.zeros((T, H), np.uint16)
     _load().oracle_combine(T, H, k, _ptr(slot), _ptr(w), _ptr(eo_bits), _ptr(y))
+    return y
+
+
+# ------------------------------------------- token loops over host threads
+# The same results as dispatch_flat / dispatch_two_level / combine, with the
+# token loops split over OpenMP threads (timing only; the layout stays serial).
+
+def parallel_threads() -> int:
+    """Threads the parallel variants use (OMP_NUM_THREADS, else all cores)."""
+    return int(_load().oracle_parallel_threads())
+
+
+def dispatch_flat_par(x_bits: np.ndarray, slot: np.ndarray) -> np.ndarray:
+    x_bits = _c(x_bits, np.uint16)
+    slot = _c(slot, np.int32)
+    T, H = x_bits.shape
+    k = slot.shape[1]
+    recv = np.zeros((T * k, H), np.uint16)
+    _load().oracle_dispatch_flat_par(T, H, k, _ptr(slot), _ptr(x_bits), _ptr(recv))
+    return recv
+
+
+def dispatch_two_level_par(x_bits: np.ndarray, lay: dict, R: int, N: int):
+    x_bits = _c(x_bits, np.uint16)
+    T, H = x_bits.shape
+    slot = _c(lay["slot"], np.int32)
+    k = slot.shape[1]
+    U = int(lay["node_offsets"][N])
+    staging = np.zeros((max(U, 1), H), np.uint16)
+    recv = np.zeros((T * k, H), np.uint16)
+    _load().oracle_dispatch_two_level_par(
+        T, H, k, R, N, _ptr(slot), _ptr(_c(lay["rank_offsets"], np.int32)),
+        _ptr(_c(lay["node_offsets"], np.int32)), _ptr(_c(lay["node_slot"], np.int32)),
+        _ptr(x_bits), _ptr(staging), _ptr(recv))
+    return staging[:U], recv
+
+
+def combine_par(eo_bits: np.ndarray, w: np.ndarray, slot: np.ndarray) -> np.ndarray:
+    eo_bits = _c(eo_bits, np.uint16)
+    w = _c(w, np.float32)
+    slot = _c(slot, np.int32)
+    T, k = slot.shape
+    H = eo_bits.shape[1]
+    y = np.zeros((T, H), np.uint16)
+    _load().oracle_combine_par(T, H, k, _ptr(slot), _ptr(w), _ptr(eo_bits), _ptr(y))
     return y
 
 

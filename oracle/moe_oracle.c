@@ -47,6 +47,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <math.h>
 
 /* Status codes.  Their meaning mirrors the library's public status enum by
@@ -478,6 +481,91 @@ void oracle_combine_tokens(int64_t n_tokens, const int64_t *tokens,
             y_rows[i * H + h] = oracle_f32_to_bf16(acc);
         }
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* Token loops over host threads (timing only)                         */
+/* ------------------------------------------------------------------ */
+
+/* oracle_dispatch_flat, oracle_dispatch_two_level and oracle_combine with
+ * their token loops split over OpenMP threads.  Each token's rows are written
+ * by one thread with exactly the arithmetic of the serial functions, so the
+ * results are identical; the layout stays serial (its slot order is defined
+ * by token order).  These exist to time the oracle on all host cores beside
+ * the single-thread runs; the serial functions above are the reference. */
+int oracle_parallel_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_dispatch_flat_par(int64_t T, int32_t H, int32_t k,
+                              const int32_t *slot, const uint16_t *x,
+                              uint16_t *recv)
+{
+    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < k; ++j) {
+            int64_t dst = slot[t * k + j];
+            memcpy(recv + dst * H, x + t * H, row_bytes);
+        }
+}
+
+void oracle_dispatch_two_level_par(int64_t T, int32_t H, int32_t k, int32_t R,
+                                   int32_t N, const int32_t *slot,
+                                   const int32_t *rank_offsets,
+                                   const int32_t *node_offsets,
+                                   const int32_t *node_slot,
+                                   const uint16_t *x, uint16_t *staging,
+                                   uint16_t *recv)
+{
+    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+    int32_t ranks_per_node = R / N;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t n = 0; n < N; ++n) {
+            int32_t ns = node_slot[t * N + n];
+            if (ns >= 0) {
+                int64_t row = (int64_t)node_offsets[n] + ns;
+                memcpy(staging + row * H, x + t * H, row_bytes);
+            }
+        }
+    for (int32_t n = 0; n < N; ++n) {
+        int32_t lo = rank_offsets[n * ranks_per_node];
+        int32_t hi = rank_offsets[(n + 1) * ranks_per_node];
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < T; ++t) {
+            int32_t ns = node_slot[t * N + n];
+            if (ns < 0)
+                continue;
+            int64_t srow = (int64_t)node_offsets[n] + ns;
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t dst = slot[t * k + j];
+                if (dst >= lo && dst < hi)
+                    memcpy(recv + (int64_t)dst * H, staging + srow * H, row_bytes);
+            }
+        }
+    }
+}
+
+void oracle_combine_par(int64_t T, int32_t H, int32_t k, const int32_t *slot,
+                        const float *w, const uint16_t *eo, uint16_t *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                int64_t row = slot[t * k + j];
+                float v = oracle_bf16_to_f32(eo[row * H + h]);
+                acc = fmaf(w[t * k + j], v, acc);
+            }
+            y[t * H + h] = oracle_f32_to_bf16(acc);
+        }
 }
 
 /* Combine in the reduce-scatter order (INC-MoE abstract: combine as a
