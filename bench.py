@@ -187,6 +187,19 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- oracle leg
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    import platform
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or platform.machine()
+
+
 def oracle_step_time(d, tokens, reps, eo_bits, parallel=False):
     """Time the oracle (plain C loops, one thread) on the first `tokens`
     tokens of the workload: layout, dispatch, combine.  Best of `reps`.
@@ -839,7 +852,8 @@ def main():
         cpu = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": 1,
                "kind": "oracle",
                "sample": f"full workload ({wl.T} tokens: layout+dispatch+combine), best of "
-                         f"{reps + 1} runs, single thread on {os.cpu_count()} host cores"}
+                         f"{reps + 1} runs, single thread on {os.cpu_count()} host cores",
+               "cpu_model": cpu_model()}
         import oracle
         threads = oracle.parallel_threads()
         one = oracle_step_time(d, wl.T, 1, eo_bits, parallel=True)
