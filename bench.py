@@ -600,7 +600,8 @@ def main():
         capi.moe_dispatch_allgather(cfg, b.lay.struct, b.x, b.gathered, b.recv)
         capi.moe_combine_reducescatter(cfg, b.lay.struct, b.eo, b.w, b.partial, b.y)
 
-    cluster_layout = args.layout == "cluster" and wl.T <= 131072
+    # one cluster launch when asked for, and always for one chunk of 256 tokens
+    cluster_layout = (args.layout == "cluster" and wl.T <= 131072) or wl.T <= 256
     small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
     layout_launches = 1 if cluster_layout else (2 if small_layout else 3)
     # moe_layout_dispatch as the count + assign/dispatch pair (the library's

@@ -24,9 +24,10 @@
 // slower inside a CUDA-graph step than the three kernels below, whose launch
 // latencies overlap through programmatic dependent launch, so it is opt-in.
 //
-// By default, count then assign with the scan folded in (up to 256 chunks of
-// 256 tokens), else three kernels; no global sort and no atomics on
-// positions:
+// By default (more than one chunk of 256 tokens), count then assign with the
+// scan folded in (up to 256 chunks), else three kernels; no global sort and
+// no atomics on positions.  A batch of one chunk takes the cluster kernel
+// with a cluster of one CTA:
 //   count  : one CTA per chunk of 256 tokens builds an expert histogram (and a
 //            node-touch histogram) in shared memory and writes it to the
 //            workspace column of its chunk, cnt[e][chunk].
@@ -777,7 +778,10 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     a.node_slot = p.node_slot;
     a.node_src = p.nodes ? p.node_src : nullptr;
     a.err = p.err;
-    if (p.cluster && p.T <= kClusterMaxTokens)
+    // One chunk of tokens (T <= 256): one CTA sees every token, so the
+    // single-cluster kernel (a cluster of one CTA) does the whole layout in one
+    // launch, with no count kernel and no kernel boundary before the ranks.
+    if ((p.cluster && p.T <= kClusterMaxTokens) || (p.T > 0 && a.C == 1))
         return p.k <= 8 ? launch_layout_cluster<8>(a, stream) : launch_layout_cluster<32>(a, stream);
     return p.k <= 8 ? launch_layout_k<8>(a, stream) : launch_layout_k<32>(a, stream);
 }
