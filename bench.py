@@ -12,7 +12,7 @@ device synchronise on both sides).  Steps alternate between two independent
 buffer sets (inputs, layout, outputs), so no step finds its inputs in L2:
 a buffer is touched again only after about twice the step's traffic (the
 OLMoE-shaped step alone moves 302 MB, 2.4x the L2).  Steps are replayed from
-CUDA graphs of two steps.  Stage costs come from the same protocol applied
+CUDA graphs of GRAPH_STEPS (10) steps.  Stage costs come from the same protocol applied
 to graphs of layout only and layout + dispatch: dispatch = (layout +
 dispatch) - layout, combine = step - (layout + dispatch).  The decoupled
 pack -> copy -> unpack path is timed the same way for comparison.
@@ -59,6 +59,9 @@ def measured_peak():
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
 
+
+# Steps per CUDA graph replay in the timed loops.
+GRAPH_STEPS = 10
 
 KERNEL_SOURCES = {
     "combine": ["combine.cu", "moe_common.cuh"],
@@ -631,49 +634,52 @@ def main():
             if st != capi.MOE_OK:
                 raise SystemExit(f"device error after warm-up: {capi.moe_status_string(st)}")
 
-    # CUDA graphs over the two buffer sets: a pair of steps (A then B), and a
-    # single step for an odd K; stage prefixes for the breakdown.
+    # CUDA graphs over the two buffer sets: GRAPH_STEPS steps alternating A
+    # and B, a pair (A then B) and a single step for the remainder of K; stage
+    # prefixes for the breakdown.  Programmatic dependent launch overlaps
+    # consecutive kernels inside a graph but not across two replays, so longer
+    # graphs measure the steady state a model-level graph sees (one replay
+    # boundary costs about 2 us).
     side = torch.cuda.Stream(dev)
 
-    def capture(fn):
+    def capture(fn, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
-            fn()
+            for i in range(n):
+                fn(sets[i % 2])
         return g
 
-    A, B = sets
-    graphs = {
-        "step": (capture(lambda: (step(A), step(B))), capture(lambda: step(A))),
-        "L": (capture(lambda: (layout(A), layout(B))), capture(lambda: layout(A))),
-        "LD": (capture(lambda: (layout_dispatch(A), layout_dispatch(B))),
-               capture(lambda: layout_dispatch(A))),
-    }
+    def graph_set(fn):
+        return capture(fn, GRAPH_STEPS), capture(fn, 2), capture(fn, 1)
+
+    graphs = {"step": graph_set(step), "L": graph_set(layout), "LD": graph_set(layout_dispatch)}
     if with_decoupled:
-        graphs["decoupled"] = (capture(lambda: (decoupled_step(A), decoupled_step(B))),
-                               capture(lambda: decoupled_step(A)))
+        graphs["decoupled"] = graph_set(decoupled_step)
     if with_agrs:
-        graphs["agrs"] = (capture(lambda: (agrs_step(A), agrs_step(B))), capture(lambda: agrs_step(A)))
+        graphs["agrs"] = graph_set(agrs_step)
     if with_fp8:
-        graphs["fp8"] = (capture(lambda: (fp8_step(A), fp8_step(B))), capture(lambda: fp8_step(A)))
-        graphs["fp8_LD"] = (capture(lambda: (fp8_layout_dispatch(A), fp8_layout_dispatch(B))),
-                            capture(lambda: fp8_layout_dispatch(A)))
+        graphs["fp8"] = graph_set(fp8_step)
+        graphs["fp8_LD"] = graph_set(fp8_layout_dispatch)
     if with_ep:
-        graphs["ep"] = (capture(lambda: (ep_step(A), ep_step(B))), capture(lambda: ep_step(A)))
-    for pair, single in graphs.values():
-        pair.replay()
-        single.replay()
+        graphs["ep"] = graph_set(ep_step)
+    for gs in graphs.values():
+        for g in gs:
+            g.replay()
     torch.cuda.synchronize()
 
     def timed(name, K):
         """K steps back to back between two events on the stream (ms)."""
-        pair, single = graphs[name]
+        multi, pair, single = graphs[name]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
         e0.record()
-        for _ in range(K // 2):
+        for _ in range(K // GRAPH_STEPS):
+            multi.replay()
+        rest = K % GRAPH_STEPS
+        for _ in range(rest // 2):
             pair.replay()
-        if K % 2:
+        if rest % 2:
             single.replay()
         e1.record()
         torch.cuda.synchronize()
@@ -687,7 +693,7 @@ def main():
                           dtype=torch.float32, device=dev)
 
     def flushed_steps(K):
-        single = graphs["step"][1]
+        single = graphs["step"][2]
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(K)]
         barrier()
@@ -881,9 +887,9 @@ def main():
                                    ("count + assign kernels" if small_layout
                                     else "count/scan/assign kernels")),
                            entry="moe_layout + moe_dispatch" if args.unfused else "moe_layout_dispatch",
-                           timing="K steps back to back (CUDA graphs of two steps) between two CUDA "
-                                  "events on the launching stream; stage costs from graphs of "
-                                  "layout, layout+dispatch and the full step"),
+                           timing=f"K steps back to back (CUDA graphs of {GRAPH_STEPS} steps) between "
+                                  "two CUDA events on the launching stream; stage costs from graphs "
+                                  "of layout, layout+dispatch and the full step"),
             "pct_of_peak": round(100 * value / world / peak, 2),
             "peak_gbs": peak, "peak_source": peak_src,
             "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
