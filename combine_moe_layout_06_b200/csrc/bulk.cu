@@ -6,8 +6,9 @@
 // SM's bulk-copy unit instead of by registers:
 //
 //  dispatch: each warp runs its own pipeline of kDispStages shared-memory
-//    stages.  Lane 0 starts a cp.async.bulk global->shared load of a row
-//    chunk into a stage (completion counted on the stage's mbarrier); when
+//    stages (8 stages of 2 KB by default: the best ring shape of a sweep at
+//    16 KB per warp).  Lane 0 starts a cp.async.bulk global->shared load of
+//    a row chunk into a stage (completion counted on the stage's mbarrier); when
 //    it lands, every lane that holds a destination row issues a
 //    cp.async.bulk shared->global store of the stage to that row.  Rows are
 //    read once and written k times without passing through registers, so

@@ -12,8 +12,9 @@
 // rounds to nearest even.
 //
 // Work items are (token, row chunk) pairs, a chunk being 32*VPL vectors of
-// the row, over a persistent grid sized to what is resident; each warp takes
-// a contiguous token-major range of items, so a token's k slots and weights
+// the row, over a grid from persistent_grid() (resident, or whole resident
+// waves for large problems); each warp takes a contiguous token-major range
+// of items, so a token's k slots and weights
 // (held one per lane) are loaded once, and the next token's are fetched
 // while the current chunk's rows are in flight.  The chunk of up to KB
 // expert rows is loaded before any FMA, so KB*VPL streaming loads per lane

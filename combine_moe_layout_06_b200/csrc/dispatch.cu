@@ -11,10 +11,11 @@
 // pack -> copy -> unpack path that section "传统 MoE 通信的痛点" describes.
 //
 // Register engine: work items are (source row, row chunk) pairs, a chunk
-// being 32*VPL vectors, handed out warp by warp over a persistent grid sized
-// to what is resident.  Lanes hold the destination rows (k <= 32 slots, or
-// N <= 32 nodes); the chunk is loaded once with streaming loads and stored
-// to every destination with evict-first stores.
+// being 32*VPL vectors, handed out warp by warp over a grid from
+// persistent_grid() (resident, or whole resident waves for large
+// problems).  Lanes hold the destination rows (k <= 32 slots, or N <= 32
+// nodes); the chunk is loaded once with streaming loads and stored to every
+// destination with evict-first stores.
 #include <climits>
 #include <initializer_list>
 
