@@ -506,13 +506,11 @@ void oracle_dispatch_flat_par(int64_t T, int32_t H, int32_t k,
                               const int32_t *slot, const uint16_t *x,
                               uint16_t *recv)
 {
-    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
+    size_t bytes = sizeof(uint16_t) * (size_t)H;
 #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < T; ++t)
-        for (int32_t j = 0; j < k; ++j) {
-            int64_t dst = slot[t * k + j];
-            memcpy(recv + dst * H, x + t * H, row_bytes);
-        }
+    for (int64_t tok = 0; tok < T; ++tok)
+        for (int32_t col = 0; col < k; ++col)
+            memcpy(recv + (int64_t)slot[tok * k + col] * H, x + tok * H, bytes);
 }
 
 void oracle_dispatch_two_level_par(int64_t T, int32_t H, int32_t k, int32_t R,
@@ -523,30 +521,29 @@ void oracle_dispatch_two_level_par(int64_t T, int32_t H, int32_t k, int32_t R,
                                    const uint16_t *x, uint16_t *staging,
                                    uint16_t *recv)
 {
-    size_t row_bytes = sizeof(uint16_t) * (size_t)H;
-    int32_t ranks_per_node = R / N;
+    size_t bytes = sizeof(uint16_t) * (size_t)H;
+    int32_t per_node = R / N;
 #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < T; ++t)
-        for (int32_t n = 0; n < N; ++n) {
-            int32_t ns = node_slot[t * N + n];
-            if (ns >= 0) {
-                int64_t row = (int64_t)node_offsets[n] + ns;
-                memcpy(staging + row * H, x + t * H, row_bytes);
-            }
-        }
-    for (int32_t n = 0; n < N; ++n) {
-        int32_t lo = rank_offsets[n * ranks_per_node];
-        int32_t hi = rank_offsets[(n + 1) * ranks_per_node];
-#pragma omp parallel for schedule(static)
-        for (int64_t t = 0; t < T; ++t) {
-            int32_t ns = node_slot[t * N + n];
-            if (ns < 0)
+    for (int64_t tok = 0; tok < T; ++tok)
+        for (int32_t nd = 0; nd < N; ++nd) {
+            int32_t rank_in_node = node_slot[tok * N + nd];
+            if (rank_in_node < 0)
                 continue;
-            int64_t srow = (int64_t)node_offsets[n] + ns;
-            for (int32_t j = 0; j < k; ++j) {
-                int32_t dst = slot[t * k + j];
-                if (dst >= lo && dst < hi)
-                    memcpy(recv + (int64_t)dst * H, staging + srow * H, row_bytes);
+            memcpy(staging + ((int64_t)node_offsets[nd] + rank_in_node) * H, x + tok * H, bytes);
+        }
+    for (int32_t nd = 0; nd < N; ++nd) {
+        int32_t first = rank_offsets[nd * per_node];
+        int32_t last = rank_offsets[(nd + 1) * per_node];
+#pragma omp parallel for schedule(static)
+        for (int64_t tok = 0; tok < T; ++tok) {
+            int32_t rank_in_node = node_slot[tok * N + nd];
+            if (rank_in_node < 0)
+                continue;
+            const uint16_t *from = staging + ((int64_t)node_offsets[nd] + rank_in_node) * H;
+            for (int32_t col = 0; col < k; ++col) {
+                int32_t to = slot[tok * k + col];
+                if (to >= first && to < last)
+                    memcpy(recv + (int64_t)to * H, from, bytes);
             }
         }
     }
@@ -556,15 +553,13 @@ void oracle_combine_par(int64_t T, int32_t H, int32_t k, const int32_t *slot,
                         const float *w, const uint16_t *eo, uint16_t *y)
 {
 #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < T; ++t)
-        for (int32_t h = 0; h < H; ++h) {
-            float acc = 0.0f;
-            for (int32_t j = 0; j < k; ++j) {
-                int64_t row = slot[t * k + j];
-                float v = oracle_bf16_to_f32(eo[row * H + h]);
-                acc = fmaf(w[t * k + j], v, acc);
-            }
-            y[t * H + h] = oracle_f32_to_bf16(acc);
+    for (int64_t tok = 0; tok < T; ++tok)
+        for (int32_t col_h = 0; col_h < H; ++col_h) {
+            float sum = 0.0f;
+            for (int32_t col = 0; col < k; ++col)
+                sum = fmaf(w[tok * k + col],
+                           oracle_bf16_to_f32(eo[(int64_t)slot[tok * k + col] * H + col_h]), sum);
+            y[tok * H + col_h] = oracle_f32_to_bf16(sum);
         }
 }
 
