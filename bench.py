@@ -1,23 +1,36 @@
 """Benchmark: MoE dispatch + combine fused with layout on B200.
 
 One step = the whole hot path over one batch: layout (histogram, scan, slot
-assignment), fused dispatch (flat, or two-level through node staging for the
-DeepSeek-V3-shaped workload) and fused combine.  The combine reads a separate
-stand-in expert-output buffer (as it would after the expert GEMMs), so no
-step reads rows the same step just wrote through L2.
+assignment), fused dispatch (two-level through node staging for the
+DeepSeek-V3-shaped workload, flat for the others) and fused combine.  The
+combine reads a separate stand-in expert-output buffer (as it would after the
+expert GEMMs), so no step reads rows the same step just wrote through L2.
+
+One GPU (the default): the headline is the DeepSeek-V3-shaped workload
+(T=16384 H=7168 E=256 k=8, R=8 ranks on N=2 nodes, two-level dispatch), the
+largest of the five.  `per_workload` holds the same measurement of the other
+four workloads, timed in the same process under the same protocol.
 
 Timing: W untimed warm-up steps, then exactly K timed steps back to back,
 bracketed by two CUDA events on the launching stream (and a barrier plus a
 device synchronise on both sides).  Steps alternate between two independent
-buffer sets (inputs, layout, outputs), so no step finds its inputs in L2:
-a buffer is touched again only after about twice the step's traffic (the
-OLMoE-shaped step alone moves 302 MB, 2.4x the L2).  Steps are replayed from
-CUDA graphs of GRAPH_STEPS (10) steps.  Stage costs come from the same protocol applied
-to graphs of layout only and layout + dispatch: dispatch = (layout +
-dispatch) - layout, combine = step - (layout + dispatch).  The decoupled
-pack -> copy -> unpack path is timed the same way for comparison.
-Multi-GPU runs are independent replicas (no collective on the data path):
-value = bytes all ranks moved / the max over ranks of the timed time.
+buffer sets (inputs, layout, outputs), so no step finds its inputs in L2: a
+buffer is touched again only after about twice the step's traffic.  Steps
+are replayed from CUDA graphs of GRAPH_STEPS (10) steps.  Stage costs come
+from the same protocol applied to graphs of layout only and layout +
+dispatch: dispatch = (layout + dispatch) - layout, combine = step - (layout
++ dispatch).  The decoupled pack -> copy -> unpack path is timed the same
+way for comparison.
+
+Several GPUs (torchrun, one rank per GPU): the headline is expert
+parallelism over sharded sources across the processes.  Every rank routes a
+batch of its own; the per-expert counts are all-gathered (NCCL); the
+dispatch and combine kernels store to and load from every rank's receive and
+expert-output buffers through CUDA IPC mappings; an NCCL all-reduce of one
+word separates dispatch, the experts' slot and combine, as a barrier would.
+value = bytes all ranks moved / the max over ranks of the timed time.  The
+single-GPU step run on every rank at once (no collective on the data path)
+is kept as `replicas`.
 
 Metric: achieved algorithmic HBM GB/s of dispatch + combine.  Algorithmic
 bytes per step are T*H*2 + T*k*H*2 for dispatch (read each token row once,
@@ -25,12 +38,13 @@ write each destination row once) and the same for combine (read each expert
 row once, write each output row once); layout metadata and node staging
 traffic are not credited.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload olmoe]
-                    [--impl reference] [--engine auto|vector|bulk]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3]
+                    [--tokens T] [--impl reference] [--engine auto|vector|bulk]
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import os
@@ -49,6 +63,8 @@ from combine_moe_layout_06_b200 import inputs  # noqa: E402
 METRIC = "dispatch+combine achieved HBM GB/s, % of B200 peak, and tokens/s on 1 GPU"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "dsv3"
+WORKLOAD_ORDER = ("tiny", "olmoe", "qwen3", "dsv3", "longctx")
 
 
 def measured_peak():
@@ -125,9 +141,16 @@ def algorithmic_bytes(wl, tokens=None):
 NODE_SKEW = dict(T=16384, H=7168, E=256, k=8, R=8, N=2, hot_frac=0.9, seed=1240)
 
 
+def workload_inputs(name, tokens=0, source=0):
+    d = inputs.make_source(name, source)
+    return inputs.prefix(d, tokens) if tokens else d
+
+
 def workload_desc(wl):
+    full = inputs.WORKLOADS[wl.name].T
+    name = wl.name if wl.T == full else f"{wl.name} (first {wl.T} of {full} tokens)"
     return {
-        "workload": f"{wl.name}: {inputs.DESCRIPTIONS[wl.name]}",
+        "workload": f"{name}: {inputs.DESCRIPTIONS[wl.name]}",
         "tokens": wl.T, "hidden": wl.H, "experts": wl.E, "top_k": wl.k,
         "virtual_ranks": wl.R, "virtual_nodes": wl.N,
         "dispatch_mode": "two-level node staging" if wl.two_level else "flat",
@@ -230,14 +253,26 @@ def oracle_step_time(d, tokens, reps, eo_bits, parallel=False):
     return best
 
 
+# Bytes of dispatch + combine per reference-arm step: the sample is the first
+# tokens of the workload whose step moves about this many bytes.
+REF_SAMPLE_BYTES = 128 << 20
+
+
+def reference_tokens(wl, requested=0):
+    if requested:
+        return max(1, min(wl.T, requested))
+    per_token = sum(algorithmic_bytes(wl, 1))
+    return max(1, min(wl.T, REF_SAMPLE_BYTES // per_token))
+
+
 def run_reference(args):
     """The comparison arm: the oracle, as it stands, on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    d = inputs.make(args.workload)
+    d = workload_inputs(args.workload, args.tokens)
     wl = d["workload"]
-    tokens = max(1, min(wl.T, args.ref_tokens or max(1, wl.T // 8)))
+    tokens = reference_tokens(wl, args.ref_tokens)
     eo = inputs.random_bf16_bits((tokens * wl.k, wl.H), seed=wl.seed + 7)
     for _ in range(args.warmup):
         oracle_step_time(d, tokens, 1, eo)
@@ -297,7 +332,26 @@ def hbm_probe():
 
 # ---------------------------------------------------------------- our arm
 
-def node_balance(args, dev, world, barrier, flags):
+@dataclasses.dataclass
+class Ctx:
+    world: int
+    rank: int
+    local: int
+    dev: object
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+
+def engine_flags(args):
+    from combine_moe_layout_06_b200 import capi
+    return {"auto": 0, "vector": capi.MOE_FLAG_COPY_VECTOR,
+            "bulk": capi.MOE_FLAG_COPY_BULK}[args.engine]
+
+
+def node_balance(args, ctx):
     """Two-level dispatch on a hot-node routing (NODE_SKEW), with the second
     phase walking (node, token) pairs (no node_src) and staging rows
     (node_src given).  Same protocol as the main step: two buffer sets,
@@ -306,11 +360,11 @@ def node_balance(args, dev, world, barrier, flags):
     import torch
 
     from combine_moe_layout_06_b200 import buffers, capi
+    dev, world = ctx.dev, ctx.world
     sk = NODE_SKEW
     T, H, E, k, R, N = (sk[c] for c in ("T", "H", "E", "k", "R", "N"))
     d = inputs.make_node_skewed(T, H, E, k, N, sk["hot_frac"], sk["seed"])
-    cfg = capi.config(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | (flags & (
-        capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK)))
+    cfg = capi.config(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | engine_flags(args))
     bf16 = dict(dtype=torch.bfloat16, device=dev)
     rows = capi.moe_node_staging_rows(cfg)
 
@@ -351,14 +405,14 @@ def node_balance(args, dev, world, barrier, flags):
 
     def timed(key):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
+        ctx.barrier()
         torch.cuda.synchronize()
         e0.record()
         for _ in range(K2):
             graphs[key].replay()
         e1.record()
         torch.cuda.synchronize()
-        barrier()
+        ctx.barrier()
         return max_over_ranks(e0.elapsed_time(e1), world, dev) / (2 * K2)
 
     out = {}
@@ -385,13 +439,784 @@ def node_balance(args, dev, world, barrier, flags):
             "bytes_per_step": disp_b}
 
 
-def main():
+class StepBench:
+    """One workload's step over two independent buffer sets: the buffers,
+    the CUDA graphs of the step and of its stage prefixes, and the timed
+    loops.  `extras` adds the comparison paths: "decoupled" (pack / copy /
+    unpack), "agrs" (all-gather / reduce-scatter), "fp8" (e4m3 payload) and
+    "ep" (sharded sources, the workload's R ranks on this GPU)."""
+
+    def __init__(self, ctx, args, d, extras=()):
+        import torch
+
+        from combine_moe_layout_06_b200 import buffers, capi
+        self.ctx, self.args, self.d = ctx, args, d
+        wl = self.wl = d["workload"]
+        dev = ctx.dev
+        flags = capi.MOE_FLAG_TWO_LEVEL if wl.two_level else 0
+        flags |= engine_flags(args)
+        if args.layout == "cluster":
+            flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
+        if args.layout == "fused":
+            flags |= capi.MOE_FLAG_LAYOUT_FUSED
+        if args.two_level_fused:
+            flags |= capi.MOE_FLAG_TWO_LEVEL_FUSED
+        self.flags = flags
+        cfg = self.cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
+        # the decoupled comparison path packs per rank: one "node" per rank
+        copy_bits = flags & (capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK)
+        dcfg = self.dcfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R,
+                                       capi.MOE_FLAG_TWO_LEVEL | copy_bits)
+        eo_bits = self.eo_bits = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
+        bf16 = dict(dtype=torch.bfloat16, device=dev)
+        self.with_decoupled = "decoupled" in extras
+        self.with_agrs = "agrs" in extras and wl.R <= capi.MOE_MAX_NODES
+        self.with_fp8 = "fp8" in extras and wl.H % 8 == 0
+        self.with_ep = "ep" in extras and wl.R <= capi.MOE_MAX_NODES and not wl.two_level
+
+        # Expert parallelism over sharded sources with every rank on this
+        # GPU: rank g routes tokens [sb[g], sb[g+1]); its receive and
+        # expert-output buffers are the rank's rows of the set's recv / eo
+        # (pointer tables).  The per-expert counts of each shard come from
+        # the library's own layout, the rows per rank from its C ABI.
+        G = self.G = wl.R
+        sb = self.sb = (np.arange(G + 1, dtype=np.int64) * wl.T) // G
+        if self.with_ep:
+            ep_cfgs = self.ep_cfgs = [capi.config(int(sb[g + 1] - sb[g]), wl.H, wl.E, wl.k, wl.R, 1,
+                                                  copy_bits) for g in range(G)]
+            topk_all = torch.from_numpy(d["topk_idx"]).to(dev)
+            counts = []
+            for g in range(G):
+                lay = buffers.DeviceLayout(ep_cfgs[g], dev)
+                capi.moe_layout(ep_cfgs[g], topk_all[int(sb[g]):int(sb[g + 1])], lay.struct)
+                counts.append(lay.expert_counts.cpu().numpy())
+            ep_rows = self.ep_rows = np.array(capi.moe_ep_receive_rows(np.stack(counts), wl.R))
+            ep_first = np.concatenate([[0], np.cumsum(ep_rows)])
+            del topk_all
+
+        outer = self
+
+        class EpShards:
+            """Per-rank layouts and sharded-source arrays of one buffer set."""
+
+            def __init__(self, b):
+                i32 = dict(dtype=torch.int32, device=dev)
+                self.lays = [buffers.DeviceLayout(c, dev) for c in outer.ep_cfgs]
+                self.counts_all = torch.zeros((G, wl.E), **i32)
+                self.arrays = [(torch.zeros(wl.E + 1, **i32), torch.zeros(wl.R + 1, **i32),
+                                torch.zeros(max(c.num_tokens * wl.k, 1), **i32))
+                               for c in outer.ep_cfgs]
+                self.structs = [capi.ep_layout_struct(*a) for a in self.arrays]
+                row = wl.H * 2
+                self.recv_bufs = [b.recv.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
+                self.eo_bufs = [b.eo.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
+                self.cap = int(ep_rows.max())
+
+        class BufferSet:
+            """One independent set of the step's inputs and outputs."""
+
+            def __init__(self):
+                self.lay = buffers.DeviceLayout(cfg, dev)
+                self.x = buffers.bf16_from_bits(d["x"], dev)
+                self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
+                self.w = torch.from_numpy(d["topk_w"]).to(dev)
+                self.eo = buffers.bf16_from_bits(eo_bits, dev)
+                self.recv = torch.empty((wl.T * wl.k, wl.H), **bf16)
+                self.y = torch.empty((wl.T, wl.H), **bf16)
+                self.staging = None
+                if wl.two_level:
+                    self.staging = torch.empty((capi.moe_node_staging_rows(cfg), wl.H), **bf16)
+                if outer.with_decoupled:
+                    self.dlay = buffers.DeviceLayout(dcfg, dev)
+                    rows = capi.moe_node_staging_rows(dcfg)
+                    self.dsend = torch.empty((rows, wl.H), **bf16)
+                    self.dxfer = torch.empty((rows, wl.H), **bf16)
+                    self.csend = torch.empty((wl.T * wl.k, wl.H), **bf16)
+                    self.cxfer = torch.empty((wl.T * wl.k, wl.H), **bf16)
+                if outer.with_fp8:
+                    rows = wl.T * wl.k
+                    self.recv_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
+                    self.recv_s = torch.empty(rows, dtype=torch.float32, device=dev)
+                    self.eo_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
+                    self.eo_s = torch.empty(rows, dtype=torch.float32, device=dev)
+                    # expert outputs as an fp8 producer would emit them
+                    capi.moe_quantize_rows_fp8(self.eo, rows, wl.H, self.eo_q, self.eo_s)
+                    if wl.two_level:
+                        srows = capi.moe_node_staging_rows(cfg)
+                        self.st_q = torch.empty((srows, wl.H), dtype=torch.uint8, device=dev)
+                        self.st_s = torch.empty(srows, dtype=torch.float32, device=dev)
+                if outer.with_agrs:
+                    self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
+                    self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
+                self.ep = EpShards(self) if outer.with_ep else None
+
+        self.sets = [BufferSet(), BufferSet()]
+        self.ep_streams = [torch.cuda.Stream(dev) for _ in range(G)] if self.with_ep else []
+
+        # one cluster launch when asked for, and always for one chunk of 256 tokens
+        self.cluster_layout = (args.layout == "cluster" and wl.T <= 131072) or wl.T <= 256
+        self.small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
+        layout_launches = 1 if self.cluster_layout else (2 if self.small_layout else 3)
+        # moe_layout_dispatch as the count + assign/dispatch pair (the
+        # library's rule: flat, 16-byte rows, at most 256 experts, no engine
+        # or layout override)
+        self.ld_pair = (not args.unfused and not wl.two_level and args.layout == "fused"
+                        and (wl.H * 2) % 16 == 0 and wl.E <= 256)
+        # two-level: pack + expand, or one kernel with --two-level-fused
+        # (16-byte rows, N + k <= 32)
+        self.two_kernels = wl.two_level and (not args.two_level_fused or args.engine == "vector"
+                                             or (wl.H * 2) % 16 or wl.N + wl.k > 32)
+        self.launches_per_step = (2 if self.ld_pair else
+                                  layout_launches + (2 if self.two_kernels else 1)) + 1
+        self.graphs = {}
+
+    # ---- the step and its parts
+    def layout(self, b):
+        from combine_moe_layout_06_b200 import capi
+        capi.moe_layout(self.cfg, b.topk, b.lay.struct)
+
+    def layout_dispatch(self, b):
+        from combine_moe_layout_06_b200 import capi
+        if self.args.unfused:
+            self.layout(b)
+            capi.moe_dispatch(self.cfg, b.lay.struct, b.x, b.recv, b.staging)
+        else:
+            capi.moe_layout_dispatch(self.cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
+
+    def step(self, b):
+        from combine_moe_layout_06_b200 import capi
+        self.layout_dispatch(b)
+        capi.moe_combine(self.cfg, b.lay.struct, b.eo, b.w, b.y)
+
+    def decoupled_step(self, b):
+        from combine_moe_layout_06_b200 import capi
+        capi.moe_layout(self.dcfg, b.topk, b.dlay.struct)
+        capi.moe_dispatch_decoupled(self.dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
+        capi.moe_combine_decoupled(self.dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
+
+    def fp8_layout_dispatch(self, b):
+        from combine_moe_layout_06_b200 import capi
+        self.layout(b)
+        if self.wl.two_level:
+            capi.moe_dispatch_fp8_two_level(self.cfg, b.lay.struct, b.x, b.st_q, b.st_s,
+                                            b.recv_q, b.recv_s)
+        else:
+            capi.moe_dispatch_fp8(self.cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
+
+    def fp8_step(self, b):
+        from combine_moe_layout_06_b200 import capi
+        self.fp8_layout_dispatch(b)
+        capi.moe_combine_fp8(self.cfg, b.lay.struct, b.eo_q, b.eo_s, b.w, b.y)
+
+    def ep_phase(self, fn):
+        """Run fn(g) for every rank on its own stream, all after the work
+        enqueued so far and before anything enqueued later (the ranks of a
+        multi-GPU system run concurrently; the joins stand for its barriers)."""
+        import torch
+        cur = torch.cuda.current_stream()
+        for st in self.ep_streams:
+            st.wait_stream(cur)
+        for g, st in enumerate(self.ep_streams):
+            with torch.cuda.stream(st):
+                fn(g)
+        for st in self.ep_streams:
+            cur.wait_stream(st)
+
+    def ep_step(self, b):
+        from combine_moe_layout_06_b200 import capi
+        e, sb, G, cfgs = b.ep, self.sb, self.G, self.ep_cfgs
+
+        def sh(t, g):
+            return t[int(sb[g]):int(sb[g + 1])]
+
+        def local(g):
+            capi.moe_layout(cfgs[g], sh(b.topk, g), e.lays[g].struct)
+            e.counts_all[g].copy_(e.lays[g].expert_counts)   # the count all-gather
+
+        def send(g):
+            capi.moe_ep_layout(cfgs[g], g, G, sh(b.topk, g), e.counts_all, e.lays[g].struct,
+                               e.structs[g])
+            capi.moe_ep_dispatch(cfgs[g], e.lays[g].struct, e.structs[g], sh(b.x, g),
+                                 e.recv_bufs, e.cap)
+
+        def gather(g):
+            capi.moe_ep_combine(cfgs[g], e.lays[g].struct, e.structs[g], e.eo_bufs, e.cap,
+                                sh(b.w, g), sh(b.y, g))
+
+        self.ep_phase(local)
+        self.ep_phase(send)
+        self.ep_phase(gather)
+
+    def agrs_step(self, b):
+        from combine_moe_layout_06_b200 import capi
+        self.layout(b)
+        capi.moe_dispatch_allgather(self.cfg, b.lay.struct, b.x, b.gathered, b.recv)
+        capi.moe_combine_reducescatter(self.cfg, b.lay.struct, b.eo, b.w, b.partial, b.y)
+
+    # ---- running and timing
+    def layouts(self):
+        for b in self.sets:
+            yield b.lay
+            if self.with_decoupled:
+                yield b.dlay
+            if self.with_ep:
+                yield from b.ep.lays
+
+    def check_errors(self, where):
+        from combine_moe_layout_06_b200 import capi
+        for lay in self.layouts():
+            st = capi.moe_get_error(lay.struct)
+            if st != capi.MOE_OK:
+                raise SystemExit(f"device error {where} ({self.wl.name}): {capi.moe_status_string(st)}")
+
+    def prepare(self, warmup):
+        """Warm-up steps of every path, then the CUDA graphs: GRAPH_STEPS steps
+        alternating the two sets, a pair and a single step for the remainder
+        of K, for the step and its stage prefixes.  Programmatic dependent
+        launch overlaps consecutive kernels inside a graph but not across two
+        replays, so longer graphs measure the steady state a model-level graph
+        sees (one replay boundary costs about 2 us)."""
+        import torch
+        paths = [self.step]
+        if self.with_decoupled:
+            paths.append(self.decoupled_step)
+        if self.with_agrs:
+            paths.append(self.agrs_step)
+        if self.with_fp8:
+            paths.append(self.fp8_step)
+        if self.with_ep:
+            paths.append(self.ep_step)
+        for i in range(warmup):
+            for fn in paths:
+                fn(self.sets[i % 2])
+        torch.cuda.synchronize()
+        self.check_errors("after warm-up")
+        side = torch.cuda.Stream(self.ctx.dev)
+
+        def capture(fn, n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                for i in range(n):
+                    fn(self.sets[i % 2])
+            return g
+
+        def graph_set(fn):
+            return capture(fn, GRAPH_STEPS), capture(fn, 2), capture(fn, 1)
+
+        self.graphs = {"step": graph_set(self.step), "L": graph_set(self.layout),
+                       "LD": graph_set(self.layout_dispatch)}
+        if self.with_decoupled:
+            self.graphs["decoupled"] = graph_set(self.decoupled_step)
+        if self.with_agrs:
+            self.graphs["agrs"] = graph_set(self.agrs_step)
+        if self.with_fp8:
+            self.graphs["fp8"] = graph_set(self.fp8_step)
+            self.graphs["fp8_LD"] = graph_set(self.fp8_layout_dispatch)
+        if self.with_ep:
+            self.graphs["ep"] = graph_set(self.ep_step)
+        for gs in self.graphs.values():
+            for g in gs:
+                g.replay()
+        torch.cuda.synchronize()
+
+    def timed(self, name, K):
+        """K steps back to back between two events on the stream (ms, max
+        over ranks)."""
+        import torch
+        multi, pair, single = self.graphs[name]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        self.ctx.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K // GRAPH_STEPS):
+            multi.replay()
+        rest = K % GRAPH_STEPS
+        for _ in range(rest // 2):
+            pair.replay()
+        if rest % 2:
+            single.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        self.ctx.barrier()
+        return max_over_ranks(e0.elapsed_time(e1), self.ctx.world, self.ctx.dev)
+
+    def flushed_steps(self, K):
+        """One step at a time after writing a scratch buffer of twice the L2
+        outside the timed region (the cold variant of the back-to-back
+        measurement); per-step times, median and mean."""
+        import torch
+        dev, world = self.ctx.dev, self.ctx.world
+        scratch = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4,
+                              dtype=torch.float32, device=dev)
+        single = self.graphs["step"][2]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        self.ctx.barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            scratch.fill_(1.0)
+            e0.record()
+            single.replay()
+            e1.record()
+        torch.cuda.synchronize()
+        self.ctx.barrier()
+        ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
+        return {"median_ms": round(max_over_ranks(statistics.median(ts), world, dev), 5),
+                "mean_ms": round(max_over_ranks(statistics.fmean(ts), world, dev), 5),
+                "steps": K, "flush_bytes": scratch.numel() * 4}
+
+    def measure(self, K, flushed=True):
+        """Every timed loop of this workload, under one clock sampler."""
+        raw = {}
+        with ClockSampler(self.ctx.local) as clocks:
+            raw["step"] = self.timed("step", K)
+            raw["L"] = self.timed("L", K) / K
+            raw["LD"] = self.timed("LD", K) / K
+            for name in ("decoupled", "agrs", "fp8", "ep"):
+                if name in self.graphs:
+                    raw[name] = self.timed(name, K)
+            if "fp8_LD" in self.graphs:
+                raw["fp8_LD"] = self.timed("fp8_LD", K) / K
+            if flushed:
+                raw["flushed"] = self.flushed_steps(K)
+        raw["clocks"] = clocks.summary()
+        self.check_errors("in the timed region")
+        return raw
+
+    def report(self, raw, K):
+        """The line's entries for this workload (headline or per-workload)."""
+        import torch
+        wl, world = self.wl, self.ctx.world
+        total_ms = raw["step"]
+        ms_per_step = total_ms / K
+        t_l, t_ld = raw["L"], raw["LD"]
+        # Stage costs by subtraction.  With the count + assign/dispatch pair
+        # the assignment runs inside the dispatch kernel: the pair's whole
+        # cost counts as dispatch (the layout alone, moe_layout's kernels, is
+        # reported beside it).
+        if self.ld_pair:
+            t_layout, t_dispatch, t_combine = 0.0, t_ld, ms_per_step - t_ld
+        else:
+            t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
+        disp_b, comb_b = algorithmic_bytes(wl)
+        step_bytes = disp_b + comb_b
+        value = job_gbs(step_bytes, world, K, total_ms * 1e-3)
+        peak, peak_src = measured_peak()
+        dom = "dispatch" if t_dispatch >= t_combine else "combine"
+        dom_kernel = "layout_dispatch" if dom == "dispatch" and self.ld_pair else dom
+        dom_bytes = disp_b if dom == "dispatch" else comb_b
+        dom_ms = t_dispatch if dom == "dispatch" else t_combine
+        achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+        l2 = torch.cuda.get_device_properties(self.ctx.dev).L2_cache_size
+        out = {
+            "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(ms_per_step, 5),
+            "config": dict(
+                workload_desc(wl),
+                l2=("inputs larger than L2: steps alternate between two independent buffer "
+                    "sets, each step moves %.1f MB (%.2fx L2)" % (step_bytes / 1e6, step_bytes / l2)),
+                engine=self.args.engine,
+                layout=("count kernel + assign/dispatch kernel" if self.ld_pair
+                        else "one cluster launch" if self.cluster_layout else
+                        ("count + assign kernels" if self.small_layout else "count/scan/assign kernels")),
+                two_level_dispatch=(None if not wl.two_level else
+                                    "node pack + node expansion" if self.two_kernels else
+                                    "one kernel (staging rows read back from L2)"),
+                entry="moe_layout + moe_dispatch" if self.args.unfused else "moe_layout_dispatch",
+                timing=f"K steps back to back (CUDA graphs of {GRAPH_STEPS} steps) between two CUDA "
+                       "events on the launching stream; stage costs from graphs of layout, "
+                       "layout+dispatch and the full step"),
+            "pct_of_peak": round(100 * value / world / peak, 2),
+            "peak_gbs": peak, "peak_source": peak_src,
+            "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+            "tokens_per_s": round(wl.T * world * K / (total_ms * 1e-3), 1),
+            "tokens_per_s_dispatch_combine": round(wl.T * world / ((t_dispatch + t_combine) * 1e-3), 1),
+            "dispatch_combine_only_gbs": round(step_bytes / ((t_dispatch + t_combine) * 1e-3) / 1e9, 2),
+            "kernels_ms": ({"layout_dispatch": round(t_dispatch, 5), "combine": round(t_combine, 5),
+                            "layout_kernels_alone": round(t_l, 5)} if self.ld_pair else
+                           {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
+                            "combine": round(t_combine, 5)}),
+            "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 2),
+                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": profiled_traffic(dom_kernel, wl.name if wl.T == inputs.WORKLOADS[wl.name].T
+                                                     else "none"),
+                         "peak_kind": f"{peak_src} copy bandwidth"},
+            "clocks": raw["clocks"],
+            "step_bytes": step_bytes,
+        }
+        if "flushed" in raw:
+            out["flushed_step"] = raw["flushed"]
+        if "decoupled" in raw:
+            dec_value = job_gbs(step_bytes, world, K, raw["decoupled"] * 1e-3)
+            out["decoupled_3pass"] = {
+                "value": round(dec_value, 2), "unit": "GB/s",
+                "ms_per_step": round(raw["decoupled"] / K, 5),
+                "fused_speedup": round(value / dec_value, 3),
+                "path": "layout (per-rank groups) + pack/copy/unpack dispatch + pack/copy/unpack combine"}
+        if "agrs" in raw:
+            ag_value = job_gbs(step_bytes, world, K, raw["agrs"] * 1e-3)
+            out["allgather_reducescatter"] = {
+                "value": round(ag_value, 2), "unit": "GB/s", "ms_per_step": round(raw["agrs"] / K, 5),
+                "fused_speedup": round(value / ag_value, 3),
+                "path": "layout + all-gather dispatch (R copies, per-rank select) + "
+                        "reduce-scatter combine (per-rank fp32 partials, rank-order sum)"}
+        if "fp8" in raw:
+            fp8_ms = raw["fp8"]
+            fp8_bytes = 2 * (wl.T * wl.H * 2 + wl.T * wl.k * (wl.H + 4))
+            out["fp8_payload"] = {
+                "value": round(job_gbs(fp8_bytes, world, K, fp8_ms * 1e-3), 2), "unit": "GB/s",
+                "ms_per_step": round(fp8_ms / K, 5),
+                "tokens_per_s": round(wl.T * world * K / (fp8_ms * 1e-3), 1),
+                "speedup_vs_bf16_step": round(total_ms / fp8_ms, 3),
+                "kernels_ms": {"dispatch": round(raw["fp8_LD"] - t_l, 5),
+                               "combine": round(fp8_ms / K - raw["fp8_LD"], 5)},
+                "bytes_per_step": fp8_bytes,
+                "path": ("layout + fp8 two-level dispatch (quantize once into node staging, "
+                         "expand codes and scales; staging not credited) + " if wl.two_level else
+                         "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + ")
+                        + "fp8 combine (expert rows already e4m3)"}
+        if "ep" in raw:
+            ep_value = job_gbs(step_bytes, world, K, raw["ep"] * 1e-3)
+            out["expert_parallel_virtual_ranks"] = {
+                "value": round(ep_value, 2), "unit": "GB/s", "ms_per_step": round(raw["ep"] / K, 5),
+                "ranks": self.G, "vs_single_source": round(ep_value / value, 3),
+                "receive_rows": [int(r) for r in self.ep_rows],
+                "path": f"{self.G} source ranks on this GPU, one stream each, joined between "
+                        "phases: layout of its shard and the count all-gather (device copies); "
+                        "sharded-source layout and dispatch into every rank's receive buffer; "
+                        "combine from every rank's expert outputs (pointer tables)"}
+        return out
+
+    def e2e(self, steps):
+        """End to end through the C ABI from pinned host buffers, pipelined
+        over the two buffer sets: step i's inputs go up on a copy stream
+        while step i-1 computes, and step i's result comes down on another
+        copy stream while step i+1 computes.  Every step still copies all its
+        inputs in and its result out; the events only order each set's
+        reuse.  Returns the entry of the line (wall clock, max over ranks)."""
+        import torch
+
+        from combine_moe_layout_06_b200 import capi
+        d, wl, dev, world = self.d, self.wl, self.ctx.dev, self.ctx.world
+        x_h = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        topk_h = torch.from_numpy(d["topk_idx"]).pin_memory()
+        w_h = torch.from_numpy(d["topk_w"]).pin_memory()
+        y_h = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in self.sets]
+        h2d = x_h.numel() * 2 + topk_h.numel() * 4 + w_h.numel() * 4
+        d2h = y_h[0].numel() * 2
+        s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        inputs_up = [torch.cuda.Event() for _ in self.sets]
+        computed = [torch.cuda.Event() for _ in self.sets]
+        result_down = [torch.cuda.Event() for _ in self.sets]
+
+        def run(compute: bool) -> float:
+            torch.cuda.synchronize()
+            self.ctx.barrier()
+            t0 = time.perf_counter()
+            for i in range(steps):
+                j = i % 2
+                b = self.sets[j]
+                if i >= 2:
+                    s_in.wait_event(computed[j])        # step i-2 has read this set's inputs
+                with torch.cuda.stream(s_in):
+                    b.x.copy_(x_h, non_blocking=True)
+                    b.topk.copy_(topk_h, non_blocking=True)
+                    b.w.copy_(w_h, non_blocking=True)
+                    inputs_up[j].record(s_in)
+                s_comp.wait_event(inputs_up[j])
+                if i >= 2:
+                    s_comp.wait_event(result_down[j])   # step i-2's result has left this set's y
+                with torch.cuda.stream(s_comp):
+                    if compute:
+                        capi.moe_layout_dispatch(self.cfg, b.topk, b.lay.struct, b.x, b.recv,
+                                                 b.staging)
+                        capi.moe_combine(self.cfg, b.lay.struct, b.recv, b.w, b.y)  # identity expert
+                    computed[j].record(s_comp)
+                s_out.wait_event(computed[j])
+                with torch.cuda.stream(s_out):
+                    y_h[j].copy_(b.y, non_blocking=True)
+                    result_down[j].record(s_out)
+            for s_ in (s_in, s_comp, s_out):
+                s_.synchronize()
+            return max_over_ranks(time.perf_counter() - t0, world, dev)
+
+        copies_s = run(False)
+        e2e_s = run(True)
+        step_bytes = sum(algorithmic_bytes(wl))
+        return {"value": round(job_gbs(step_bytes, world, steps, e2e_s), 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+                "copies_only_value": round(job_gbs(step_bytes, world, steps, copies_s), 3),
+                "mode": "moe_layout_dispatch + moe_combine per step, host copies pipelined "
+                        "on two copy streams over two buffer sets (wall clock)"}
+
+    def release(self):
+        import torch
+        self.graphs.clear()
+        self.sets = []
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def cpu_baselines(d, eo_bits, seconds):
+    """The oracle as it stands on the host: single thread, then its OpenMP
+    dispatch/combine variants on all host threads (full workload)."""
+    import oracle
+    wl = d["workload"]
+    step_bytes = sum(algorithmic_bytes(wl))
+    one = oracle_step_time(d, wl.T, 1, eo_bits)
+    reps = max(1, min(30, int(seconds / max(one, 1e-3))))
+    best = min(one, oracle_step_time(d, wl.T, reps, eo_bits))
+    cpu = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": 1,
+           "kind": "oracle",
+           "sample": f"full workload ({wl.T} tokens: layout+dispatch+combine), best of "
+                     f"{reps + 1} runs, single thread on {os.cpu_count()} host cores",
+           "cpu_model": cpu_model()}
+    threads = oracle.parallel_threads()
+    one = oracle_step_time(d, wl.T, 1, eo_bits, parallel=True)
+    reps = max(1, min(30, int(seconds / 2 / max(one, 1e-3))))
+    best = min(one, oracle_step_time(d, wl.T, reps, eo_bits, parallel=True))
+    cpu_par = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": threads,
+               "kind": "oracle, dispatch and combine token loops over OpenMP threads "
+                       "(layout serial)",
+               "sample": f"full workload ({wl.T} tokens), best of {reps + 1} runs"}
+    return cpu, cpu_par
+
+
+# ---------------------------------------------------------------- several GPUs
+
+def ep_plan(local_counts, num_ranks, group=None, out=None):
+    """Host side of the sharded-source set-up on every rank: all-gather the
+    per-expert counts (source-rank order), then the rows each expert rank
+    receives (the library's moe_ep_receive_rows) and the buffer capacity
+    every rank allocates (the largest).  Returns (counts_all, rows, cap)."""
+    from combine_moe_layout_06_b200 import capi
+    from combine_moe_layout_06_b200 import ep as epmod
+    counts_all = epmod.gather_counts(local_counts, group, out=out)
+    rows = capi.moe_ep_receive_rows(counts_all.cpu().numpy(), num_ranks)
+    return counts_all, rows, max(max(rows), 1)
+
+
+def ep_shuffle(args, ctx, d):
+    """Expert parallelism over sharded sources across the processes (one
+    rank per GPU, NCCL process group): see the module docstring."""
+    import torch
+    import torch.distributed as dist
+
+    from combine_moe_layout_06_b200 import buffers, capi
+    from combine_moe_layout_06_b200 import ep as epmod
+    wl = d["workload"]
+    G, g, dev = ctx.world, ctx.rank, ctx.dev
+    cfg = capi.config(wl.T, wl.H, wl.E, wl.k, G, 1, engine_flags(args))
+    me = epmod.ExpertParallelRank(cfg, g, G, dev)
+    bf16 = dict(dtype=torch.bfloat16, device=dev)
+    topk = torch.from_numpy(d["topk_idx"]).to(dev)
+    x = buffers.bf16_from_bits(d["x"], dev)
+    w = torch.from_numpy(d["topk_w"]).to(dev)
+    y = torch.empty((wl.T, wl.H), **bf16)
+    counts_all = torch.zeros((G, wl.E), dtype=torch.int32, device=dev)
+    # set-up: one layout and count exchange sizes every rank's buffers
+    capi.moe_layout(cfg, topk, me.local.struct)
+    _, rows, cap = ep_plan(me.local.expert_counts, G, out=counts_all)
+    recv = torch.empty((cap, wl.H), **bf16)
+    eo = torch.empty((cap, wl.H), **bf16)
+    recv_peers = epmod.share_buffer(recv)
+    eo_peers = epmod.share_buffer(eo)
+    recv_ptrs = [p for p, _ in recv_peers]
+    eo_ptrs = [p for p, _ in eo_peers]
+    fence_word = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def fence():
+        # every rank's work enqueued so far is complete before any rank's
+        # later work starts (stream-ordered: an NCCL all-reduce of one word)
+        dist.all_reduce(fence_word)
+
+    def step(xb, topkb, wb, yb):
+        capi.moe_layout(cfg, topkb, me.local.struct)
+        epmod.gather_counts(me.local.expert_counts, out=counts_all)
+        capi.moe_ep_layout(cfg, g, G, topkb, counts_all, me.local.struct, me.ep)
+        capi.moe_ep_dispatch(cfg, me.local.struct, me.ep, xb, recv_ptrs, cap)
+        fence()    # every row has landed: the experts would run here
+        capi.moe_ep_combine(cfg, me.local.struct, me.ep, eo_ptrs, cap, wb, yb)
+        fence()    # no rank's next dispatch overwrites rows a peer still reads
+
+    # stand-in expert outputs: the received rows themselves (identity expert)
+    step(x, topk, w, y)
+    torch.cuda.synchronize()
+    eo.copy_(recv)
+    fence()
+    for _ in range(args.warmup):
+        step(x, topk, w, y)
+    torch.cuda.synchronize()
+    st = capi.moe_get_error(me.local.struct)
+    if st != capi.MOE_OK:
+        raise SystemExit(f"device error in the expert-parallel warm-up: {capi.moe_status_string(st)}")
+    K = args.steps
+    with ClockSampler(ctx.local) as clocks:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ctx.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(K):
+            step(x, topk, w, y)
+        e1.record()
+        torch.cuda.synchronize()
+        ctx.barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1), G, dev)
+    st = capi.moe_get_error(me.local.struct)
+    if st != capi.MOE_OK:
+        raise SystemExit(f"device error in the expert-parallel run: {capi.moe_status_string(st)}")
+
+    # end to end: this rank's inputs up from pinned host memory, the step,
+    # its output down, every step (wall clock, max over ranks)
+    steps_e2e = args.e2e_steps or min(K, 20)
+    x_h = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    topk_h = torch.from_numpy(d["topk_idx"]).pin_memory()
+    w_h = torch.from_numpy(d["topk_w"]).pin_memory()
+    y_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x2, topk2, w2 = torch.empty_like(x), torch.empty_like(topk), torch.empty_like(w)
+    torch.cuda.synchronize()
+    ctx.barrier()
+    t0 = time.perf_counter()
+    for _ in range(steps_e2e):
+        x2.copy_(x_h, non_blocking=True)
+        topk2.copy_(topk_h, non_blocking=True)
+        w2.copy_(w_h, non_blocking=True)
+        step(x2, topk2, w2, y)
+        y_h.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_s = max_over_ranks(time.perf_counter() - t0, G, dev)
+    step_bytes = sum(algorithmic_bytes(wl))
+    out = {
+        "value": round(job_gbs(step_bytes, G, K, ms * 1e-3), 2), "ms_per_step": round(ms / K, 5),
+        "receive_rows": [int(r) for r in rows], "capacity_rows": int(cap),
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(job_gbs(step_bytes, G, steps_e2e, e2e_s), 3), "unit": "GB/s",
+                "h2d_bytes_per_step": x_h.numel() * 2 + topk_h.numel() * 4 + w_h.numel() * 4,
+                "d2h_bytes_per_step": y_h.numel() * 2, "steps": steps_e2e,
+                "mode": "per rank: host copies of its inputs, the expert-parallel step, its "
+                        "output back (wall clock, max over ranks)"},
+        "launches_per_step": 5,
+    }
+    # unmap the peers' buffers only once no rank still writes to them
+    torch.cuda.synchronize()
+    ctx.barrier()
+    del recv_peers, eo_peers, recv_ptrs, eo_ptrs
+    torch.cuda.synchronize()
+    ctx.barrier()
+    return out
+
+
+def run_several(args, ctx):
+    import torch
+    d = workload_inputs(args.workload, args.tokens, source=ctx.rank)
+    wl = d["workload"]
+    shuffle = ep_shuffle(args, ctx, d)
+    torch.cuda.empty_cache()
+    replicas = StepBench(ctx, args, d)
+    replicas.prepare(args.warmup)
+    rep = replicas.report(replicas.measure(args.steps, flushed=False), args.steps)
+    replicas.release()
+    if ctx.rank == 0:
+        K = args.steps
+        line = {
+            "metric": METRIC, "value": shuffle["value"], "unit": "GB/s", "n_gpus": ctx.world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": shuffle["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_desc(wl),
+                           dispatch_mode="flat, one expert rank per GPU (sharded sources)",
+                           parallelism=f"expert parallelism over {ctx.world} processes, one rank "
+                                       "per GPU, every rank routing a batch of its own",
+                           l2="inputs larger than L2: each rank's step moves %.0f MB"
+                              % (sum(algorithmic_bytes(wl)) / 1e6),
+                           timing="K eager steps between two CUDA events on the launching stream, "
+                                  "max over ranks"),
+            "tokens_per_s": round(wl.T * ctx.world * K / (shuffle["ms_per_step"] * K * 1e-3), 1),
+            "expert_parallel": {k: v for k, v in shuffle.items() if k not in ("e2e", "clocks")},
+            "replicas": {k: rep[k] for k in ("value", "ms_per_step", "kernels_ms", "roofline",
+                                             "pct_of_peak", "config")},
+            "clocks": shuffle["clocks"],
+            "e2e": shuffle["e2e"],
+            "gpu_launches": shuffle["launches_per_step"] * K,
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- one GPU
+
+def run_one(args, ctx):
+    import torch
+    d = workload_inputs(args.workload, args.tokens)
+    wl = d["workload"]
+    K = args.steps
+    main = StepBench(ctx, args, d, extras=[e for e, off in (
+        ("decoupled", args.no_decoupled), ("agrs", args.no_agrs), ("fp8", args.no_fp8),
+        ("ep", args.no_ep)) if not off])
+    main.prepare(args.warmup)
+    head = main.report(main.measure(K), K)
+    e2e = main.e2e(args.e2e_steps or min(K, 50))
+    launches = main.launches_per_step * K
+    eo_bits = main.eo_bits
+    main.release()
+    del main
+
+    balance = None
+    if not args.no_node_balance:
+        with ClockSampler(ctx.local) as nb_clocks:
+            balance = node_balance(args, ctx)
+        balance["clocks"] = nb_clocks.summary()
+        torch.cuda.empty_cache()
+
+    per = {}
+    names = [] if args.no_per_workload else [n for n in (args.per_workload.split(",")
+                                                         if args.per_workload else WORKLOAD_ORDER)
+                                             if n and n != args.workload]
+    for name in names:
+        pd = workload_inputs(name)
+        sb = StepBench(ctx, args, pd, extras=[] if args.no_decoupled else ["decoupled"])
+        sb.prepare(args.warmup)
+        per[name] = sb.report(sb.measure(K, flushed=False), K)
+        sb.release()
+        del sb
+
+    cpu = cpu_par = None
+    if ctx.rank == 0 and not args.no_cpu_baseline:
+        cpu, cpu_par = cpu_baselines(d, eo_bits, args.cpu_seconds)
+
+    line = {"metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": ctx.world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic"}
+    head["config"]["parallelism"] = "single GPU"
+    for key, val in head.items():
+        if key not in ("value", "unit", "ms_per_step"):
+            line[key] = val
+    line.update({
+        "node_balance": balance,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+        "cpu_baseline_parallel": cpu_par,
+        "per_workload": per or None,
+    })
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="olmoe", choices=sorted(inputs.WORKLOADS))
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    p.add_argument("--tokens", type=int, default=0,
+                   help="time only the first T tokens of the workload (a scaled-down case of "
+                        "the same shape and routing, e.g. for ncu captures)")
+    p.add_argument("--per-workload", default="",
+                   help="comma-separated workloads for per_workload (default: every other one)")
+    p.add_argument("--no-per-workload", action="store_true")
     p.add_argument("--engine", default="auto", choices=["auto", "vector", "bulk"])
     p.add_argument("--layout", default="kernels", choices=["kernels", "fused", "cluster"],
                    help="kernels: layout kernels then the dispatch kernel; fused: a count kernel "
@@ -416,8 +1241,13 @@ def main():
     p.add_argument("--ref-tokens", type=int, default=0)
     p.add_argument("--hbm-probe", action="store_true",
                    help="measure write-only / read-only / copy HBM bandwidth and exit")
-    args = p.parse_args()
+    args = p.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    return args
+
+
+def main():
+    args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.hbm_probe:
@@ -426,504 +1256,19 @@ def main():
     import torch
     import torch.distributed as dist
 
-    from combine_moe_layout_06_b200 import buffers, capi
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    d = inputs.make(args.workload)
-    wl = d["workload"]
-    flags = capi.MOE_FLAG_TWO_LEVEL if wl.two_level else 0
-    flags |= {"auto": 0, "vector": capi.MOE_FLAG_COPY_VECTOR, "bulk": capi.MOE_FLAG_COPY_BULK}[args.engine]
-    if args.layout == "cluster":
-        flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
-    if args.layout == "fused":
-        flags |= capi.MOE_FLAG_LAYOUT_FUSED
-    if args.two_level_fused:
-        flags |= capi.MOE_FLAG_TWO_LEVEL_FUSED
-    cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
-    # the decoupled comparison path packs per rank: one "node" per rank
-    dcfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.R,
-                       capi.MOE_FLAG_TWO_LEVEL | (flags & (capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK)))
     dev = torch.device("cuda", local)
-    eo_bits = inputs.random_bf16_bits((wl.T * wl.k, wl.H), seed=wl.seed + 7)
-    bf16 = dict(dtype=torch.bfloat16, device=dev)
-
-    # Expert parallelism over sharded sources with every rank on this GPU:
-    # rank g routes tokens [sb[g], sb[g+1]); its receive and expert-output
-    # buffers are the rank's rows of the set's recv / eo (pointer tables).
-    G = wl.R
-    sb = (np.arange(G + 1, dtype=np.int64) * wl.T) // G
-    from combine_moe_layout_06_b200 import ep as epmod
-    shard_counts = np.stack([np.bincount(d["topk_idx"][sb[g]:sb[g + 1]].ravel(), minlength=wl.E)
-                             for g in range(G)])
-    ep_rows = epmod.receive_rows(shard_counts, wl.R)
-    ep_first = np.concatenate([[0], np.cumsum(ep_rows)])
-    ep_cfgs = [capi.config(int(sb[g + 1] - sb[g]), wl.H, wl.E, wl.k, wl.R, 1,
-                           flags & (capi.MOE_FLAG_COPY_VECTOR | capi.MOE_FLAG_COPY_BULK))
-               for g in range(G)]
-
-    class EpShards:
-        """Per-rank layouts and sharded-source arrays of one buffer set."""
-
-        def __init__(self, b):
-            i32 = dict(dtype=torch.int32, device=dev)
-            self.lays = [buffers.DeviceLayout(c, dev) for c in ep_cfgs]
-            self.counts_all = torch.zeros((G, wl.E), **i32)
-            self.arrays = [(torch.zeros(wl.E + 1, **i32), torch.zeros(wl.R + 1, **i32),
-                            torch.zeros(max(c.num_tokens * wl.k, 1), **i32)) for c in ep_cfgs]
-            self.structs = [capi.ep_layout_struct(*a) for a in self.arrays]
-            row = wl.H * 2
-            self.recv_bufs = [b.recv.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
-            self.eo_bufs = [b.eo.data_ptr() + int(ep_first[r]) * row for r in range(wl.R)]
-            self.cap = int(ep_rows.max())
-
-    class BufferSet:
-        """One independent set of the step's inputs and outputs."""
-
-        def __init__(self, decoupled=False, agrs=False, fp8=False, ep=False):
-            self.lay = buffers.DeviceLayout(cfg, dev)
-            self.x = buffers.bf16_from_bits(d["x"], dev)
-            self.topk = torch.from_numpy(d["topk_idx"]).to(dev)
-            self.w = torch.from_numpy(d["topk_w"]).to(dev)
-            self.eo = buffers.bf16_from_bits(eo_bits, dev)
-            self.recv = torch.empty((wl.T * wl.k, wl.H), **bf16)
-            self.y = torch.empty((wl.T, wl.H), **bf16)
-            self.staging = None
-            if wl.two_level:
-                self.staging = torch.empty((capi.moe_node_staging_rows(cfg), wl.H), **bf16)
-            if decoupled:
-                self.dlay = buffers.DeviceLayout(dcfg, dev)
-                rows = capi.moe_node_staging_rows(dcfg)
-                self.dsend = torch.empty((rows, wl.H), **bf16)
-                self.dxfer = torch.empty((rows, wl.H), **bf16)
-                self.csend = torch.empty((wl.T * wl.k, wl.H), **bf16)
-                self.cxfer = torch.empty((wl.T * wl.k, wl.H), **bf16)
-            if fp8:
-                rows = wl.T * wl.k
-                self.recv_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
-                self.recv_s = torch.empty(rows, dtype=torch.float32, device=dev)
-                self.eo_q = torch.empty((rows, wl.H), dtype=torch.uint8, device=dev)
-                self.eo_s = torch.empty(rows, dtype=torch.float32, device=dev)
-                # expert outputs as an fp8 producer would emit them
-                capi.moe_quantize_rows_fp8(self.eo, rows, wl.H, self.eo_q, self.eo_s)
-                if wl.two_level:
-                    srows = capi.moe_node_staging_rows(cfg)
-                    self.st_q = torch.empty((srows, wl.H), dtype=torch.uint8, device=dev)
-                    self.st_s = torch.empty(srows, dtype=torch.float32, device=dev)
-            if agrs:
-                self.gathered = torch.empty((wl.R * wl.T, wl.H), **bf16)
-                self.partial = torch.empty((wl.R * wl.T, wl.H), dtype=torch.float32, device=dev)
-            self.ep = EpShards(self) if ep else None
-
-    with_decoupled = not args.no_decoupled
-    with_agrs = not args.no_agrs and wl.R <= capi.MOE_MAX_NODES
-    with_fp8 = not args.no_fp8 and wl.H % 8 == 0
-    with_ep = not args.no_ep and wl.R <= capi.MOE_MAX_NODES and not wl.two_level
-    sets = [BufferSet(with_decoupled, with_agrs, with_fp8, with_ep) for _ in range(2)]
-
-    def layout(b):
-        capi.moe_layout(cfg, b.topk, b.lay.struct)
-
-    def layout_dispatch(b):
-        if args.unfused:
-            layout(b)
-            capi.moe_dispatch(cfg, b.lay.struct, b.x, b.recv, b.staging)
-        else:
-            capi.moe_layout_dispatch(cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
-
-    def step(b):
-        layout_dispatch(b)
-        capi.moe_combine(cfg, b.lay.struct, b.eo, b.w, b.y)
-
-    def decoupled_step(b):
-        capi.moe_layout(dcfg, b.topk, b.dlay.struct)
-        capi.moe_dispatch_decoupled(dcfg, b.dlay.struct, b.x, b.dsend, b.dxfer, b.recv)
-        capi.moe_combine_decoupled(dcfg, b.dlay.struct, b.eo, b.w, b.csend, b.cxfer, b.y)
-
-    def fp8_layout_dispatch(b):
-        layout(b)
-        if wl.two_level:
-            capi.moe_dispatch_fp8_two_level(cfg, b.lay.struct, b.x, b.st_q, b.st_s, b.recv_q, b.recv_s)
-        else:
-            capi.moe_dispatch_fp8(cfg, b.lay.struct, b.x, b.recv_q, b.recv_s)
-
-    def fp8_step(b):
-        fp8_layout_dispatch(b)
-        capi.moe_combine_fp8(cfg, b.lay.struct, b.eo_q, b.eo_s, b.w, b.y)
-
-    ep_streams = [torch.cuda.Stream(dev) for _ in range(G)] if wl.R <= capi.MOE_MAX_NODES else []
-
-    def ep_phase(fn):
-        """Run fn(g) for every rank on its own stream, all after the work
-        enqueued so far and before anything enqueued later (the ranks of a
-        multi-GPU system run concurrently; the joins stand for its barriers)."""
-        cur = torch.cuda.current_stream()
-        for st in ep_streams:
-            st.wait_stream(cur)
-        for g, st in enumerate(ep_streams):
-            with torch.cuda.stream(st):
-                fn(g)
-        for st in ep_streams:
-            cur.wait_stream(st)
-
-    def ep_step(b):
-        e = b.ep
-        sh = lambda t, g: t[int(sb[g]):int(sb[g + 1])]
-
-        def local(g):
-            capi.moe_layout(ep_cfgs[g], sh(b.topk, g), e.lays[g].struct)
-            e.counts_all[g].copy_(e.lays[g].expert_counts)   # the count all-gather
-
-        def send(g):
-            capi.moe_ep_layout(ep_cfgs[g], g, G, sh(b.topk, g), e.counts_all, e.lays[g].struct,
-                               e.structs[g])
-            capi.moe_ep_dispatch(ep_cfgs[g], e.lays[g].struct, e.structs[g], sh(b.x, g),
-                                 e.recv_bufs, e.cap)
-
-        def gather(g):
-            capi.moe_ep_combine(ep_cfgs[g], e.lays[g].struct, e.structs[g], e.eo_bufs, e.cap,
-                                sh(b.w, g), sh(b.y, g))
-
-        ep_phase(local)
-        ep_phase(send)
-        ep_phase(gather)
-
-    def agrs_step(b):
-        layout(b)
-        capi.moe_dispatch_allgather(cfg, b.lay.struct, b.x, b.gathered, b.recv)
-        capi.moe_combine_reducescatter(cfg, b.lay.struct, b.eo, b.w, b.partial, b.y)
-
-    # one cluster launch when asked for, and always for one chunk of 256 tokens
-    cluster_layout = (args.layout == "cluster" and wl.T <= 131072) or wl.T <= 256
-    small_layout = wl.T <= 256 * 256      # count + assign (scan folded in)
-    layout_launches = 1 if cluster_layout else (2 if small_layout else 3)
-    # moe_layout_dispatch as the count + assign/dispatch pair (the library's
-    # rule: flat, 16-byte rows, at most 256 experts, no engine or layout
-    # override)
-    ld_pair = (not args.unfused and not wl.two_level and args.layout == "fused"
-               and (wl.H * 2) % 16 == 0 and wl.E <= 256)
-    # two-level: pack + expand, or one kernel with --two-level-fused (16-byte rows, N + k <= 32)
-    two_kernels = wl.two_level and (not args.two_level_fused or args.engine == "vector"
-                                    or (wl.H * 2) % 16 or wl.N + wl.k > 32)
-    launches_per_step = (2 if ld_pair else layout_launches + (2 if two_kernels else 1)) + 1
-
-    for i in range(args.warmup):
-        step(sets[i % 2])
-        if with_decoupled:
-            decoupled_step(sets[i % 2])
-        if with_agrs:
-            agrs_step(sets[i % 2])
-        if with_fp8:
-            fp8_step(sets[i % 2])
-        if with_ep:
-            ep_step(sets[i % 2])
-    torch.cuda.synchronize()
-    for b in sets:
-        for lay in [b.lay] + ([b.dlay] if with_decoupled else []) + (b.ep.lays if with_ep else []):
-            st = capi.moe_get_error(lay.struct)
-            if st != capi.MOE_OK:
-                raise SystemExit(f"device error after warm-up: {capi.moe_status_string(st)}")
-
-    # CUDA graphs over the two buffer sets: GRAPH_STEPS steps alternating A
-    # and B, a pair (A then B) and a single step for the remainder of K; stage
-    # prefixes for the breakdown.  Programmatic dependent launch overlaps
-    # consecutive kernels inside a graph but not across two replays, so longer
-    # graphs measure the steady state a model-level graph sees (one replay
-    # boundary costs about 2 us).
-    side = torch.cuda.Stream(dev)
-
-    def capture(fn, n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=side):
-            for i in range(n):
-                fn(sets[i % 2])
-        return g
-
-    def graph_set(fn):
-        return capture(fn, GRAPH_STEPS), capture(fn, 2), capture(fn, 1)
-
-    graphs = {"step": graph_set(step), "L": graph_set(layout), "LD": graph_set(layout_dispatch)}
-    if with_decoupled:
-        graphs["decoupled"] = graph_set(decoupled_step)
-    if with_agrs:
-        graphs["agrs"] = graph_set(agrs_step)
-    if with_fp8:
-        graphs["fp8"] = graph_set(fp8_step)
-        graphs["fp8_LD"] = graph_set(fp8_layout_dispatch)
-    if with_ep:
-        graphs["ep"] = graph_set(ep_step)
-    for gs in graphs.values():
-        for g in gs:
-            g.replay()
-    torch.cuda.synchronize()
-
-    def timed(name, K):
-        """K steps back to back between two events on the stream (ms)."""
-        multi, pair, single = graphs[name]
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(K // GRAPH_STEPS):
-            multi.replay()
-        rest = K % GRAPH_STEPS
-        for _ in range(rest // 2):
-            pair.replay()
-        if rest % 2:
-            single.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        barrier()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev)
-
-    # One step at a time after writing a scratch buffer of twice the L2
-    # outside the timed region (the cold variant of the back-to-back
-    # measurement); per-step times, median and mean.
-    scratch = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4,
-                          dtype=torch.float32, device=dev)
-
-    def flushed_steps(K):
-        single = graphs["step"][2]
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
-        barrier()
-        torch.cuda.synchronize()
-        for e0, e1 in evs:
-            scratch.fill_(1.0)
-            e0.record()
-            single.replay()
-            e1.record()
-        torch.cuda.synchronize()
-        barrier()
-        ts = sorted(e0.elapsed_time(e1) for e0, e1 in evs)
-        return {"median_ms": round(max_over_ranks(statistics.median(ts), world, dev), 5),
-                "mean_ms": round(max_over_ranks(statistics.fmean(ts), world, dev), 5),
-                "steps": K, "flush_bytes": scratch.numel() * 4}
-
-    K = args.steps
-    with ClockSampler(local) as clocks:
-        total_ms = timed("step", K)
-        t_l = timed("L", K) / K
-        t_ld = timed("LD", K) / K
-        dec_ms = timed("decoupled", K) if with_decoupled else None
-        agrs_ms = timed("agrs", K) if with_agrs else None
-        fp8_ms = timed("fp8", K) if with_fp8 else None
-        fp8_ld = timed("fp8_LD", K) / K if with_fp8 else None
-        ep_ms = timed("ep", K) if with_ep else None
-        flushed = flushed_steps(K)
-    ms_per_step = total_ms / K
-    # Stage costs by subtraction.  With the count + assign/dispatch pair the
-    # assignment runs inside the dispatch kernel: the pair's whole cost
-    # counts as dispatch (the layout alone, moe_layout's kernels, is reported
-    # beside it).
-    if ld_pair:
-        t_layout, t_dispatch, t_combine = 0.0, t_ld, ms_per_step - t_ld
-    else:
-        t_layout, t_dispatch, t_combine = t_l, t_ld - t_l, ms_per_step - t_ld
-    for b in sets:
-        st = capi.moe_get_error(b.lay.struct)
-        if st != capi.MOE_OK:
-            raise SystemExit(f"device error in the timed region: {capi.moe_status_string(st)}")
-
-    disp_b, comb_b = algorithmic_bytes(wl)
-    step_bytes = disp_b + comb_b
-    value = job_gbs(step_bytes, world, K, total_ms * 1e-3)
-    peak, peak_src = measured_peak()
-    dom = "dispatch" if t_dispatch >= t_combine else "combine"
-    dom_kernel = "layout_dispatch" if dom == "dispatch" and ld_pair else dom
-    dom_bytes = disp_b if dom == "dispatch" else comb_b
-    dom_ms = t_dispatch if dom == "dispatch" else t_combine
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    decoupled = None
-    if dec_ms is not None:
-        dec_value = job_gbs(step_bytes, world, K, dec_ms * 1e-3)
-        decoupled = {"value": round(dec_value, 2), "unit": "GB/s",
-                     "ms_per_step": round(dec_ms / K, 5),
-                     "fused_speedup": round(value / dec_value, 3),
-                     "path": "layout (per-rank groups) + pack/copy/unpack dispatch + "
-                             "pack/copy/unpack combine"}
-
-    agrs = None
-    if agrs_ms is not None:
-        ag_value = job_gbs(step_bytes, world, K, agrs_ms * 1e-3)
-        agrs = {"value": round(ag_value, 2), "unit": "GB/s", "ms_per_step": round(agrs_ms / K, 5),
-                "fused_speedup": round(value / ag_value, 3),
-                "path": "layout + all-gather dispatch (R copies, per-rank select) + "
-                        "reduce-scatter combine (per-rank fp32 partials, rank-order sum)"}
-
-    fp8 = None
-    if fp8_ms is not None:
-        fp8_bytes = 2 * (wl.T * wl.H * 2 + wl.T * wl.k * (wl.H + 4))
-        fp8 = {"value": round(job_gbs(fp8_bytes, world, K, fp8_ms * 1e-3), 2), "unit": "GB/s",
-               "ms_per_step": round(fp8_ms / K, 5),
-               "tokens_per_s": round(wl.T * world * K / (fp8_ms * 1e-3), 1),
-               "speedup_vs_bf16_step": round(total_ms / fp8_ms, 3),
-               "kernels_ms": {"dispatch": round(fp8_ld - t_l, 5),  # fp8 path: layout kernels + dispatch
-                              "combine": round(fp8_ms / K - fp8_ld, 5)},
-               "bytes_per_step": fp8_bytes,
-               "path": ("layout + fp8 two-level dispatch (quantize once into node staging, "
-                        "expand codes and scales; staging not credited) + " if wl.two_level else
-                        "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + ")
-                       + "fp8 combine (expert rows already e4m3)"}
-
-    graphs.clear()
-    balance = None
-    if not args.no_node_balance:
-        with ClockSampler(local) as nb_clocks:
-            balance = node_balance(args, dev, world, barrier, flags)
-        balance["clocks"] = nb_clocks.summary()
-
-    ep_line = None
-    if ep_ms is not None:
-        for b in sets:
-            for lay in b.ep.lays:
-                st = capi.moe_get_error(lay.struct)
-                if st != capi.MOE_OK:
-                    raise SystemExit(f"device error in the sharded-source run: {capi.moe_status_string(st)}")
-        ep_value = job_gbs(step_bytes, world, K, ep_ms * 1e-3)
-        ep_line = {"value": round(ep_value, 2), "unit": "GB/s", "ms_per_step": round(ep_ms / K, 5),
-                   "ranks": G, "vs_single_source": round(ep_value / value, 3),
-                   "receive_rows": [int(r) for r in ep_rows],
-                   "path": f"{G} source ranks on this GPU, one stream each, joined between "
-                           "phases: layout of its shard and the count all-gather (device copies); "
-                           "sharded-source layout and dispatch into every rank's receive buffer; "
-                           "combine from every rank's expert outputs (pointer tables)"}
-
-    # End to end through the C ABI from pinned host buffers, pipelined over
-    # the two buffer sets: step i's inputs go up on a copy stream while step
-    # i-1 computes, and step i's result comes down on another copy stream
-    # while step i+1 computes.  Every step still copies all its inputs in and
-    # its result out; the events only order each set's reuse.
-    e2e_steps = args.e2e_steps or min(K, 50)
-    x_h = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
-    topk_h = torch.from_numpy(d["topk_idx"]).pin_memory()
-    w_h = torch.from_numpy(d["topk_w"]).pin_memory()
-    y_h = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in sets]
-    h2d = x_h.numel() * 2 + topk_h.numel() * 4 + w_h.numel() * 4
-    d2h = y_h[0].numel() * 2
-    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    ev = lambda: torch.cuda.Event()
-    inputs_up, computed, result_down = [ev() for _ in sets], [ev() for _ in sets], [ev() for _ in sets]
-
-    def e2e_run(compute: bool) -> float:
-        """Wall seconds for e2e_steps pipelined steps (max over ranks);
-        compute=False moves the same bytes with no kernels (the copy bound)."""
-        torch.cuda.synchronize()
-        barrier()
-        t0 = time.perf_counter()
-        for i in range(e2e_steps):
-            j = i % 2
-            b = sets[j]
-            if i >= 2:
-                s_in.wait_event(computed[j])        # step i-2 has read this set's inputs
-            with torch.cuda.stream(s_in):
-                b.x.copy_(x_h, non_blocking=True)
-                b.topk.copy_(topk_h, non_blocking=True)
-                b.w.copy_(w_h, non_blocking=True)
-                inputs_up[j].record(s_in)
-            s_comp.wait_event(inputs_up[j])
-            if i >= 2:
-                s_comp.wait_event(result_down[j])   # step i-2's result has left this set's y
-            with torch.cuda.stream(s_comp):
-                if compute:
-                    capi.moe_layout_dispatch(cfg, b.topk, b.lay.struct, b.x, b.recv, b.staging)
-                    capi.moe_combine(cfg, b.lay.struct, b.recv, b.w, b.y)   # identity expert
-                computed[j].record(s_comp)
-            s_out.wait_event(computed[j])
-            with torch.cuda.stream(s_out):
-                y_h[j].copy_(b.y, non_blocking=True)
-                result_down[j].record(s_out)
-        for s_ in (s_in, s_comp, s_out):
-            s_.synchronize()
-        return max_over_ranks(time.perf_counter() - t0, world, dev)
-
-    copies_s = e2e_run(False)
-    e2e_s = e2e_run(True)
-    e2e_value = job_gbs(step_bytes, world, e2e_steps, e2e_s)
-
-    cpu = cpu_par = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        one = oracle_step_time(d, wl.T, 1, eo_bits)
-        reps = max(1, min(30, int(args.cpu_seconds / max(one, 1e-3))))
-        best = min(one, oracle_step_time(d, wl.T, reps, eo_bits))
-        cpu = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": 1,
-               "kind": "oracle",
-               "sample": f"full workload ({wl.T} tokens: layout+dispatch+combine), best of "
-                         f"{reps + 1} runs, single thread on {os.cpu_count()} host cores",
-               "cpu_model": cpu_model()}
-        import oracle
-        threads = oracle.parallel_threads()
-        one = oracle_step_time(d, wl.T, 1, eo_bits, parallel=True)
-        reps = max(1, min(30, int(args.cpu_seconds / 2 / max(one, 1e-3))))
-        best = min(one, oracle_step_time(d, wl.T, reps, eo_bits, parallel=True))
-        cpu_par = {"value": round(step_bytes / best / 1e9, 3), "unit": "GB/s", "cores": threads,
-                   "kind": "oracle, dispatch and combine token loops over OpenMP threads "
-                           "(layout serial)",
-                   "sample": f"full workload ({wl.T} tokens), best of {reps + 1} runs"}
-
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_desc(wl), parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                           l2=("inputs larger than L2: steps alternate between two independent "
-                               "buffer sets, each step moves %.0f MB (%.1fx L2)"
-                               % (step_bytes / 1e6, step_bytes / torch.cuda.get_device_properties(dev).L2_cache_size)),
-                           engine=args.engine,
-                           layout=("count kernel + assign/dispatch kernel" if ld_pair
-                                   else "one cluster launch" if cluster_layout else
-                                   ("count + assign kernels" if small_layout
-                                    else "count/scan/assign kernels")),
-                           entry="moe_layout + moe_dispatch" if args.unfused else "moe_layout_dispatch",
-                           timing=f"K steps back to back (CUDA graphs of {GRAPH_STEPS} steps) between "
-                                  "two CUDA events on the launching stream; stage costs from graphs "
-                                  "of layout, layout+dispatch and the full step"),
-            "pct_of_peak": round(100 * value / world / peak, 2),
-            "peak_gbs": peak, "peak_source": peak_src,
-            "pct_of_nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-            "tokens_per_s": round(wl.T * world * K / (total_ms * 1e-3), 1),
-            "tokens_per_s_dispatch_combine": round(wl.T * world / ((t_dispatch + t_combine) * 1e-3), 1),
-            "flushed_step": flushed,
-            "dispatch_combine_only_gbs": round(step_bytes / ((t_dispatch + t_combine) * 1e-3) / 1e9, 2),
-            "kernels_ms": ({"layout_dispatch": round(t_dispatch, 5), "combine": round(t_combine, 5),
-                            "layout_kernels_alone": round(t_l, 5)} if ld_pair else
-                           {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
-                            "combine": round(t_combine, 5)}),
-            "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 2),
-                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": profiled_traffic(dom_kernel, wl.name),
-                         "peak_kind": f"{peak_src} copy bandwidth"},
-            "decoupled_3pass": decoupled,
-            "allgather_reducescatter": agrs,
-            "fp8_payload": fp8,
-            "node_balance": balance,
-            "expert_parallel_virtual_ranks": ep_line,
-            "clocks": clocks.summary(),
-            "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                    "copies_only_value": round(job_gbs(step_bytes, world, e2e_steps, copies_s), 3),
-                    "mode": "moe_layout_dispatch + moe_combine per step, host copies pipelined "
-                            "on two copy streams over two buffer sets (wall clock)"},
-            "gpu_launches": launches_per_step * K,
-            "cpu_baseline": cpu,
-            "cpu_baseline_parallel": cpu_par,
-        }
-        print(json.dumps(line), flush=True)
     if world > 1:
-        dist.destroy_process_group()
-    return 0
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    ctx = Ctx(world, rank, local, dev)
+    try:
+        return run_several(args, ctx) if world > 1 else run_one(args, ctx)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
 
 
 if __name__ == "__main__":

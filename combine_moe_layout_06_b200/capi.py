@@ -53,6 +53,7 @@ ENTRY_POINTS = (
     "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
     "moe_combine_reducescatter", "moe_quantize_rows_fp8", "moe_dispatch_fp8", "moe_combine_fp8",
     "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine", "moe_dispatch_fp8_two_level",
+    "moe_ep_receive_rows",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -122,6 +123,7 @@ def lib() -> ctypes.CDLL:
     L.moe_ep_layout.argtypes = [C, ctypes.c_int32, ctypes.c_int32, P, P, LP, EP, P]
     L.moe_ep_dispatch.argtypes = [C, LP, EP, P, PP, ctypes.c_int64, P]
     L.moe_ep_combine.argtypes = [C, LP, EP, PP, ctypes.c_int64, P, P, P]
+    L.moe_ep_receive_rows.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -253,6 +255,20 @@ def moe_ep_layout(cfg: MoeConfig, source_rank: int, num_sources: int, topk_idx, 
     _check(lib().moe_ep_layout(ctypes.byref(cfg), source_rank, num_sources, _ptr(topk_idx),
                                _ptr(counts_all), ctypes.byref(local), ctypes.byref(ep),
                                _stream(stream)), "moe_ep_layout")
+
+
+def moe_ep_receive_rows(counts_all, num_ranks: int):
+    """Rows each of `num_ranks` expert ranks receives, from every source's
+    expert counts (host int32 [num_sources][num_experts]) -> list of int."""
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(counts_all), dtype=np.int32)
+    if c.ndim != 2:
+        raise ValueError("counts_all must be [num_sources][num_experts]")
+    out = (ctypes.c_int64 * max(int(num_ranks), 1))()
+    _check(lib().moe_ep_receive_rows(c.shape[1], int(num_ranks), c.shape[0],
+                                     c.ctypes.data_as(ctypes.c_void_p), out),
+           "moe_ep_receive_rows")
+    return list(out)[: int(num_ranks)]
 
 
 def moe_ep_dispatch(cfg: MoeConfig, local: MoeLayout, ep: MoeEpLayout, x, recv_bufs,

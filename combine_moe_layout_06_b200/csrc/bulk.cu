@@ -23,8 +23,9 @@
 //    stages leave room for 16 warps per SM to hide the summing latency.
 //
 // Every mbarrier wait is bounded; a wait that gives up records kErrTimeout,
-// stops issuing work, drains what it started and returns.  No load uses
-// cluster multicast.  Requires 16-byte aligned rows and base addresses.
+// stops issuing work, drains what it started and returns.  Every bulk load
+// is issued per CTA, into that CTA's own shared memory.  Requires 16-byte
+// aligned rows and base addresses.
 #include <climits>
 #include <initializer_list>
 

@@ -356,6 +356,25 @@ moe_status_t check_ep(const moe_config_t* c, const moe_layout_t* L, const moe_ep
 
 }  // namespace
 
+moe_status_t moe_ep_receive_rows(int32_t num_experts, int32_t num_ranks, int32_t num_sources,
+                                 const int32_t* counts_all, int64_t* rows_out) {
+    if (num_experts < 1 || num_ranks < 1 || num_sources < 1 || counts_all == nullptr ||
+        rows_out == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    if (num_experts < num_ranks) return MOE_ERR_EMPTY_RANK;
+    const int64_t n = (int64_t)num_sources * num_experts;
+    for (int64_t i = 0; i < n; ++i)
+        if (counts_all[i] < 0) return MOE_ERR_INVALID_ARG;
+    const moe::Partition part = moe::Partition::make(num_experts, num_ranks, 1);
+    for (int32_t r = 0; r < num_ranks; ++r) {
+        int64_t rows = 0;
+        for (int32_t e = part.first_expert(r); e < part.first_expert(r + 1); ++e)
+            for (int32_t g = 0; g < num_sources; ++g) rows += counts_all[(int64_t)g * num_experts + e];
+        rows_out[r] = rows;
+    }
+    return MOE_OK;
+}
+
 moe_status_t moe_ep_layout(const moe_config_t* c, int32_t g, int32_t G, const int32_t* topk_idx,
                            const int32_t* counts_all, const moe_layout_t* L,
                            const moe_ep_layout_t* ep, void* stream) {

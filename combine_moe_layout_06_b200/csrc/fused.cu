@@ -31,7 +31,7 @@
 //
 // Results equal moe_layout() followed by moe_dispatch() bit for bit.  The
 // ticket counter lives in the workspace: it must be zero before the first
-// launch, and every launch leaves it zero.  No load uses cluster multicast.
+// launch, and every launch leaves it zero.  Each CTA issues its own bulk loads.
 #include "layout_common.cuh"
 #include "moe_kernels.h"
 

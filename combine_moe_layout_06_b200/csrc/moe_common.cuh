@@ -207,7 +207,7 @@ __device__ __forceinline__ void warp_report(int* err_word, int bits) {
     if (any && (threadIdx.x & 31) == 0 && err_word != nullptr) atomicOr(err_word, any);
 }
 
-// ---- bulk copies (TMA, non-tensor, no multicast) and mbarriers ------------
+// ---- per-CTA bulk copies (TMA, non-tensor) and mbarriers -------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

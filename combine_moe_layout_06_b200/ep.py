@@ -20,29 +20,24 @@ import torch.distributed as dist
 from . import buffers, capi
 
 
-def gather_counts(local_counts: torch.Tensor, group=None) -> torch.Tensor:
+def gather_counts(local_counts: torch.Tensor, group=None, out: torch.Tensor | None = None
+                  ) -> torch.Tensor:
     """All-gather of every rank's int32 [E] expert counts -> [G, E], source
-    rank order.  The tensors live where the group's backend wants them (CPU
-    for gloo, the GPU for NCCL)."""
+    rank order, written into `out` when given.  The tensors live where the
+    group's backend wants them (CPU for gloo, the GPU for NCCL)."""
     world = dist.get_world_size(group)
-    parts = [torch.empty_like(local_counts) for _ in range(world)]
-    dist.all_gather(parts, local_counts.contiguous(), group=group)
-    return torch.stack(parts)
+    E = local_counts.numel()
+    if out is None:
+        out = torch.empty((world, E), dtype=local_counts.dtype, device=local_counts.device)
+    dist.all_gather_into_tensor(out.view(-1), local_counts.contiguous(), group=group)
+    return out
 
 
-def receive_rows(counts_all: np.ndarray, num_ranks: int) -> np.ndarray:
-    """Rows each rank receives: the experts of rank r (ceil/floor partition,
-    the first E mod R ranks holding one more) summed over all sources."""
-    counts_all = np.asarray(counts_all)
-    E = counts_all.shape[1]
-    base, rem = divmod(E, num_ranks)
-    sizes = [base + (1 if r < rem else 0) for r in range(num_ranks)]
-    per_expert = counts_all.sum(axis=0)
-    out, e0 = [], 0
-    for n in sizes:
-        out.append(int(per_expert[e0:e0 + n].sum()))
-        e0 += n
-    return np.array(out, np.int64)
+def receive_rows(counts_all, num_ranks: int) -> np.ndarray:
+    """Rows each expert rank receives, from the gathered counts [G, E]
+    (moe_ep_receive_rows() of the library: the ceil/floor partition's
+    experts of each rank, summed over all sources)."""
+    return np.array(capi.moe_ep_receive_rows(np.asarray(counts_all), num_ranks), np.int64)
 
 
 def share_buffer(t: torch.Tensor, group=None) -> list:

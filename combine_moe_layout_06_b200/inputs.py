@@ -151,7 +151,34 @@ def x_bf16_bits(x_f32: np.ndarray) -> np.ndarray:
 def make(name: str) -> dict:
     """Inputs of a named workload: x (uint16 bf16 bits [T,H]), topk_idx
     (int32 [T,k]), topk_w (float32 [T,k]) and routing metadata."""
-    wl = WORKLOADS[name]
+    return _generate(WORKLOADS[name])
+
+
+def make_source(name: str, source: int) -> dict:
+    """Inputs of source rank `source` of a named workload when every rank
+    routes a batch of its own (same shape and routing recipe, the seed moved
+    by 1000 per rank; rank 0 gets the workload's own inputs)."""
+    if source == 0:
+        return make(name)
+    return _generate(dataclasses.replace(WORKLOADS[name], seed=WORKLOADS[name].seed + 1000 * source))
+
+
+def prefix(d: dict, tokens: int) -> dict:
+    """The first `tokens` tokens of a workload's inputs (same rows, same
+    routes and weights) as a scaled-down case of the same shape; the
+    workload record's T becomes `tokens`."""
+    wl = d["workload"]
+    tokens = max(1, min(int(tokens), wl.T))
+    out = dict(d)
+    out["workload"] = dataclasses.replace(wl, T=tokens)
+    for key in ("x", "topk_idx", "topk_w"):
+        out[key] = np.ascontiguousarray(d[key][:tokens])
+    if "home_node" in d:
+        out["home_node"] = d["home_node"][:tokens]
+    return out
+
+
+def _generate(wl: Workload) -> dict:
     xrng, rrng = _streams(wl.seed)
     x = xrng.standard_normal((wl.T, wl.H), dtype=np.float32)
     logits, extra = router_logits(wl, rrng)

@@ -342,6 +342,20 @@ typedef struct moe_ep_layout {
     int32_t *slot;
 } moe_ep_layout_t;
 
+/* Rows every expert rank receives, from the gathered counts of step 2 (host
+ * arithmetic only, for sizing the receive and expert-output buffers before
+ * the first step): rows_out[r] = the sum over sources g and over rank r's
+ * experts e (the ceil/floor contiguous partition of moe_expert_partition())
+ * of counts_all[g][e].  These equal the differences of the rank_offsets
+ * that moe_ep_layout() writes.
+ *   counts_all  HOST int32 [num_sources][num_experts], every count >= 0
+ *   rows_out    HOST int64 [num_ranks]
+ * Errors (nothing written): MOE_ERR_INVALID_ARG for a NULL pointer, a size
+ * below 1 or a negative count; MOE_ERR_EMPTY_RANK when num_experts <
+ * num_ranks. */
+moe_status_t moe_ep_receive_rows(int32_t num_experts, int32_t num_ranks, int32_t num_sources,
+                                 const int32_t *counts_all, int64_t *rows_out);
+
 /* Step 3.  cfg: this rank's shard (as in step 1); source_rank g in
  * [0, num_sources); counts_all: device int32 [num_sources][E] with row g equal
  * to local->expert_counts; topk_idx: the shard's routes; local: the layout of
