@@ -15,7 +15,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe_layout.so")
+# MOE_LAYOUT_LIB names another build of the library (e.g. a test build with
+# shortened device waits); the in-tree build is the default.
+LIB_PATH = os.environ.get("MOE_LAYOUT_LIB") or os.path.join(_HERE, "libmoe_layout.so")
 
 MOE_MAX_EXPERTS = 1024
 MOE_MAX_TOPK = 32

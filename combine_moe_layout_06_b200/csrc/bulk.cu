@@ -27,6 +27,7 @@
 // is issued per CTA, into that CTA's own shared memory.  Requires 16-byte
 // aligned rows and base addresses.
 #include <climits>
+#include <cstdlib>
 #include <initializer_list>
 
 #include "moe_kernels.h"
@@ -78,6 +79,12 @@ struct BulkArgs {
     int early;                // start source loads before waiting (see RowMoveParams)
     char* staging = nullptr;  // node_dispatch_kernel: node staging rows
     int64_t staging_rows = 0;
+#ifdef MOE_TEST_HOOKS
+    // Test builds only: the flat dispatch's warp 0 of block 0 announces the
+    // bytes of this item on its stage's mbarrier but issues no load for it,
+    // so that wait runs out on a healthy GPU (nothing is left in flight).
+    int64_t test_skip_item = -1;
+#endif
 };
 
 // Drain after a timeout: wait (bounded) for every stage this warp still
@@ -148,10 +155,17 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
         int64_t row, base;
         uint32_t bytes;
         const int64_t src_row = source(first + q, row, base, bytes);
+#ifdef MOE_TEST_HOOKS
+        const bool skip = MODE == kFlat && blockIdx.x == 0 && warp == 0 && first + q == a.test_skip_item;
+#else
+        constexpr bool skip = false;
+#endif
         if (lane == 0) {
             if (src_row >= 0) {
                 mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_load(stage0 + (size_t)s * a.chunk, a.src + src_row * a.row_bytes + base, bytes, &full[s]);
+                if (!skip)
+                    bulk_load(stage0 + (size_t)s * a.chunk, a.src + src_row * a.row_bytes + base, bytes,
+                              &full[s]);
             } else {
                 mbar_arrive_expect_tx(&full[s], 0);  // empty item: complete the phase
             }
@@ -558,7 +572,10 @@ bool bulk_eligible(size_t row_bytes, std::initializer_list<const void*> ptrs) {
 
 cudaError_t launch_dispatch_flat_bulk(const RowMoveParams& p, const void* x, void* recv,
                                       cudaStream_t stream) {
-    const BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kDispChunk);
+    BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kDispChunk);
+#ifdef MOE_TEST_HOOKS
+    if (const char* v = std::getenv("MOE_TEST_SKIP_LOAD")) a.test_skip_item = std::atoll(v);
+#endif
     return launch_disp_bulk<kFlat>(a, p.T, stream);
 }
 

@@ -1,12 +1,13 @@
 // capi.cu -- the C ABI of libmoe_layout.so (declared in include/moe_layout.h):
 // host-side validation, then the kernel launchers.  No entry point
 // allocates device memory.
-#include "moe_layout.h"
-#include "moe_kernels.h"
+#include "capi_internal.h"
 
 namespace {
 
+using moe::check_layout_ptrs;
 using moe::CopyEngine;
+using moe::layout_params;
 
 constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK |
                                  MOE_FLAG_LAYOUT_CLUSTER | MOE_FLAG_LAYOUT_FUSED |
@@ -21,18 +22,6 @@ CopyEngine engine_of(uint32_t flags) {
 }
 
 bool two_level(const moe_config_t* c) { return (c->flags & MOE_FLAG_TWO_LEVEL) != 0; }
-
-moe_status_t check_layout_ptrs(const moe_config_t* c, const moe_layout_t* L) {
-    // Per-token arrays may be NULL only when there are no tokens.
-    const bool tokens = c->num_tokens > 0;
-    if (L == nullptr || L->expert_counts == nullptr || L->expert_offsets == nullptr ||
-        L->rank_offsets == nullptr || (tokens && L->slot == nullptr) || L->error_word == nullptr)
-        return MOE_ERR_INVALID_ARG;
-    if (two_level(c) && (L->node_counts == nullptr || L->node_offsets == nullptr ||
-                         (tokens && L->node_slot == nullptr)))
-        return MOE_ERR_INVALID_ARG;
-    return MOE_OK;
-}
 
 int64_t staging_rows(const moe_config_t* c) {
     const int32_t m = c->num_nodes < c->top_k ? c->num_nodes : c->top_k;
@@ -85,15 +74,31 @@ moe_status_t dispatch_impl(const moe_config_t* c, const moe_layout_t* L, const v
     return cuda_status(e);
 }
 
-moe::LayoutParams layout_params(const moe_config_t* c, const int32_t* topk_idx,
-                                const moe_layout_t* L) {
-    moe::LayoutParams p;
+}  // namespace
+
+namespace moe {
+
+moe_status_t check_layout_ptrs(const moe_config_t* c, const moe_layout_t* L) {
+    // Per-token arrays may be NULL only when there are no tokens.
+    const bool tokens = c->num_tokens > 0;
+    if (L == nullptr || L->expert_counts == nullptr || L->expert_offsets == nullptr ||
+        L->rank_offsets == nullptr || (tokens && L->slot == nullptr) || L->error_word == nullptr)
+        return MOE_ERR_INVALID_ARG;
+    const bool nodes = (c->flags & MOE_FLAG_TWO_LEVEL) != 0;
+    if (nodes && (L->node_counts == nullptr || L->node_offsets == nullptr ||
+                  (tokens && L->node_slot == nullptr)))
+        return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+LayoutParams layout_params(const moe_config_t* c, const int32_t* topk_idx, const moe_layout_t* L) {
+    LayoutParams p;
     p.T = c->num_tokens;
     p.k = c->top_k;
     p.E = c->num_experts;
     p.R = c->num_ranks;
     p.N = c->num_nodes;
-    p.nodes = two_level(c);
+    p.nodes = (c->flags & MOE_FLAG_TWO_LEVEL) != 0;
     p.cluster = (c->flags & MOE_FLAG_LAYOUT_CLUSTER) != 0;
     p.topk = topk_idx;
     p.expert_counts = L->expert_counts;
@@ -109,7 +114,7 @@ moe::LayoutParams layout_params(const moe_config_t* c, const int32_t* topk_idx,
     return p;
 }
 
-}  // namespace
+}  // namespace moe
 
 extern "C" {
 

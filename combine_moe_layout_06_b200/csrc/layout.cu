@@ -746,14 +746,17 @@ size_t fused_workspace_offset(int64_t T, int E) {
     return round_up(sizeof(int) * (size_t)E * (size_t)C, 256);
 }
 
-size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes) {
+size_t layout_scratch_bytes(int64_t T, int E, int N, bool nodes) {
     const int64_t C = (T + kTokensPerCta - 1) / kTokensPerCta;
     size_t b = round_up(sizeof(int) * (size_t)E * (size_t)C, 256);
-    if (nodes)
-        b += round_up(sizeof(int) * (size_t)N * (size_t)C, 256);
-    else
-        b += kFusedBarrierBytes + round_up(sizeof(int) * (size_t)E * kFusedMaxCtas, 256);
+    if (nodes) b += round_up(sizeof(int) * (size_t)N * (size_t)C, 256);
     return b < 256 ? 256 : b;
+}
+
+size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes) {
+    if (nodes) return layout_scratch_bytes(T, E, N, nodes);
+    return fused_workspace_offset(T, E) + kFusedBarrierBytes +
+           round_up(sizeof(int) * (size_t)E * kFusedMaxCtas, 256);
 }
 
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {

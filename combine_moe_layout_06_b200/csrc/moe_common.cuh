@@ -238,8 +238,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait for an mbarrier phase: false once kMaxWaitNs of wall time
 // (%globaltimer) have passed without the phase completing, which callers
-// turn into kErrTimeout instead of spinning forever.
-constexpr uint64_t kMaxWaitNs = 200ull * 1000 * 1000;
+// turn into kErrTimeout instead of spinning forever.  200 ms by default; a
+// test build of the library shortens it with -DMOE_MAX_WAIT_NS=<ns>.
+#ifndef MOE_MAX_WAIT_NS
+#define MOE_MAX_WAIT_NS (200ull * 1000 * 1000)
+#endif
+constexpr uint64_t kMaxWaitNs = MOE_MAX_WAIT_NS;
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -39,6 +39,10 @@ struct LayoutParams {
 // must be zero before the first launch and is left zero by every launch,
 // then an [E][kFusedMaxCtas] histogram matrix.
 size_t layout_workspace_bytes(int64_t T, int E, int N, bool nodes);
+// The part of the workspace launch_layout() itself reads and writes (the
+// chunk histograms, and the node histograms with node staging); every word
+// of it is written by a launch before that launch reads it.
+size_t layout_scratch_bytes(int64_t T, int E, int N, bool nodes);
 cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream);
 
 // ---- layout and flat dispatch, assignment folded into the dispatch (fused.cu)

@@ -440,12 +440,15 @@ moe_status_t moe_combine_fp8(const moe_config_t *cfg, const moe_layout_t *layout
  * inside the library's device memory (held on every GPU that loads the
  * library until the process exits); layout->workspace is ignored and may be
  * NULL.  Nothing is allocated.
- *  - Limit: configurations whose moe_layout_workspace_bytes() exceeds
+ *  - Limit: the layout's scratch is its per-chunk histograms, 4 * E *
+ *    ceil(T / 256) bytes, plus 4 * N * ceil(T / 256) with MOE_FLAG_TWO_LEVEL,
+ *    each rounded up to 256 bytes.  Configurations that need more than
  *    MOE_LAYOUT_NOALLOC_SCRATCH_BYTES are refused with MOE_ERR_INVALID_ARG
- *    before anything is enqueued.
- *  - The first call on a device looks up the array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    before anything is enqueued (e.g. E = 256 allows T up to 1,048,576).
+ *  - Every call looks up the array's device address on the current device
+ *    (a host-side lookup, nothing is enqueued).  The first call on a device
+ *    may also load the library's device code there; make that first call
+ *    before any stream capture.
  *  - All calls on a device share the one array: calls that overlap on the
  *    GPU (other streams, or other threads' streams) race and give wrong
  *    layouts.  Order them on one stream or with events.
