@@ -588,6 +588,10 @@ class StepBench:
         self.layout_dispatch(b)
         capi.moe_combine(self.cfg, b.lay.struct, b.eo, b.w, b.y)
 
+    def combine(self, b):
+        from combine_moe_layout_06_b200 import capi
+        capi.moe_combine(self.cfg, b.lay.struct, b.eo, b.w, b.y)
+
     def decoupled_step(self, b):
         from combine_moe_layout_06_b200 import capi
         capi.moe_layout(self.dcfg, b.topk, b.dlay.struct)
@@ -704,7 +708,7 @@ class StepBench:
             return capture(fn, GRAPH_STEPS), capture(fn, 2), capture(fn, 1)
 
         self.graphs = {"step": graph_set(self.step), "L": graph_set(self.layout),
-                       "LD": graph_set(self.layout_dispatch)}
+                       "LD": graph_set(self.layout_dispatch), "C": graph_set(self.combine)}
         if self.with_decoupled:
             self.graphs["decoupled"] = graph_set(self.decoupled_step)
         if self.with_agrs:
@@ -772,6 +776,7 @@ class StepBench:
             raw["step"] = self.timed("step", K)
             raw["L"] = self.timed("L", K) / K
             raw["LD"] = self.timed("LD", K) / K
+            raw["C"] = self.timed("C", K) / K
             for name in ("decoupled", "agrs", "fp8", "ep"):
                 if name in self.graphs:
                     raw[name] = self.timed(name, K)
@@ -834,7 +839,9 @@ class StepBench:
             "kernels_ms": ({"layout_dispatch": round(t_dispatch, 5), "combine": round(t_combine, 5),
                             "layout_kernels_alone": round(t_l, 5)} if self.ld_pair else
                            {"layout": round(t_layout, 5), "dispatch": round(t_dispatch, 5),
-                            "combine": round(t_combine, 5)}),
+                            "combine": round(t_combine, 5),
+                            # combines alone, back to back (layouts from the warm-up)
+                            "combine_alone": round(raw["C"], 5)}),
             "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 2),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": profiled_traffic(dom_kernel, wl.name if wl.T == inputs.WORKLOADS[wl.name].T

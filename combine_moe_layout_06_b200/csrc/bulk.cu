@@ -77,6 +77,7 @@ struct BulkArgs {
     int64_t src_rows, dst_rows;
     int* err;
     int early;                // start source loads before waiting (see RowMoveParams)
+    int late_trigger = 0;     // let the dependent grid launch at the end (pdl_trigger_at_end)
     char* staging = nullptr;  // node_dispatch_kernel: node staging rows
     int64_t staging_rows = 0;
 #ifdef MOE_TEST_HOOKS
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
     // Flat and node-pack sources are x rows, which need no layout data: with
     // early inputs the first stages are loaded while the layout still runs.
     const bool early = a.early != 0 && (MODE == kFlat || MODE == kNodePack);
-    pdl_trigger();
+    if (!a.late_trigger) pdl_trigger();
     if (!early) pdl_wait();
 
     int errbits = 0;
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
             inflight |= 1u << ((q - 1) % kDispStages);
         }
     }
+    if (a.late_trigger) pdl_trigger();
     bulk_wait_all();
     warp_report(a.err, errbits);
 }
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
     }
     __syncwarp();
     const bool early = a.early != 0;
-    pdl_trigger();
+    if (!a.late_trigger) pdl_trigger();
     if (!early) pdl_wait();
 
     const int64_t items = a.T * a.cpr;
@@ -409,6 +411,7 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
         for (int i = 0; i < 3; ++i)
             if (inflight & (1u << i)) (void)mbar_wait(&bar[i], (parity >> i) & 1u);
     }
+    if (a.late_trigger) pdl_trigger();
     bulk_wait_all();
     warp_report(a.err, errbits);
 }
@@ -523,11 +526,12 @@ __global__ void __launch_bounds__(kBulkThreads) combine_bulk_kernel(BulkArgs a) 
 }
 
 template <auto Kernel>
-cudaError_t launch_bulk(const BulkArgs& a, int64_t items, size_t smem, cudaStream_t stream) {
+cudaError_t launch_bulk(BulkArgs a, int64_t items, size_t smem, cudaStream_t stream) {
     if (items <= 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = persistent_grid<Kernel>(items, kBulkThreads, smem);
+    a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<Kernel>(kBulkThreads, smem)) ? 1 : 0;
     return launch_pdl(Kernel, dim3(grid), dim3(kBulkThreads), smem, stream, a);
 }
 
@@ -606,6 +610,8 @@ cudaError_t launch_node_dispatch_bulk(const RowMoveParams& p, const void* x, voi
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = persistent_grid<node_dispatch_kernel>(items, kNfThreads, smem);
+    a.late_trigger =
+        pdl_trigger_at_end(grid, resident_blocks<node_dispatch_kernel>(kNfThreads, smem)) ? 1 : 0;
     return launch_pdl(node_dispatch_kernel, dim3(grid), dim3(kNfThreads), smem, stream, a);
 }
 

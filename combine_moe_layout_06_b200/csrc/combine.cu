@@ -58,6 +58,7 @@ struct CombArgs {
     const int* rank_offsets;
     int ep_ranks;
     int64_t ep_capacity;
+    int late_trigger;  // let the dependent grid launch at the end (pdl_trigger_at_end)
 };
 
 // Lane r < ep_ranks: rank r's rows [lo, hi) and its buffer (EP only).
@@ -100,7 +101,7 @@ template <typename V, int VPL, int KB, bool EP = false>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     constexpr int EPV = VecInfo<V>::kElems;
     constexpr int CHUNK = 32 * VPL;
-    pdl_trigger();
+    if (!a.late_trigger) pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     EpLane el = {0, 0, 0ull};
@@ -181,6 +182,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
             }
         }
     }
+    if (a.late_trigger) pdl_trigger();
     warp_report(a.err, errbits);
 }
 
@@ -189,6 +191,7 @@ cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
     constexpr auto kern = combine_kernel<V, VPL, KB, EP>;
     const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
     const int grid = persistent_grid<kern>(a.T * cpr, kThreads, 0, MOE_COMBINE_IPW);
+    a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<kern>(kThreads)) ? 1 : 0;
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
 }
 

@@ -74,11 +74,25 @@ struct LayoutArgs {
     int* node_slot;
     int* node_src;  // [U] staging row -> token, or nullptr
     int* err;
+    // the assign kernel copies the whole [E][C] (and [N][C]) histogram into
+    // shared memory with bulk copies (16-byte aligned workspace, small enough)
+    bool bulk_hist;
 };
+
+// Histogram bytes the assign kernel copies into shared memory at most, and
+// the fewest chunks for which it does: up to 32 chunks one round of plain
+// loads reads the histogram as fast (measured on B200: the olmoe layout, 16
+// chunks, took 7.0 us with the copy and 6.6 us without; dsv3, 64 chunks,
+// 16.4 us against 22.5 us).
+constexpr size_t kBulkHistMaxBytes = 128 * 1024;
+#ifndef MOE_BULK_HIST_MIN_CHUNKS
+#define MOE_BULK_HIST_MIN_CHUNKS 33
+#endif
+__host__ __device__ inline size_t round16(size_t v) { return (v + 15) / 16 * 16; }
 
 template <int KMAX>
 __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs a) {
-    extern __shared__ int smem[];
+    extern __shared__ __align__(16) int smem[];
     int* s_cnt = smem;           // [E]
     int* s_ncnt = smem + a.E;    // [N]
     for (int i = threadIdx.x; i < a.E + a.N; i += blockDim.x) smem[i] = 0;
@@ -165,7 +179,7 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutArgs a)
 
 template <int KMAX>
 __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs a) {
-    extern __shared__ int smem[];
+    extern __shared__ __align__(16) int smem[];
     int* s_wcnt = smem;                                                    // [8][E]
     unsigned* s_mask = reinterpret_cast<unsigned*>(smem + kLayoutWarps * a.E);  // [8][E]
     int* s_wn = smem + 2 * kLayoutWarps * a.E;                             // [8][N]
@@ -264,13 +278,21 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_kernel(LayoutArgs
 // waiting for the count kernel: topk_idx was written before the layout
 // began, and the count kernel waits for its writer before it lets this grid
 // launch.  It lets its dependent grid launch only after the histogram reads.
-// Shared memory (ints): tot[E+N] base[E+N] wcnt[8][E] mask[8][E] wn[8][N].
+// Shared memory (ints): tot[E+N] base[E+N] wcnt[8][E] mask[8][E] wn[8][N],
+// then (bulk_hist) the [E][C] histogram and the [N][C] node histogram, each
+// padded to 16 bytes, and an mbarrier.
 constexpr int kFusedScanMaxChunks = 256;
+
+// Offset (ints) of the copied histograms in the assign kernel's shared
+// memory: after the fixed part, rounded up to a multiple of 4 ints.
+__host__ __device__ inline int assign_scan_hist_offset(int E, int N) {
+    return (2 * (E + N) + 2 * kLayoutWarps * E + kLayoutWarps * N + 3) & ~3;
+}
 
 template <int KMAX>
 __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(LayoutArgs a) {
     __shared__ int s_warp[32];
-    extern __shared__ int smem[];
+    extern __shared__ __align__(16) int smem[];
     const int E = a.E, N = a.N, EN = a.E + a.N, C = a.C;
     int* tot = smem;
     int* base = tot + EN;
@@ -278,7 +300,16 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
     unsigned* s_mask = reinterpret_cast<unsigned*>(s_wcnt + kLayoutWarps * E);
     int* s_wn = reinterpret_cast<int*>(s_mask + kLayoutWarps * E);
     const int words = 2 * kLayoutWarps * E + kLayoutWarps * N;
+    const size_t hist_e = round16(sizeof(int) * (size_t)E * C);
+    const size_t hist_n = a.nodes ? round16(sizeof(int) * (size_t)N * C) : 0;
+    // the copied histograms start at the next 16-byte boundary
+    int* s_hist = smem + assign_scan_hist_offset(E, N);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(s_hist) + hist_e + hist_n);
     for (int i = threadIdx.x; i < words; i += blockDim.x) s_wcnt[i] = 0;
+    if (a.bulk_hist && threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+    }
     __syncthreads();
 
     const int warp = threadIdx.x >> 5;
@@ -307,9 +338,19 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
         }
     }
     pdl_wait();
+    if (a.bulk_hist && threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(hist_e + hist_n));
+        bulk_load(s_hist, a.cnt, (uint32_t)hist_e, bar);
+        if (hist_n) bulk_load(reinterpret_cast<char*>(s_hist) + hist_e, a.ncnt, (uint32_t)hist_n, bar);
+    }
 
-    // totals and earlier-chunk rows of each expert / node.  Each round of
-    // loads costs an L2 round trip, so the shape of the read follows C:
+    // totals and earlier-chunk rows of each expert / node.  Bulk path: one
+    // round trip brings the whole histogram into shared memory; warp w then
+    // reduces rows w, w + 8, ..., four rows at a time, lane l summing
+    // columns l, l + 32, ... (conflict-free) and one warp reduction per row
+    // for the total and one for the chunks before this CTA's.
+    // Otherwise each round of loads costs an L2 round trip, so the shape of
+    // the read follows C:
     //  - C <= 32: the [E+N][C] histogram is walked column-major (neighbouring
     //    threads on different rows, so their shared-memory adds do not
     //    collide), eight loads per thread in flight -- one round for E*C up
@@ -321,7 +362,50 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
         base[i] = 0;
     }
     __syncthreads();
-    if (C <= 32) {
+    if (a.bulk_hist) {
+        if (!__syncthreads_and(mbar_wait(bar, 0))) {
+            // the copy never completed: give up on this chunk, once the copy
+            // is no longer in flight (bounded), and report it
+            if (threadIdx.x == 0) {
+                (void)mbar_wait(bar, 0);
+                atomicOr(a.err, kErrTimeout);
+            }
+            __syncthreads();
+            return;
+        }
+        const int* h_n = reinterpret_cast<const int*>(reinterpret_cast<const char*>(s_hist) + hist_e);
+        const int cta = (int)blockIdx.x;
+        for (int i0 = warp * 4; i0 < EN; i0 += kLayoutWarps * 4) {
+            int sum[4], pre[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                sum[r] = 0;
+                pre[r] = 0;
+                const int i = i0 + r;
+                if (i < EN) {
+                    const int* row = i < E ? s_hist + (size_t)i * C : h_n + (size_t)(i - E) * C;
+                    for (int c = lane; c < C; c += 32) {
+                        const int v = row[c];
+                        sum[r] += v;
+                        pre[r] += c < cta ? v : 0;
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                sum[r] = __reduce_add_sync(kFullMask, sum[r]);
+                pre[r] = __reduce_add_sync(kFullMask, pre[r]);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (i0 + r < EN) {
+                        tot[i0 + r] = sum[r];
+                        base[i0 + r] = pre[r];
+                    }
+            }
+        }
+    } else if (C <= 32) {
         const int64_t nall = (int64_t)EN * C;
         for (int64_t f0 = threadIdx.x; f0 < nall; f0 += 8 * (int64_t)blockDim.x) {
             int v[8], row[8], col[8];
@@ -463,7 +547,7 @@ __global__ void __launch_bounds__(1024) layout_cluster_kernel(LayoutArgs a, int6
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     __shared__ int s_warp[32];
-    extern __shared__ int smem[];
+    extern __shared__ __align__(16) int smem[];
     const int E = a.E, N = a.N, EN = a.E + a.N;
     const int ES = (E & 1) ? E : E + 1;
     const int W = blockDim.x >> 5;
@@ -633,8 +717,10 @@ cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t stream) {
         if (err != cudaSuccess) return err;
     }
     if (a.C > 0 && a.C <= kFusedScanMaxChunks) {
-        const size_t smem =
-            sizeof(int) * (size_t)(2 * (a.E + a.N) + 2 * kLayoutWarps * a.E + kLayoutWarps * a.N);
+        size_t smem = sizeof(int) * (size_t)assign_scan_hist_offset(a.E, a.N);
+        if (a.bulk_hist)
+            smem += round16(sizeof(int) * (size_t)a.E * a.C) +
+                    (a.nodes ? round16(sizeof(int) * (size_t)a.N * a.C) : 0) + sizeof(uint64_t);
         if (smem > 48 * 1024) {
             err = cudaFuncSetAttribute(layout_assign_scan_kernel<KMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -781,6 +867,14 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
     a.node_slot = p.node_slot;
     a.node_src = p.nodes ? p.node_src : nullptr;
     a.err = p.err;
+    {
+        // the histograms start 256 bytes apart from the workspace base, so a
+        // 16-byte aligned workspace makes both bulk copies aligned
+        const size_t bytes = round16(sizeof(int) * (size_t)p.E * a.C) +
+                             (p.nodes ? round16(sizeof(int) * (size_t)p.N * a.C) : 0);
+        a.bulk_hist = reinterpret_cast<uintptr_t>(p.workspace) % 16 == 0 &&
+                      bytes <= kBulkHistMaxBytes && a.C >= MOE_BULK_HIST_MIN_CHUNKS;
+    }
     // One chunk of tokens (T <= 256): one CTA sees every token, so the
     // single-cluster kernel (a cluster of one CTA) does the whole layout in one
     // launch, with no count kernel and no kernel boundary before the ranks.

@@ -340,6 +340,32 @@ inline int blocks_per_sm(int threads, size_t smem = 0) {
     return cached;
 }
 
+// Blocks of a kernel resident on the whole device at once.
+template <auto Kernel>
+inline int64_t resident_blocks(int threads, size_t smem = 0) {
+    return (int64_t)device_sm_count() * blocks_per_sm<Kernel>(threads, smem);
+}
+
+// Where a row-moving kernel lets its dependent grid launch (programmatic
+// dependent launch).  The dependent grid launches once every CTA of this
+// grid has triggered or exited, and its CTAs then occupy SM slots while they
+// wait for this grid to finish.  Triggering at entry hides the dependent's
+// launch latency, which pays when the whole grid is resident at once.  In a
+// grid of several waves, the entry trigger of the last wave lets the
+// dependent's CTAs in while the last wave still moves rows, and measured on
+// B200 that slowed the step (a one-kernel two-level dispatch followed by a
+// combine: 809 us per step against 761 us with the trigger at the end).
+// MOE_PDL_POLICY: 0 = always at entry, 1 = at the end for grids of more than
+// one wave (default), 2 = always at the end.
+#ifndef MOE_PDL_POLICY
+#define MOE_PDL_POLICY 1
+#endif
+inline bool pdl_trigger_at_end(int64_t grid, int64_t resident) {
+    if (MOE_PDL_POLICY == 0) return false;
+    if (MOE_PDL_POLICY == 2) return true;
+    return grid > resident;
+}
+
 // Grid for a warp-strided loop over `warp_items` items.  Small problems get
 // a persistent grid (each warp one contiguous range of items).  When a
 // resident grid would give each warp at least 2 * items_per_warp items, the
