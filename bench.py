@@ -364,7 +364,9 @@ def node_balance(args, ctx):
     sk = NODE_SKEW
     T, H, E, k, R, N = (sk[c] for c in ("T", "H", "E", "k", "R", "N"))
     d = inputs.make_node_skewed(T, H, E, k, N, sk["hot_frac"], sk["seed"])
-    cfg = capi.config(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | engine_flags(args))
+    # the expansion kernel is what is compared, so the split form
+    cfg = capi.config(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | capi.MOE_FLAG_TWO_LEVEL_SPLIT |
+                      engine_flags(args))
     bf16 = dict(dtype=torch.bfloat16, device=dev)
     rows = capi.moe_node_staging_rows(cfg)
 
@@ -459,8 +461,8 @@ class StepBench:
             flags |= capi.MOE_FLAG_LAYOUT_CLUSTER
         if args.layout == "fused":
             flags |= capi.MOE_FLAG_LAYOUT_FUSED
-        if args.two_level_fused:
-            flags |= capi.MOE_FLAG_TWO_LEVEL_FUSED
+        if args.two_level_split:
+            flags |= capi.MOE_FLAG_TWO_LEVEL_SPLIT
         self.flags = flags
         cfg = self.cfg = capi.config(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, flags)
         # the decoupled comparison path packs per rank: one "node" per rank
@@ -562,9 +564,9 @@ class StepBench:
         # or layout override)
         self.ld_pair = (not args.unfused and not wl.two_level and args.layout == "fused"
                         and (wl.H * 2) % 16 == 0 and wl.E <= 256)
-        # two-level: pack + expand, or one kernel with --two-level-fused
-        # (16-byte rows, N + k <= 32)
-        self.two_kernels = wl.two_level and (not args.two_level_fused or args.engine == "vector"
+        # two-level: one kernel (16-byte rows, N + k <= 32), else or with
+        # --two-level-split a pack kernel then an expansion kernel
+        self.two_kernels = wl.two_level and (args.two_level_split or args.engine == "vector"
                                              or (wl.H * 2) % 16 or wl.N + wl.k > 32)
         self.launches_per_step = (2 if self.ld_pair else
                                   layout_launches + (2 if self.two_kernels else 1)) + 1
@@ -1228,8 +1230,9 @@ def parse_args(argv=None):
     p.add_argument("--layout", default="kernels", choices=["kernels", "fused", "cluster"],
                    help="kernels: layout kernels then the dispatch kernel; fused: a count kernel "
                         "then an assign/dispatch kernel (flat); cluster: one-cluster layout")
-    p.add_argument("--two-level-fused", action="store_true",
-                   help="two-level dispatch in one kernel (staging rows read back from L2)")
+    p.add_argument("--two-level-split", action="store_true",
+                   help="two-level dispatch as a pack kernel then an expansion kernel (default: "
+                        "one kernel, staging rows read back from L2)")
     p.add_argument("--unfused", action="store_true",
                    help="moe_layout + moe_dispatch instead of moe_layout_dispatch")
     p.add_argument("--e2e-steps", type=int, default=0, help="end-to-end steps (0: min(K, 50))")

@@ -29,6 +29,7 @@ MOE_FLAG_COPY_BULK = 0x4
 MOE_FLAG_LAYOUT_CLUSTER = 0x8
 MOE_FLAG_LAYOUT_FUSED = 0x10
 MOE_FLAG_TWO_LEVEL_FUSED = 0x20
+MOE_FLAG_TWO_LEVEL_SPLIT = 0x40
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = 1

@@ -252,33 +252,49 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
 // 去重": a token crosses to a node once, into that node's forwarding region,
 // and is fanned out to the node's experts from there).  Per (token, chunk)
 // item a warp
-//   1. loads the x chunk into shared memory (double-buffered: the next
-//      item's chunk is loaded while this one is handled),
+//   1. loads the x chunk into a ring of kNfX shared-memory stages (the next
+//      kNfX - 1 items' chunks are in flight while this one is handled),
 //   2. stores it to the token's staging row of every node it touches (lane
 //      31 - n for node n),
-//   3. once those stores are complete, reads each node's staging row back
-//      into shared memory and stores it to the token's receive rows on that
-//      node (lane j < k for column j).
+//   3. once those stores are complete, reads the staging rows back, up to
+//      kNfR nodes at once into read-back buffers, and stores each to the
+//      token's receive rows on that node (lane j < k for column j).
 // Step 3 reads the staging rows right after they were written, so the reads
 // are served by L2 instead of a second pass over HBM.  The staging buffer and
 // the receive rows end up exactly as with the two-kernel form (pack, then
-// expansion).  Needs N + k <= 32.  Opt-in (MOE_FLAG_TWO_LEVEL_FUSED): it
-// moves fewer bytes, but nearly all of them are writes, and measured right
-// before a combine the step is slower than with the two-kernel form, whose
-// expansion mixes the staging reads into its writes.  Waits are bounded; a wait that gives up
+// expansion).  Needs N + k <= 32.  Waits are bounded; a wait that gives up
 // records kErrTimeout, drains what this warp started and stops.
-constexpr int kNfWarps = 8;
+#ifndef MOE_NF_WARPS
+#define MOE_NF_WARPS 8
+#endif
+#ifndef MOE_NF_XBUFS
+#define MOE_NF_XBUFS 2
+#endif
+#ifndef MOE_NF_RBUFS
+#define MOE_NF_RBUFS 2
+#endif
+#ifndef MOE_NF_CHUNK
+#define MOE_NF_CHUNK 2048
+#endif
+constexpr int kNfWarps = MOE_NF_WARPS;
 constexpr int kNfThreads = kNfWarps * 32;
-
+constexpr int kNfX = MOE_NF_XBUFS;  // x-chunk ring stages per warp
+constexpr int kNfR = MOE_NF_RBUFS;  // staging read-back buffers per warp
+constexpr uint32_t kNfChunk = MOE_NF_CHUNK;
+static_assert(kNfX >= 2 && kNfX < 31 && kNfR >= 1 && kNfR <= 8, "node dispatch ring shape");
+static_assert(kNfChunk % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char* xbuf = smem + (size_t)warp * 3 * a.chunk;  // X[0], X[1]
-    unsigned char* rbuf = xbuf + 2 * (size_t)a.chunk;         // R
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kNfWarps * 3 * a.chunk) + warp * 3;
+    const size_t per_warp = (size_t)(kNfX + kNfR) * a.chunk;
+    unsigned char* xbuf = smem + (size_t)warp * per_warp;  // X[kNfX]
+    unsigned char* rbuf = xbuf + (size_t)kNfX * a.chunk;    // R[kNfR]
+    // bar[s] for s < kNfX: x stage s; bar[kNfX]: the read-back buffers
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (size_t)kNfWarps * per_warp) + warp * (kNfX + 1);
+    constexpr uint32_t kRb = 1u << kNfX;  // parity / in-flight bit of the read-back
     if (lane == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+        for (int i = 0; i <= kNfX; ++i) mbar_init(&bar[i], 1);
         fence_barrier_init();
     }
     __syncwarp();
@@ -298,7 +314,8 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
         const int64_t left = a.row_bytes - off;
         bytes = left < (int64_t)a.chunk ? (uint32_t)left : a.chunk;
     };
-    auto issue_x = [&](int64_t q, int b) {
+    auto issue_x = [&](int64_t q) {
+        const int b = (int)(q % kNfX);
         int64_t t, off;
         uint32_t bytes;
         geometry(q, t, off, bytes);
@@ -307,10 +324,10 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
             bulk_load(xbuf + (size_t)b * a.chunk, a.src + t * a.row_bytes + off, bytes, &bar[b]);
         }
     };
-    uint32_t parity = 0, inflight = 0;  // bits 0, 1: X buffers; bit 2: R
-    if (mine > 0) {
-        issue_x(0, 0);
-        inflight |= 1u;
+    uint32_t parity = 0, inflight = 0;
+    for (int64_t q = 0; q < kNfX - 1 && q < mine; ++q) {
+        issue_x(q);
+        inflight |= 1u << q;
     }
     if (early) pdl_wait();
 
@@ -332,7 +349,7 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
     int64_t srow = -1;
     bool failed = false;
     for (int64_t q = 0; q < mine && !failed; ++q) {
-        const int b = (int)(q & 1);
+        const int b = (int)(q % kNfX);
         int64_t t, off;
         uint32_t bytes;
         geometry(q, t, off, bytes);
@@ -371,44 +388,64 @@ __global__ void __launch_bounds__(kNfThreads) node_dispatch_kernel(BulkArgs a) {
         // 2. one staging row per node touched
         if (srow >= 0) bulk_store(a.staging + srow * a.row_bytes + off, xbuf + (size_t)b * a.chunk, bytes);
         bulk_commit();
-        // the other X buffer was last read by the previous item's staging
-        // stores: free once all but the newest group have been read
+        // the previous item's x stage was last read by its staging stores:
+        // free once all but the newest group have been read
         bulk_wait_read<1>();
         __syncwarp();
-        if (q + 1 < mine) {
-            issue_x(q + 1, b ^ 1);
-            inflight |= 1u << (b ^ 1);
+        if (q + kNfX - 1 < mine) {
+            issue_x(q + kNfX - 1);
+            inflight |= 1u << ((q + kNfX - 1) % kNfX);
         }
         // 3. the staging rows are complete before they are read back
         if (stager) bulk_wait_all();
         __syncwarp();
         unsigned touched = __ballot_sync(kFullMask, srow >= 0);  // bit 31 - n: node n
-        while (touched) {
-            const int hb = 31 - __clz(touched);  // highest set bit: lowest node first
-            touched &= ~(1u << hb);
-            const int n = 31 - hb;
-            const int64_t row_n = __shfl_sync(kFullMask, srow, hb);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bar[2], bytes);
-                bulk_load(rbuf, a.staging + row_n * a.row_bytes + off, bytes, &bar[2]);
+        while (touched && !failed) {
+            // up to kNfR nodes, lowest first, read back together
+            int node[kNfR];
+            int64_t row_n[kNfR];
+            int nb = 0;
+#pragma unroll
+            for (int i = 0; i < kNfR; ++i) {
+                node[i] = -1;
+                row_n[i] = 0;
+                if (touched) {
+                    const int hb = 31 - __clz(touched);
+                    touched &= ~(1u << hb);
+                    node[i] = 31 - hb;
+                    row_n[i] = __shfl_sync(kFullMask, srow, hb);
+                    ++nb;
+                }
             }
-            inflight |= 4u;
-            if (!__all_sync(kFullMask, mbar_wait(&bar[2], (parity >> 2) & 1u))) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bar[kNfX], bytes * (uint32_t)nb);
+#pragma unroll
+                for (int i = 0; i < kNfR; ++i)
+                    if (i < nb)
+                        bulk_load(rbuf + (size_t)i * a.chunk, a.staging + row_n[i] * a.row_bytes + off,
+                                  bytes, &bar[kNfX]);
+            }
+            inflight |= kRb;
+            if (!__all_sync(kFullMask, mbar_wait(&bar[kNfX], (parity & kRb) ? 1u : 0u))) {
                 failed = true;
                 break;
             }
-            parity ^= 4u;
-            inflight &= ~4u;
-            if (lane < a.k && sl >= 0 && nj == n)
-                bulk_store(a.dst + (int64_t)sl * a.row_bytes + off, rbuf, bytes);
+            parity ^= kRb;
+            inflight &= ~kRb;
+            if (lane < a.k && sl >= 0) {
+#pragma unroll
+                for (int i = 0; i < kNfR; ++i)
+                    if (i < nb && nj == node[i])
+                        bulk_store(a.dst + (int64_t)sl * a.row_bytes + off, rbuf + (size_t)i * a.chunk, bytes);
+            }
             bulk_commit();
-            bulk_wait_read<0>();  // R is free for the next node
+            bulk_wait_read<0>();  // the read-back buffers are free for the next nodes
             __syncwarp();
         }
     }
     if (failed) {
         errbits |= kErrTimeout;
-        for (int i = 0; i < 3; ++i)
+        for (int i = 0; i <= kNfX; ++i)
             if (inflight & (1u << i)) (void)mbar_wait(&bar[i], (parity >> i) & 1u);
     }
     if (a.late_trigger) pdl_trigger();
@@ -600,12 +637,12 @@ bool node_dispatch_eligible(const RowMoveParams& p) { return p.N + p.k <= 32; }
 
 cudaError_t launch_node_dispatch_bulk(const RowMoveParams& p, const void* x, void* staging,
                                       int64_t staging_rows, void* recv, cudaStream_t stream) {
-    BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kDispChunk);
+    BulkArgs a = bulk_args(p, x, recv, p.T, p.T * p.k, kNfChunk);
     a.staging = static_cast<char*>(staging);
     a.staging_rows = staging_rows;
     const int64_t items = p.T * a.cpr;
     if (items <= 0) return cudaSuccess;
-    const size_t smem = (size_t)kNfWarps * 3 * (a.chunk + sizeof(uint64_t));
+    const size_t smem = (size_t)kNfWarps * ((kNfX + kNfR) * (size_t)a.chunk + (kNfX + 1) * sizeof(uint64_t));
     cudaError_t e = cudaFuncSetAttribute(node_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;

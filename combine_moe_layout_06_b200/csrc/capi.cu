@@ -11,7 +11,7 @@ using moe::layout_params;
 
 constexpr uint32_t kKnownFlags = MOE_FLAG_TWO_LEVEL | MOE_FLAG_COPY_VECTOR | MOE_FLAG_COPY_BULK |
                                  MOE_FLAG_LAYOUT_CLUSTER | MOE_FLAG_LAYOUT_FUSED |
-                                 MOE_FLAG_TWO_LEVEL_FUSED;
+                                 MOE_FLAG_TWO_LEVEL_FUSED | MOE_FLAG_TWO_LEVEL_SPLIT;
 
 moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -65,7 +65,7 @@ moe_status_t dispatch_impl(const moe_config_t* c, const moe_layout_t* L, const v
     p.early_inputs = early;
     if (!two_level(c)) return cuda_status(moe::launch_dispatch_flat(p, x, recv, s));
     const int64_t rows = staging_rows(c);
-    if ((c->flags & MOE_FLAG_TWO_LEVEL_FUSED) != 0 && p.engine != CopyEngine::kVector &&
+    if ((c->flags & MOE_FLAG_TWO_LEVEL_SPLIT) == 0 && p.engine != CopyEngine::kVector &&
         moe::bulk_eligible(p.row_bytes, {x, node_staging, recv}) && moe::node_dispatch_eligible(p))
         return cuda_status(moe::launch_node_dispatch_bulk(p, x, node_staging, rows, recv, s));
     cudaError_t e = moe::launch_node_pack(p, x, node_staging, rows, s);

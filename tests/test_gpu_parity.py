@@ -20,6 +20,7 @@ VEC = capi.MOE_FLAG_COPY_VECTOR
 BULK = capi.MOE_FLAG_COPY_BULK
 CL = capi.MOE_FLAG_LAYOUT_CLUSTER
 ONE = capi.MOE_FLAG_TWO_LEVEL_FUSED
+SPLIT = capi.MOE_FLAG_TWO_LEVEL_SPLIT
 CANARY = 0x7F81          # a signalling-NaN bf16 pattern no dispatched row holds
 
 SMALL = [
@@ -65,11 +66,12 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
     eo = inputs.random_bf16_bits((T * k, H), seed=T * k + H)
     y_ref = oracle_mod.combine(eo, w, ref["slot"])
     x_dev = M.to_dev(x)
-    # TWO: pack + expansion; TWO | ONE: one kernel (node staging, then the
-    # staging row read back) where N + k <= 32 and rows are 16-byte multiples
+    # TWO: one kernel (node staging, then the staging row read back) where
+    # N + k <= 32 and rows are 16-byte multiples, else pack + expansion;
+    # TWO | SPLIT and TWO | VEC: pack + expansion
     runs = [(f, True) for f in (0, TWO, VEC, TWO | VEC, BULK, TWO | BULK, TWO | ONE,
-                                TWO | ONE | BULK)]
-    runs += [(f, False) for f in (TWO, TWO | VEC, TWO | BULK)]   # pair-walking expansion
+                                TWO | SPLIT, TWO | SPLIT | BULK)]
+    runs += [(f, False) for f in (TWO | SPLIT, TWO | VEC, TWO | SPLIT | BULK)]   # pair-walking expansion
     for flags, node_src in runs:
         cfg = M.cfg_of(T, H, E, k, R, N, flags)
         lay, _ = M.gpu_layout(cfg, topk, node_src=node_src)
@@ -115,7 +117,7 @@ def test_large_batch_multi_kernel_layout(oracle_mod, T):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
-@pytest.mark.parametrize("engine", [0, VEC, BULK, ONE, ONE | BULK])
+@pytest.mark.parametrize("engine", [0, VEC, BULK, ONE, SPLIT, SPLIT | BULK])
 @pytest.mark.parametrize("hot_frac", [0.0, 0.9, 1.0])
 def test_skewed_node_loads(oracle_mod, engine, hot_frac):
     """One hot node (up to every token on node 0, the other nodes empty): the
@@ -290,14 +292,16 @@ def test_workload_forced_engine(oracle_mod, name, engine):
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
-def test_workload_two_level_one_kernel(oracle_mod):
-    """The one-kernel two-level dispatch on the DeepSeek-V3-shaped workload
-    at full size: staging rows and receive rows as the oracle has them."""
+@pytest.mark.parametrize("form", [ONE, SPLIT])
+def test_workload_two_level_forms(oracle_mod, form):
+    """Both two-level dispatch forms (one kernel; pack then expansion) on the
+    DeepSeek-V3-shaped workload at full size: staging rows and receive rows
+    as the oracle has them."""
     d = inputs.make("dsv3")
     wl = d["workload"]
     x, topk = d["x"], d["topk_idx"]
     ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
-    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, TWO | ONE)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, TWO | form)
     lay, _ = M.gpu_layout(cfg, topk)
     x_dev = M.to_dev(x)
     recv, staging = M.gpu_dispatch(cfg, lay, x_dev)
