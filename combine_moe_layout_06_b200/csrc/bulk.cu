@@ -264,11 +264,19 @@ __global__ void __launch_bounds__(kBulkThreads) dispatch_bulk_kernel(BulkArgs a)
 // the receive rows end up exactly as with the two-kernel form (pack, then
 // expansion).  Needs N + k <= 32.  Waits are bounded; a wait that gives up
 // records kErrTimeout, drains what this warp started and stops.
+// Ring shape (compile-time tunables).  4 warps of 6 x stages and 2
+// read-back buffers of 2 KB (64 KB per CTA) was the best of a sweep over
+// 4-16 warps, 2-8 stages, 1-4 read-back buffers and 1-2 KB chunks on the
+// DeepSeek-V3-shaped workload (step 736 us, against 750 us for 8 warps of 2
+// stages and 759 us with one read-back buffer).
 #ifndef MOE_NF_WARPS
-#define MOE_NF_WARPS 8
+#define MOE_NF_WARPS 4
 #endif
 #ifndef MOE_NF_XBUFS
-#define MOE_NF_XBUFS 2
+#define MOE_NF_XBUFS 6
+#endif
+#ifndef MOE_NF_IPW
+#define MOE_NF_IPW 4
 #endif
 #ifndef MOE_NF_RBUFS
 #define MOE_NF_RBUFS 2
@@ -646,7 +654,7 @@ cudaError_t launch_node_dispatch_bulk(const RowMoveParams& p, const void* x, voi
     cudaError_t e = cudaFuncSetAttribute(node_dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = persistent_grid<node_dispatch_kernel>(items, kNfThreads, smem);
+    const int grid = persistent_grid<node_dispatch_kernel>(items, kNfThreads, smem, MOE_NF_IPW);
     a.late_trigger =
         pdl_trigger_at_end(grid, resident_blocks<node_dispatch_kernel>(kNfThreads, smem)) ? 1 : 0;
     return launch_pdl(node_dispatch_kernel, dim3(grid), dim3(kNfThreads), smem, stream, a);

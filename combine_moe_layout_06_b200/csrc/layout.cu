@@ -74,20 +74,17 @@ struct LayoutArgs {
     int* node_slot;
     int* node_src;  // [U] staging row -> token, or nullptr
     int* err;
-    // the assign kernel copies the whole [E][C] (and [N][C]) histogram into
-    // shared memory with bulk copies (16-byte aligned workspace, small enough)
+    // the count kernel writes its histograms chunk-major ([C][E], [C][N])
+    // and the assign kernel copies them whole into shared memory with bulk
+    // copies (16-byte aligned workspace, small enough); otherwise they are
+    // expert-major ([E][C], [N][C]) and read from global memory
     bool bulk_hist;
+    bool vec_routes;  // k % 4 == 0 and topk 16-byte aligned: 16-byte route loads
+    bool vec_slots;   // k % 4 == 0 and slot 16-byte aligned: 16-byte slot stores
 };
 
-// Histogram bytes the assign kernel copies into shared memory at most, and
-// the fewest chunks for which it does: up to 32 chunks one round of plain
-// loads reads the histogram as fast (measured on B200: the olmoe layout, 16
-// chunks, took 7.0 us with the copy and 6.6 us without; dsv3, 64 chunks,
-// 16.4 us against 22.5 us).
+// Histogram bytes the assign kernel copies into shared memory at most.
 constexpr size_t kBulkHistMaxBytes = 128 * 1024;
-#ifndef MOE_BULK_HIST_MIN_CHUNKS
-#define MOE_BULK_HIST_MIN_CHUNKS 33
-#endif
 __host__ __device__ inline size_t round16(size_t v) { return (v + 15) / 16 * 16; }
 
 template <int KMAX>
@@ -95,7 +92,9 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs 
     extern __shared__ __align__(16) int smem[];
     int* s_cnt = smem;           // [E]
     int* s_ncnt = smem + a.E;    // [N]
+    unsigned char* s_node = reinterpret_cast<unsigned char*>(smem + a.E + a.N);  // [E] (nodes)
     for (int i = threadIdx.x; i < a.E + a.N; i += blockDim.x) smem[i] = 0;
+    if (a.nodes) fill_node_table(s_node, a.part, a.E);
     pdl_wait();
     pdl_trigger();
     __syncthreads();
@@ -104,12 +103,12 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs 
     int bits = 0;
     if (t < a.T) {
         int e[KMAX];
-        bits = load_route<KMAX>(a.topk, t, a.k, a.E, e);
+        bits = load_route<KMAX>(a.topk, t, a.k, a.E, e, a.vec_routes);
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)
             if (e[j] >= 0) atomicAdd(&s_cnt[e[j]], 1);
         if (a.nodes) {
-            uint32_t m = node_mask<KMAX>(a.part, e);
+            uint32_t m = node_mask<KMAX>(s_node, e);
             while (m) {
                 const int n = __ffs(m) - 1;
                 m &= m - 1;
@@ -119,11 +118,20 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_count_kernel(LayoutArgs 
     }
     warp_report(a.err, bits);
     __syncthreads();
-    for (int i = threadIdx.x; i < a.E; i += blockDim.x)
-        a.cnt[(int64_t)i * a.C + blockIdx.x] = s_cnt[i];
-    if (a.nodes)
-        for (int i = threadIdx.x; i < a.N; i += blockDim.x)
-            a.ncnt[(int64_t)i * a.C + blockIdx.x] = s_ncnt[i];
+    if (a.bulk_hist) {
+        // this chunk's counts as one contiguous row of the [C][E] matrix
+        for (int i = threadIdx.x; i < a.E; i += blockDim.x)
+            a.cnt[(int64_t)blockIdx.x * a.E + i] = s_cnt[i];
+        if (a.nodes)
+            for (int i = threadIdx.x; i < a.N; i += blockDim.x)
+                a.ncnt[(int64_t)blockIdx.x * a.N + i] = s_ncnt[i];
+    } else {
+        for (int i = threadIdx.x; i < a.E; i += blockDim.x)
+            a.cnt[(int64_t)i * a.C + blockIdx.x] = s_cnt[i];
+        if (a.nodes)
+            for (int i = threadIdx.x; i < a.N; i += blockDim.x)
+                a.ncnt[(int64_t)i * a.C + blockIdx.x] = s_ncnt[i];
+    }
 }
 
 // In-place exclusive scan of data[0..L) by one block: each thread owns a
@@ -302,10 +310,14 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
     const int words = 2 * kLayoutWarps * E + kLayoutWarps * N;
     const size_t hist_e = round16(sizeof(int) * (size_t)E * C);
     const size_t hist_n = a.nodes ? round16(sizeof(int) * (size_t)N * C) : 0;
-    // the copied histograms start at the next 16-byte boundary
+    // the copied histograms start at the next 16-byte boundary, then the
+    // mbarrier (16 bytes kept), then the table of each expert's node
     int* s_hist = smem + assign_scan_hist_offset(E, N);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(s_hist) + hist_e + hist_n);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(s_hist) +
+                                                (a.bulk_hist ? hist_e + hist_n : 0));
+    unsigned char* s_node = reinterpret_cast<unsigned char*>(bar + 2);
     for (int i = threadIdx.x; i < words; i += blockDim.x) s_wcnt[i] = 0;
+    if (a.nodes) fill_node_table(s_node, a.part, E);
     if (a.bulk_hist && threadIdx.x == 0) {
         mbar_init(bar, 1);
         fence_barrier_init();
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
     for (int j = 0; j < KMAX; ++j) e[j] = -1;
     uint32_t nm = 0;
     if (t < a.T) {
-        load_route<KMAX>(a.topk, t, a.k, E, e);  // errors were reported by count
+        load_route<KMAX>(a.topk, t, a.k, E, e, a.vec_routes);  // errors were reported by count
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)
             if (e[j] >= 0) {
@@ -328,7 +340,7 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
                 atomicOr(&s_mask[warp * E + e[j]], 1u << lane);
             }
         if (a.nodes) {
-            nm = node_mask<KMAX>(a.part, e);
+            nm = node_mask<KMAX>(s_node, e);
             uint32_t m = nm;
             while (m) {
                 const int n = __ffs(m) - 1;
@@ -373,37 +385,21 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
             __syncthreads();
             return;
         }
+        // thread i: expert (or node) i's column of the [C][E] ([C][N])
+        // matrix, the chunks before this CTA's, then the rest
         const int* h_n = reinterpret_cast<const int*>(reinterpret_cast<const char*>(s_hist) + hist_e);
         const int cta = (int)blockIdx.x;
-        for (int i0 = warp * 4; i0 < EN; i0 += kLayoutWarps * 4) {
-            int sum[4], pre[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                sum[r] = 0;
-                pre[r] = 0;
-                const int i = i0 + r;
-                if (i < EN) {
-                    const int* row = i < E ? s_hist + (size_t)i * C : h_n + (size_t)(i - E) * C;
-                    for (int c = lane; c < C; c += 32) {
-                        const int v = row[c];
-                        sum[r] += v;
-                        pre[r] += c < cta ? v : 0;
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                sum[r] = __reduce_add_sync(kFullMask, sum[r]);
-                pre[r] = __reduce_add_sync(kFullMask, pre[r]);
-            }
-            if (lane == 0) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    if (i0 + r < EN) {
-                        tot[i0 + r] = sum[r];
-                        base[i0 + r] = pre[r];
-                    }
-            }
+        for (int i = threadIdx.x; i < EN; i += blockDim.x) {
+            const int* col = i < E ? s_hist + i : h_n + (i - E);
+            const int stride = i < E ? E : N;
+            int pre = 0, c = 0;
+#pragma unroll 4
+            for (; c < cta; ++c) pre += col[c * stride];
+            int sum = pre;
+#pragma unroll 4
+            for (; c < C; ++c) sum += col[c * stride];
+            tot[i] = sum;
+            base[i] = pre;
         }
     } else if (C <= 32) {
         const int64_t nall = (int64_t)EN * C;
@@ -512,16 +508,25 @@ __global__ void __launch_bounds__(kTokensPerCta) layout_assign_scan_kernel(Layou
     const unsigned lt = lanemask_lt();
     if (t < a.T) {
         int* out = a.slot + t * a.k;
+        int sl[KMAX];
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-            if (j < a.k) {
-                int sl = -1;
-                if (e[j] >= 0) {
-                    const int idx = warp * E + e[j];
-                    sl = s_wcnt[idx] + __popc(s_mask[idx] & lt);
-                }
-                out[j] = sl;
+            sl[j] = -1;
+            if (e[j] >= 0) {
+                const int idx = warp * E + e[j];
+                sl[j] = s_wcnt[idx] + __popc(s_mask[idx] & lt);
             }
+        }
+        if (a.vec_slots) {
+#pragma unroll
+            for (int q = 0; q < KMAX / 4; ++q)
+                if (4 * q < a.k)
+                    *reinterpret_cast<int4*>(out + 4 * q) =
+                        make_int4(sl[4 * q], sl[4 * q + 1], sl[4 * q + 2], sl[4 * q + 3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < KMAX; ++j)
+                if (j < a.k) out[j] = sl[j];
         }
     }
     if (a.nodes) {
@@ -712,15 +717,16 @@ template <int KMAX>
 cudaError_t launch_layout_k(const LayoutArgs& a, cudaStream_t stream) {
     cudaError_t err;
     if (a.C > 0) {
-        const size_t smem = sizeof(int) * (size_t)(a.E + a.N);
+        const size_t smem = sizeof(int) * (size_t)(a.E + a.N) + (a.nodes ? (size_t)a.E : 0);
         err = launch_pdl(layout_count_kernel<KMAX>, dim3(a.C), dim3(kTokensPerCta), smem, stream, a);
         if (err != cudaSuccess) return err;
     }
     if (a.C > 0 && a.C <= kFusedScanMaxChunks) {
-        size_t smem = sizeof(int) * (size_t)assign_scan_hist_offset(a.E, a.N);
+        size_t smem = sizeof(int) * (size_t)assign_scan_hist_offset(a.E, a.N) + 2 * sizeof(uint64_t) +
+                      (a.nodes ? (size_t)a.E : 0);
         if (a.bulk_hist)
             smem += round16(sizeof(int) * (size_t)a.E * a.C) +
-                    (a.nodes ? round16(sizeof(int) * (size_t)a.N * a.C) : 0) + sizeof(uint64_t);
+                    (a.nodes ? round16(sizeof(int) * (size_t)a.N * a.C) : 0);
         if (smem > 48 * 1024) {
             err = cudaFuncSetAttribute(layout_assign_scan_kernel<KMAX>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -873,8 +879,13 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
         const size_t bytes = round16(sizeof(int) * (size_t)p.E * a.C) +
                              (p.nodes ? round16(sizeof(int) * (size_t)p.N * a.C) : 0);
         a.bulk_hist = reinterpret_cast<uintptr_t>(p.workspace) % 16 == 0 &&
-                      bytes <= kBulkHistMaxBytes && a.C >= MOE_BULK_HIST_MIN_CHUNKS;
+                      bytes <= kBulkHistMaxBytes && a.C <= kFusedScanMaxChunks;
+#ifdef MOE_LAYOUT_NO_BULK_HIST
+        a.bulk_hist = false;
+#endif
     }
+    a.vec_routes = p.k % 4 == 0 && reinterpret_cast<uintptr_t>(p.topk) % 16 == 0;
+    a.vec_slots = p.k % 4 == 0 && reinterpret_cast<uintptr_t>(p.slot) % 16 == 0;
     // One chunk of tokens (T <= 256): one CTA sees every token, so the
     // single-cluster kernel (a cluster of one CTA) does the whole layout in one
     // launch, with no count kernel and no kernel boundary before the ranks.

@@ -49,13 +49,27 @@ __device__ __forceinline__ int check_route(const int (&raw)[KMAX], int k, int E,
 
 // Load token t's k expert ids from global memory (all k loads issued before
 // any is examined, so they are in flight together) and validate them.
+// vec4: k % 4 == 0 and topk 16-byte aligned, so the row is read as 16-byte
+// vectors.
 template <int KMAX>
 __device__ __forceinline__ int load_route(const int* __restrict__ topk, int64_t t, int k, int E,
-                                          int (&e)[KMAX]) {
+                                          int (&e)[KMAX], bool vec4 = false) {
     const int* row = topk + t * k;
     int raw[KMAX];
+    if (vec4) {
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) raw[j] = j < k ? ld_dep(row + j) : -1;
+        for (int q = 0; q < KMAX / 4; ++q) {
+            int4 v = make_int4(-1, -1, -1, -1);
+            if (4 * q < k) v = ld_dep4(row + 4 * q);
+            raw[4 * q] = v.x;
+            raw[4 * q + 1] = v.y;
+            raw[4 * q + 2] = v.z;
+            raw[4 * q + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) raw[j] = j < k ? ld_dep(row + j) : -1;
+    }
     return check_route<KMAX>(raw, k, E, e);
 }
 
@@ -66,6 +80,20 @@ __device__ __forceinline__ uint32_t node_mask(const Partition& part, const int (
     for (int j = 0; j < KMAX; ++j)
         if (e[j] >= 0) m |= 1u << part.node_of(e[j]);
     return m;
+}
+
+// The same from a shared-memory table of each expert's node (built once per
+// CTA with fill_node_table), instead of two integer divisions per route.
+template <int KMAX>
+__device__ __forceinline__ uint32_t node_mask(const unsigned char* node_of, const int (&e)[KMAX]) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+        if (e[j] >= 0) m |= 1u << node_of[e[j]];
+    return m;
+}
+__device__ __forceinline__ void fill_node_table(unsigned char* node_of, const Partition& part, int E) {
+    for (int i = threadIdx.x; i < E; i += blockDim.x) node_of[i] = (unsigned char)part.node_of(i);
 }
 
 // Exclusive scan of one value per thread over the whole block; also returns

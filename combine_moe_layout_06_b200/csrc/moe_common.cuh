@@ -72,6 +72,13 @@ __device__ __forceinline__ int ld_dep(const int* p) {
     asm volatile("ld.global.s32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
+__device__ __forceinline__ int4 ld_dep4(const int* p) {  // 16-byte aligned
+    int4 v;
+    asm volatile("ld.global.v4.s32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
 __device__ __forceinline__ float ld_dep(const float* p) {
     float v;
     asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p));
