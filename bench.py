@@ -474,7 +474,8 @@ class StepBench:
         self.with_decoupled = "decoupled" in extras
         self.with_agrs = "agrs" in extras and wl.R <= capi.MOE_MAX_NODES
         self.with_fp8 = "fp8" in extras and wl.H % 8 == 0
-        self.with_ep = "ep" in extras and wl.R <= capi.MOE_MAX_NODES and not wl.two_level
+        # sharded sources are flat (one NVSwitch domain), also for a two-level workload
+        self.with_ep = "ep" in extras and wl.R <= capi.MOE_MAX_NODES
 
         # Expert parallelism over sharded sources with every rank on this
         # GPU: rank g routes tokens [sb[g], sb[g+1]); its receive and
@@ -1251,6 +1252,9 @@ def parse_args(argv=None):
     p.add_argument("--ref-tokens", type=int, default=0)
     p.add_argument("--hbm-probe", action="store_true",
                    help="measure write-only / read-only / copy HBM bandwidth and exit")
+    p.add_argument("--ep-processes", action="store_true",
+                   help="time the multi-process expert-parallel step even on one GPU (a process "
+                        "group of one rank; torchrun with several GPUs always takes it)")
     args = p.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     return args
@@ -1271,13 +1275,23 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    several = world > 1 or args.ep_processes
+    if several:
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            if "MASTER_PORT" not in os.environ:
+                import socket
+                with socket.socket() as sk:
+                    sk.bind(("127.0.0.1", 0))
+                    os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     ctx = Ctx(world, rank, local, dev)
     try:
-        return run_several(args, ctx) if world > 1 else run_one(args, ctx)
+        return run_several(args, ctx) if several else run_one(args, ctx)
     finally:
-        if world > 1:
+        if several:
             dist.destroy_process_group()
 
 

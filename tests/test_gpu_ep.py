@@ -228,3 +228,27 @@ def test_ep_two_processes_ipc():
         assert ok_recv, f"receive buffer of rank {rank}"
         assert ok_y, f"combine of rank {rank}"
         assert err == capi.MOE_OK
+
+
+def test_bench_multi_process_step_as_one_rank():
+    """bench.py's multi-process expert-parallel step (what `--gpus N` runs under
+    torchrun), taken by a process group of one rank on this GPU: local layout,
+    NCCL count all-gather, sharded-source layout, dispatch into and combine
+    from the ranks' buffers, NCCL barriers between the phases.  It must run
+    without a device error and report every routed row as received."""
+    import json
+    import subprocess
+    import sys
+    M.ensure_lib()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    T = 1024
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--ep-processes",
+                          "--workload", "olmoe", "--tokens", str(T), "--steps", "4", "--warmup", "3",
+                          "--e2e-steps", "2"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert res.returncode == 0, res.stderr[-3000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    wl = inputs.WORKLOADS["olmoe"]
+    assert line["n_gpus"] == 1 and line["value"] > 0
+    assert line["expert_parallel"]["receive_rows"] == [T * wl.k]
+    assert line["e2e"]["h2d_bytes_per_step"] == T * wl.H * 2 + T * wl.k * 8
+    assert line["replicas"]["value"] > 0
