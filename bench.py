@@ -1111,6 +1111,7 @@ def ep_shuffle(args, ctx, d):
     ctx.barrier()
     del recv_peers, eo_peers, recv_ptrs, eo_ptrs
     torch.cuda.synchronize()
+    torch.cuda.ipc_collect()
     ctx.barrier()
     return out
 

@@ -56,7 +56,7 @@ ENTRY_POINTS = (
     "moe_layout_noalloc", "moe_layout_dispatch", "moe_dispatch_allgather",
     "moe_combine_reducescatter", "moe_quantize_rows_fp8", "moe_dispatch_fp8", "moe_combine_fp8",
     "moe_ep_layout", "moe_ep_dispatch", "moe_ep_combine", "moe_dispatch_fp8_two_level",
-    "moe_ep_receive_rows",
+    "moe_ep_receive_rows", "moe_enable_peer_access",
 )
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -127,6 +127,7 @@ def lib() -> ctypes.CDLL:
     L.moe_ep_dispatch.argtypes = [C, LP, EP, P, PP, ctypes.c_int64, P]
     L.moe_ep_combine.argtypes = [C, LP, EP, PP, ctypes.c_int64, P, P, P]
     L.moe_ep_receive_rows.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P]
+    L.moe_enable_peer_access.argtypes = [ctypes.c_int32, ctypes.c_int32]
     for name in ENTRY_POINTS[1:]:
         getattr(L, name).restype = S
     _lib = L
@@ -272,6 +273,11 @@ def moe_ep_receive_rows(counts_all, num_ranks: int):
                                      c.ctypes.data_as(ctypes.c_void_p), out),
            "moe_ep_receive_rows")
     return list(out)[: int(num_ranks)]
+
+
+def moe_enable_peer_access(device: int, peer_device: int) -> None:
+    """Let kernels on `device` reach memory on `peer_device` (host call)."""
+    _check(lib().moe_enable_peer_access(int(device), int(peer_device)), "moe_enable_peer_access")
 
 
 def moe_ep_dispatch(cfg: MoeConfig, local: MoeLayout, ep: MoeEpLayout, x, recv_bufs,

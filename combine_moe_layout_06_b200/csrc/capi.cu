@@ -380,6 +380,27 @@ moe_status_t moe_ep_receive_rows(int32_t num_experts, int32_t num_ranks, int32_t
     return MOE_OK;
 }
 
+moe_status_t moe_enable_peer_access(int32_t device, int32_t peer_device) {
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (device < 0 || peer_device < 0 || device >= n || peer_device >= n || device == peer_device)
+        return MOE_ERR_INVALID_ARG;
+    int can = 0;
+    if (cudaDeviceCanAccessPeer(&can, device, peer_device) != cudaSuccess || !can) return MOE_ERR_CUDA;
+    int prev = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess || cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaError_t e = cudaDeviceEnablePeerAccess(peer_device, 0);
+    if (e == cudaErrorPeerAccessAlreadyEnabled) {
+        cudaGetLastError();  // an enabled pair is what was asked for
+        e = cudaSuccess;
+    }
+    const cudaError_t back = cudaSetDevice(prev);
+    return e == cudaSuccess && back == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status_t moe_ep_layout(const moe_config_t* c, int32_t g, int32_t G, const int32_t* topk_idx,
                            const int32_t* counts_all, const moe_layout_t* L,
                            const moe_ep_layout_t* ep, void* stream) {

@@ -881,7 +881,7 @@ cudaError_t launch_layout(const LayoutParams& p, cudaStream_t stream) {
         a.bulk_hist = reinterpret_cast<uintptr_t>(p.workspace) % 16 == 0 &&
                       bytes <= kBulkHistMaxBytes && a.C <= kFusedScanMaxChunks;
 #ifdef MOE_LAYOUT_NO_BULK_HIST
-        a.bulk_hist = false;
+        a.bulk_hist = false;  // build-time switch: the expert-major path everywhere (A/B timing)
 #endif
     }
     a.vec_routes = p.k % 4 == 0 && reinterpret_cast<uintptr_t>(p.topk) % 16 == 0;

@@ -42,20 +42,28 @@ def receive_rows(counts_all, num_ranks: int) -> np.ndarray:
 
 def share_buffer(t: torch.Tensor, group=None) -> list:
     """Device addresses of every rank's `t` (same shape on every rank), as
-    usable from this process: this rank's own address, and the peers'
-    through CUDA IPC mappings of their storages.  The returned list keeps the
-    mapped storages alive (second element of each pair)."""
+    usable from this process's kernels: this rank's own address, and the
+    peers' through CUDA IPC mappings of their storages.  A peer on another
+    GPU is opened in that GPU's context, so peer access from this rank's GPU
+    to it is enabled too (moe_enable_peer_access); a pair of GPUs that cannot
+    reach each other raises here, before any kernel touches peer memory.
+    The returned list keeps the mapped storages alive (second element of each
+    pair)."""
     storage = t.untyped_storage()
     handle = storage._share_cuda_()
     offset = t.storage_offset() * t.element_size()
     handles = [None] * dist.get_world_size(group)
     dist.all_gather_object(handles, (handle, offset), group=group)
     me = dist.get_rank(group)
+    mine = t.device.index
     out = []
     for r, (h, off) in enumerate(handles):
         if r == me:
             out.append((t.data_ptr(), t))
         else:
+            peer_dev = int(h[0])   # the device the peer's storage lives on
+            if peer_dev != mine:
+                capi.moe_enable_peer_access(mine, peer_dev)
             peer = torch.UntypedStorage._new_shared_cuda(*h)
             out.append((peer.data_ptr() + off, peer))
     return out

@@ -187,9 +187,11 @@ moe_status_t moe_layout_workspace_bytes(const moe_config_t *cfg, size_t *bytes);
 /* Rows a node staging buffer must hold for cfg: T * min(N, k). */
 moe_status_t moe_node_staging_rows(const moe_config_t *cfg, int64_t *rows);
 
-/* Layout: per-expert histogram, exclusive scan in expert-major/chunk-minor
- * order, and stable slot assignment (FUSCO article, "FUSCO 的核心创新":
- * the segment descriptors that drive gather-send / scatter-recv).
+/* Layout: per-expert histograms of 256-token chunks, an exclusive scan over
+ * experts and chunks (expert e's first row in chunk c is expert_offsets[e]
+ * plus e's rows in chunks before c), and stable slot assignment (FUSCO
+ * article, "FUSCO 的核心创新": the segment descriptors that drive
+ * gather-send / scatter-recv).
  *   topk_idx  device int32 [T*k], row-major [T][k], the router's choices
  *   layout    device arrays as described above (TWO_LEVEL: node arrays too)
  * Data errors go to layout->error_word. */
@@ -361,6 +363,16 @@ typedef struct moe_ep_layout {
  * num_ranks. */
 moe_status_t moe_ep_receive_rows(int32_t num_experts, int32_t num_ranks, int32_t num_sources,
                                  const int32_t *counts_all, int64_t *rows_out);
+
+/* Let kernels that run on `device` load from and store to memory that
+ * lives on `peer_device`: another rank's receive and expert-output buffers,
+ * mapped into this process (e.g. CUDA IPC handles opened by the caller).
+ * Host call; nothing is enqueued, and the calling thread's current device is
+ * restored.  Enabling a pair that is already enabled is not an error.
+ * Errors: MOE_ERR_INVALID_ARG for a device index out of range or device ==
+ * peer_device; MOE_ERR_CUDA when the two devices cannot reach each other
+ * (or no device is present). */
+moe_status_t moe_enable_peer_access(int32_t device, int32_t peer_device);
 
 /* Step 3.  cfg: this rank's shard (as in step 1); source_rank g in
  * [0, num_sources); counts_all: device int32 [num_sources][E] with row g equal

@@ -115,3 +115,14 @@ def test_argument_refusals_touch_no_device(lib):
     assert capi.moe_get_error(empty, stream=0) == capi.MOE_ERR_INVALID_ARG
     for s in range(9):
         assert capi.moe_status_string(s).startswith("MOE_")
+
+
+def test_enable_peer_access_without_a_device(lib):
+    """With no GPU visible the host call reports MOE_ERR_CUDA and changes
+    nothing (the refusals of bad device pairs are checked on a GPU)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is visible here")
+    with pytest.raises(capi.MoeError) as ei:
+        capi.moe_enable_peer_access(0, 1)
+    assert ei.value.status == capi.MOE_ERR_CUDA

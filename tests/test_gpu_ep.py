@@ -252,3 +252,19 @@ def test_bench_multi_process_step_as_one_rank():
     assert line["expert_parallel"]["receive_rows"] == [T * wl.k]
     assert line["e2e"]["h2d_bytes_per_step"] == T * wl.H * 2 + T * wl.k * 8
     assert line["replicas"]["value"] > 0
+
+
+def test_enable_peer_access_refusals_and_pairs():
+    """moe_enable_peer_access: a device paired with itself or an index
+    beyond the visible devices is refused up front; where two GPUs are
+    visible, enabling a pair twice is fine."""
+    M.ensure_lib()
+    n = torch.cuda.device_count()
+    for dev, peer in ((0, 0), (0, n), (-1, 0)):
+        with pytest.raises(capi.MoeError) as ei:
+            capi.moe_enable_peer_access(dev, peer)
+        assert ei.value.status == capi.MOE_ERR_INVALID_ARG
+    if n >= 2 and torch.cuda.can_device_access_peer(0, 1):
+        capi.moe_enable_peer_access(0, 1)
+        capi.moe_enable_peer_access(0, 1)
+    assert torch.cuda.current_device() == 0

@@ -97,6 +97,34 @@ def test_dispatch_and_combine_small(oracle_mod, T, H, E, k, R, N):
         assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
+@pytest.mark.parametrize("T,E,k,R,N,shift", [
+    (10240, 1024, 8, 8, 4, 0),    # histograms of 160 KB: read from global memory, 40 chunks
+    (7000, 256, 8, 8, 2, 4),      # workspace off a 16-byte boundary, 28 chunks
+    (60000, 256, 8, 8, 2, 4),     # workspace off a 16-byte boundary, 235 chunks
+    (33 * 256, 96, 6, 6, 3, 0),   # 33 chunks, k not a multiple of 4 (scalar routes and slots)
+])
+def test_layout_histogram_paths(oracle_mod, T, E, k, R, N, shift):
+    """The assign kernel's histogram paths: copied whole into shared memory
+    (chunk-major, the default for 16-byte aligned workspaces up to 128 KB of
+    histograms), or read from global memory (expert-major) when the
+    histograms are larger or the workspace is not 16-byte aligned, with
+    up to 32 chunks and beyond.  Each matches the oracle bit for bit."""
+    d = inputs.make_random(T, 8, E, k, seed=T + E)
+    topk = d["topk_idx"]
+    ref = oracle_mod.layout(topk, E, R, N, nodes=True)
+    for flags in (0, TWO):
+        cfg = M.cfg_of(T, 8, E, k, R, N, flags)
+        lay = M.buffers.DeviceLayout(cfg)
+        ws = torch.zeros(capi.moe_layout_workspace_bytes(cfg) + 16, dtype=torch.uint8, device="cuda")
+        struct = capi.layout_struct(lay.expert_counts, lay.expert_offsets, lay.rank_offsets, lay.slot,
+                                    lay.error_word, ws.data_ptr() + shift, lay.node_counts,
+                                    lay.node_offsets, lay.node_slot, lay.node_src)
+        capi.moe_layout(cfg, torch.from_numpy(topk).cuda(), struct)
+        want = ref if flags else {k_: v for k_, v in ref.items() if not k_.startswith("node")}
+        M.assert_layout_equal(lay.host(), want)
+        assert capi.moe_get_error(struct) == capi.MOE_OK
+
+
 @pytest.mark.parametrize("T", [40000, 140001])
 def test_large_batch_multi_kernel_layout(oracle_mod, T):
     """Above 16384 tokens the layout runs as count + assign kernels over a
