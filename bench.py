@@ -396,7 +396,7 @@ def node_balance(args, ctx):
     for v in (False, True):
         for name, fn in (("LD", ld), ("L", lo)):
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
                 fn(A, v)
                 fn(B, v)
             graphs[(name, v)] = g
@@ -702,7 +702,7 @@ class StepBench:
 
         def capture(fn, n):
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
                 for i in range(n):
                     fn(self.sets[i % 2])
             return g
