@@ -78,6 +78,8 @@ def measured_peak():
 
 # Steps per CUDA graph replay in the timed loops.
 GRAPH_STEPS = 10
+# Fewest timed steps of each per-workload entry.
+PER_WORKLOAD_MIN_STEPS = 100
 
 KERNEL_SOURCES = {
     "combine": ["combine.cu", "moe_common.cuh"],
@@ -880,7 +882,11 @@ class StepBench:
                 "kernels_ms": {"dispatch": round(raw["fp8_LD"] - t_l, 5),
                                "combine": round(fp8_ms / K - raw["fp8_LD"], 5)},
                 "bytes_per_step": fp8_bytes,
-                "path": ("layout + fp8 two-level dispatch (quantize once into node staging, "
+                "path": ("layout + fp8 two-level dispatch (each row quantized once, its codes and "
+                         "scale staged once per node touched, read back from L2 and expanded to "
+                         "the node's receive rows, one kernel; staging not credited) + "
+                         if wl.two_level and not self.args.two_level_split else
+                         "layout + fp8 two-level dispatch (quantize once into node staging, then "
                          "expand codes and scales; staging not credited) + " if wl.two_level else
                          "layout + fp8 dispatch (quantize once, k copies of e4m3 codes + scale) + ")
                         + "fp8 combine (expert rows already e4m3)"}
@@ -1183,11 +1189,16 @@ def run_one(args, ctx):
     names = [] if args.no_per_workload else [n for n in (args.per_workload.split(",")
                                                          if args.per_workload else WORKLOAD_ORDER)
                                              if n and n != args.workload]
+    # the other workloads are extra entries, timed over at least PER_WORKLOAD_MIN_STEPS
+    # steps (the headline keeps exactly K): a few hundred microseconds of steps
+    # would leave one disturbance too much weight
+    K_pw = max(K, PER_WORKLOAD_MIN_STEPS)
     for name in names:
         pd = workload_inputs(name)
         sb = StepBench(ctx, args, pd, extras=[] if args.no_decoupled else ["decoupled"])
         sb.prepare(args.warmup)
-        per[name] = sb.report(sb.measure(K, flushed=False), K)
+        per[name] = sb.report(sb.measure(K_pw, flushed=False), K_pw)
+        per[name]["steps"] = K_pw
         sb.release()
         del sb
 

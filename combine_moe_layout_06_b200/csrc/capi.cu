@@ -504,6 +504,12 @@ moe_status_t moe_dispatch_fp8_two_level(const moe_config_t* c, const moe_layout_
     if (!moe::fp8_eligible(c->hidden, {x}, {staging_q, recv_q})) return MOE_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t rows = staging_rows(c);
+    if ((c->flags & MOE_FLAG_TWO_LEVEL_SPLIT) == 0) {
+        const moe::RowMoveParams p = move_params(c, L);
+        if (moe::fp8_node_dispatch_eligible(p, c->hidden, {x, staging_q, recv_q}))
+            return cuda_status(moe::launch_fp8_node_dispatch(p, x, c->hidden, staging_q, staging_scale,
+                                                             rows, recv_q, recv_scale, s));
+    }
     // phase 1: each token quantized once, into the staging row of every node it touches
     cudaError_t e = moe::launch_quantize_fp8(x, c->num_tokens, c->hidden, L->node_slot, c->num_nodes,
                                              rows, staging_q, staging_scale, L->error_word, s,

@@ -15,6 +15,14 @@
 //    token's k receive rows (fp8 dispatch: quantize once, write k copies).
 //  quantize_fp8_kernel (any H % 8 == 0): the same with two passes over the
 //    row (amax, then convert) and 8-byte code stores.
+//  quantize_node_dispatch_kernel (two-level, H % 16 == 0, H <= 8192,
+//    N + k <= 32): one warp per token quantizes its row once (row in
+//    registers, as above), stores the codes and scale to the token's
+//    staging row on every node it touches, then reads each staging row back
+//    (from L2: the same lane's own bytes, ld.global.cg) and stores it to the
+//    token's receive rows on that node.  The FUSCO article's forwarding
+//    ("负载均衡与跨节点去重": a token crosses to a node once, then fans out
+//    inside it) in one launch instead of a quantizer and two expansions.
 //  combine_ring_fp8_kernel (H % 16 == 0, k <= 8) and combine_fp8_kernel
 //    (any H % 8 == 0, k <= 32): the fused combine on codes, coef_j = w[t][j]
 //    * scale[slot[t][j]] and acc = fma(coef_j, decode(code), acc) for j = 0
@@ -23,6 +31,8 @@
 //    registers would hold; the code widening (e4m3 -> f16 -> f32 conversions)
 //    then bounds it.
 #include <cuda_fp8.h>
+
+#include <climits>
 
 #include "moe_kernels.h"
 
@@ -203,6 +213,170 @@ __global__ void __launch_bounds__(W * 32) quantize_rows16_kernel(Fp8Args a) {
             }
         }
     }
+    warp_report(a.err, errbits);
+}
+
+// One-kernel fp8 two-level dispatch (see the file comment).
+struct Fp8NodeArgs {
+    const uint4* src;        // bf16 x rows, 8 values per vector
+    int64_t T;
+    int k, N, ranks_per_node;
+    int64_t G;               // 16-value groups per row
+    const int* slot;         // [T*k]
+    const int* node_slot;    // [T*N]
+    const int* node_offsets; // [N+1]
+    const int* rank_offsets; // [R+1]
+    uint4* staging_q;        // [staging_rows][G] 16-code groups
+    float* staging_s;
+    int64_t staging_rows;
+    uint4* recv_q;           // [recv_rows][G]
+    float* recv_s;
+    int64_t recv_rows;
+    int* err;
+    int late_trigger;        // let the dependent grid launch at the end (pdl_trigger_at_end)
+};
+
+__device__ __forceinline__ uint4 ld_l2(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_l2(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+template <int NG, int W>
+__global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeArgs a) {
+    if (!a.late_trigger) pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int N = a.N;
+    // node n: lane n holds its receive-row range [lo, hi); lane 31 - n its
+    // first staging row
+    int n_lo = INT_MAX, n_hi = INT_MIN, n_first = 0;
+    if (lane < N) {
+        n_lo = ld_dep(a.rank_offsets + lane * a.ranks_per_node);
+        n_hi = ld_dep(a.rank_offsets + (lane + 1) * a.ranks_per_node);
+    }
+    const bool stager = lane >= 32 - N;
+    const int my_node = 31 - lane;
+    if (stager) n_first = ld_dep(a.node_offsets + my_node);
+    const int64_t G = a.G;
+    const int64_t nw = (int64_t)gridDim.x * W;
+    int errbits = 0;
+    for (int64_t t = (int64_t)blockIdx.x * W + (threadIdx.x >> 5); t < a.T; t += nw) {
+        // column j's receive row and its node; node n's staging row
+        int sl = -1, nj = -1;
+        int64_t srow = -1;
+        if (lane < a.k) {
+            const int s = ld_dep(a.slot + t * a.k + lane);
+            if (s >= 0 && s < a.recv_rows) sl = s;
+            else if (s != -1) errbits |= kErrBadLayout;
+        }
+        for (int n = 0; n < N; ++n) {
+            const int lo = __shfl_sync(kFullMask, n_lo, n);
+            const int hi = __shfl_sync(kFullMask, n_hi, n);
+            if (sl >= lo && sl < hi) nj = n;
+        }
+        if (sl >= 0 && nj < 0) errbits |= kErrBadLayout;
+        if (stager) {
+            const int ns = ld_dep(a.node_slot + t * N + my_node);
+            if (ns >= 0) {
+                const int64_t r = (int64_t)n_first + ns;
+                if (r >= 0 && r < a.staging_rows) srow = r;
+                else errbits |= kErrBadLayout;
+            }
+        }
+        // the row, held in registers: lane l owns 16-value groups l, l+32, ...
+        const uint4* src = a.src + t * 2 * G;
+        uint4 raw[NG][2];
+#pragma unroll
+        for (int i = 0; i < NG; ++i) {
+            const int64_t g = lane + 32 * i;
+            raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
+            if (g < G) {
+                raw[i][0] = ld_stream(src + 2 * g);
+                raw[i][1] = ld_stream(src + 2 * g + 1);
+            }
+        }
+        // amax as quantize_rows16_kernel finds it (NaNs have no magnitude)
+        uint32_t m2 = 0;
+        auto fold = [&](uint32_t w) {
+            const uint32_t x = w & 0x7FFF7FFFu;
+            m2 = __vmaxu2(m2, x & ~__vcmpgtu2(x, 0x7F807F80u));
+        };
+#pragma unroll
+        for (int i = 0; i < NG; ++i)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                fold(raw[i][h].x);
+                fold(raw[i][h].y);
+                fold(raw[i][h].z);
+                fold(raw[i][h].w);
+            }
+        uint32_t amax_bits = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+        amax_bits = __reduce_max_sync(kFullMask, amax_bits);
+        const float amax = __uint_as_float(amax_bits);
+        const float inv = amax > 0.f ? 448.0f / amax : 1.0f;
+        const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+        // 1. codes and scale into the staging row of every node touched
+        if (srow >= 0) a.staging_s[srow] = scale;
+        const unsigned smask = __ballot_sync(kFullMask, srow >= 0);  // bit 31 - n: node n
+#pragma unroll
+        for (int i = 0; i < NG; ++i) {
+            uint2 c[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float f[8];
+                unpack_bf16<uint4>(raw[i][h], f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
+                c[h] = to_e4m3x8(f);
+            }
+            const uint4 code = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+            const int64_t g = lane + 32 * i;
+            unsigned m = smask;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int64_t d = __shfl_sync(kFullMask, srow, j);
+                if (g < G) a.staging_q[d * G + g] = code;
+            }
+        }
+        __syncwarp();  // the staging scales are seen by the lanes that read them back
+        // 2. each staging row read back and stored to the node's receive rows
+        unsigned m = smask;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            const int n = 31 - j;
+            const int64_t row_n = __shfl_sync(kFullMask, srow, j);
+            const unsigned cols = __ballot_sync(kFullMask, sl >= 0 && nj == n);
+            if ((cols >> lane) & 1u) a.recv_s[sl] = ld_l2(a.staging_s + row_n);
+            uint4 back[NG];
+#pragma unroll
+            for (int i = 0; i < NG; ++i) {
+                const int64_t g = lane + 32 * i;
+                back[i] = g < G ? ld_l2(a.staging_q + row_n * G + g) : make_uint4(0, 0, 0, 0);
+            }
+            unsigned cm = cols;
+            while (cm) {
+                const int q = __ffs(cm) - 1;
+                cm &= cm - 1;
+                const int64_t d = __shfl_sync(kFullMask, (int64_t)sl, q);
+#pragma unroll
+                for (int i = 0; i < NG; ++i) {
+                    const int64_t g = lane + 32 * i;
+                    if (g < G) st_stream(a.recv_q + d * G + g, back[i]);
+                }
+            }
+        }
+    }
+    if (a.late_trigger) pdl_trigger();
     warp_report(a.err, errbits);
 }
 
@@ -467,6 +641,51 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, c
     constexpr auto kern = quantize_fp8_kernel;
     const int grid = persistent_grid<kern>(rows, kThreads);
     return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
+namespace {
+template <int NG, int W>
+cudaError_t launch_node_q(Fp8NodeArgs a, cudaStream_t stream) {
+    constexpr auto kern = quantize_node_dispatch_kernel<NG, W>;
+    const int grid = persistent_grid<kern>(a.T, W * 32);
+    a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<kern>(W * 32)) ? 1 : 0;
+    return launch_pdl(kern, dim3(grid), dim3(W * 32), 0, stream, a);
+}
+}  // namespace
+
+bool fp8_node_dispatch_eligible(const RowMoveParams& p, int64_t hidden, std::initializer_list<const void*> ptrs) {
+    uintptr_t bits = 0;
+    for (const void* q : ptrs) bits |= reinterpret_cast<uintptr_t>(q);
+    return hidden % 16 == 0 && hidden <= 512 * 16 && p.N + p.k <= 32 && bits % 16 == 0;
+}
+
+cudaError_t launch_fp8_node_dispatch(const RowMoveParams& p, const void* x, int64_t hidden,
+                                     void* staging_q, float* staging_scale, int64_t staging_rows,
+                                     void* recv_q, float* recv_scale, cudaStream_t stream) {
+    if (p.T <= 0) return cudaSuccess;
+    Fp8NodeArgs a;
+    a.src = static_cast<const uint4*>(x);
+    a.T = p.T;
+    a.k = p.k;
+    a.N = p.N;
+    a.ranks_per_node = p.ranks_per_node;
+    a.G = hidden / 16;
+    a.slot = p.slot;
+    a.node_slot = p.node_slot;
+    a.node_offsets = p.node_offsets;
+    a.rank_offsets = p.rank_offsets;
+    a.staging_q = static_cast<uint4*>(staging_q);
+    a.staging_s = staging_scale;
+    a.staging_rows = staging_rows;
+    a.recv_q = static_cast<uint4*>(recv_q);
+    a.recv_s = recv_scale;
+    a.recv_rows = p.T * p.k;
+    a.err = p.err;
+    a.late_trigger = 0;
+    if (hidden <= 512 * 2) return launch_node_q<2, 8>(a, stream);
+    if (hidden <= 512 * 4) return launch_node_q<4, 8>(a, stream);
+    if (hidden <= 512 * 8) return launch_node_q<8, 8>(a, stream);
+    return launch_node_q<16, 4>(a, stream);
 }
 
 cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,

@@ -139,6 +139,16 @@ bool fp8_eligible(int64_t hidden, std::initializer_list<const void*> bf16_ptrs,
 cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, const int* slot, int k,
                                 int64_t dst_rows, void* q, float* scale, int* err,
                                 cudaStream_t stream, const int* dst_base = nullptr);
+// Two-level fp8 dispatch in one kernel: each x row quantized once, its codes
+// and scale stored to its staging row on every node touched, then each
+// staging row read back and stored to the token's receive rows on that
+// node.  Needs H % 16 == 0, H <= 8192, N + k <= 32 and 16-byte aligned x,
+// staging and receive code buffers.
+bool fp8_node_dispatch_eligible(const RowMoveParams& p, int64_t hidden,
+                                std::initializer_list<const void*> ptrs);
+cudaError_t launch_fp8_node_dispatch(const RowMoveParams& p, const void* x, int64_t hidden,
+                                     void* staging_q, float* staging_scale, int64_t staging_rows,
+                                     void* recv_q, float* recv_scale, cudaStream_t stream);
 // y[t] = bf16_rne(sum_j fma(w[t][j] * scale[slot], decode(q[slot]), .))
 cudaError_t launch_combine_fp8(const CombineParams& p, const void* q, const float* scale, void* y,
                                cudaStream_t stream);

@@ -126,17 +126,22 @@ def test_fp8_workload_olmoe(oracle_mod):
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
+@pytest.mark.parametrize("form", [0, capi.MOE_FLAG_TWO_LEVEL_SPLIT])
 @pytest.mark.parametrize("node_src", [True, False])
 @pytest.mark.parametrize("T,H,E,k,R,N", [
-    (33, 136, 13, 4, 5, 5),
+    (33, 136, 13, 4, 5, 5),         # H % 16 != 0: the split form whatever the flag
     (257, 2048, 64, 8, 4, 2),
-    (600, 7168, 32, 8, 8, 4),       # beyond the register-resident quantizer
+    (600, 7168, 32, 8, 8, 4),       # 14 groups of 16 values per lane
+    (300, 8192, 64, 16, 16, 16),    # N + k = 32, the one-kernel limit
 ])
-def test_fp8_two_level(oracle_mod, T, H, E, k, R, N, node_src):
+def test_fp8_two_level(oracle_mod, T, H, E, k, R, N, node_src, form):
+    """Both fp8 two-level forms (one kernel: quantize, stage, read back,
+    expand; split: quantizer then two expansions) give the oracle's staging
+    and receive codes and scales."""
     d = inputs.make_random(T, H, E, k, seed=T + N)
     x, topk = d["x"], d["topk_idx"]
     ref = oracle_mod.layout(topk, E, R, N, nodes=True)
-    cfg = M.cfg_of(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL)
+    cfg = M.cfg_of(T, H, E, k, R, N, capi.MOE_FLAG_TWO_LEVEL | form)
     lay, _ = M.gpu_layout(cfg, topk, node_src=node_src)
     rows = capi.moe_node_staging_rows(cfg)
     st_q = torch.full((rows, H), 0x55, dtype=torch.uint8, device="cuda")
@@ -154,6 +159,35 @@ def test_fp8_two_level(oracle_mod, T, H, E, k, R, N, node_src):
     assert np.array_equal(st_s.cpu().numpy()[:U], xs[ref["node_src"]])
     assert np.all(_u8(st_q)[U:] == 0x55)
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
+@pytest.mark.parametrize("form", [0, capi.MOE_FLAG_TWO_LEVEL_SPLIT])
+def test_fp8_two_level_dsv3_workload(oracle_mod, form):
+    """The DeepSeek-V3-shaped workload at full size through the fp8
+    two-level dispatch: receive codes and scales as the oracle's fp8
+    dispatch, staging rows as its quantizer of the staged tokens."""
+    d = inputs.make("dsv3")
+    wl = d["workload"]
+    x, topk = d["x"], d["topk_idx"]
+    ref = oracle_mod.layout(topk, wl.E, wl.R, wl.N, nodes=True)
+    cfg = M.cfg_of(wl.T, wl.H, wl.E, wl.k, wl.R, wl.N, capi.MOE_FLAG_TWO_LEVEL | form)
+    lay, _ = M.gpu_layout(cfg, topk)
+    rows = capi.moe_node_staging_rows(cfg)
+    st_q = torch.empty((rows, wl.H), dtype=torch.uint8, device="cuda")
+    st_s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    recv_q = torch.empty((wl.T * wl.k, wl.H), dtype=torch.uint8, device="cuda")
+    recv_s = torch.empty(wl.T * wl.k, dtype=torch.float32, device="cuda")
+    capi.moe_dispatch_fp8_two_level(cfg, lay.struct, M.to_dev(x), st_q, st_s, recv_q, recv_s)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+    rq, rs = oracle_mod.dispatch_fp8(x, ref["slot"])
+    assert np.array_equal(_u8(recv_q), rq)
+    assert np.array_equal(recv_s.cpu().numpy(), rs)
+    del recv_q
+    xq, xs = oracle_mod.quantize_rows_fp8(x)
+    U = int(ref["node_offsets"][-1])
+    assert np.array_equal(_u8(st_q)[:U], xq[ref["node_src"]])
+    assert np.array_equal(st_s.cpu().numpy()[:U], xs[ref["node_src"]])
+    torch.cuda.empty_cache()
 
 
 def test_fp8_refusals():
