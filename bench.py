@@ -518,7 +518,9 @@ class StepBench:
                 self.cap = int(ep_rows.max())
 
         class BufferSet:
-            """One independent set of the step's inputs and outputs."""
+            """One independent set of the step's inputs and outputs (the
+            comparison paths' buffers are added by extras(), once both sets'
+            step buffers exist)."""
 
             def __init__(self):
                 self.lay = buffers.DeviceLayout(cfg, dev)
@@ -531,6 +533,8 @@ class StepBench:
                 self.staging = None
                 if wl.two_level:
                     self.staging = torch.empty((capi.moe_node_staging_rows(cfg), wl.H), **bf16)
+
+            def extras(self):
                 if outer.with_decoupled:
                     self.dlay = buffers.DeviceLayout(dcfg, dev)
                     rows = capi.moe_node_staging_rows(dcfg)
@@ -556,6 +560,8 @@ class StepBench:
                 self.ep = EpShards(self) if outer.with_ep else None
 
         self.sets = [BufferSet(), BufferSet()]
+        for b in self.sets:
+            b.extras()
         self.ep_streams = [torch.cuda.Stream(dev) for _ in range(G)] if self.with_ep else []
 
         # one cluster launch when asked for, and always for one chunk of 256 tokens
