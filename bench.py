@@ -1184,13 +1184,6 @@ def run_one(args, ctx):
     main.release()
     del main
 
-    balance = None
-    if not args.no_node_balance:
-        with ClockSampler(ctx.local) as nb_clocks:
-            balance = node_balance(args, ctx)
-        balance["clocks"] = nb_clocks.summary()
-        torch.cuda.empty_cache()
-
     per = {}
     names = [] if args.no_per_workload else [n for n in (args.per_workload.split(",")
                                                          if args.per_workload else WORKLOAD_ORDER)
@@ -1207,6 +1200,13 @@ def run_one(args, ctx):
         per[name]["steps"] = K_pw
         sb.release()
         del sb
+
+    balance = None
+    if not args.no_node_balance:
+        with ClockSampler(ctx.local) as nb_clocks:
+            balance = node_balance(args, ctx)
+        balance["clocks"] = nb_clocks.summary()
+        torch.cuda.empty_cache()
 
     cpu = cpu_par = None
     if ctx.rank == 0 and not args.no_cpu_baseline:

@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace moe {
 
 // Device error-word bits (moe_layout_t.error_word).
@@ -332,19 +334,31 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
-// Resident blocks per SM of a kernel at a block size (queried once per
-// kernel).
+// Resident blocks per SM of a kernel at a block size and dynamic shared
+// memory size, queried once per (kernel, threads, smem) and cached: a
+// kernel's shared memory can depend on the row size (its chunk), so one
+// process may launch it at several sizes.
 template <auto Kernel>
 inline int blocks_per_sm(int threads, size_t smem = 0) {
-    static int cached = 0;
-    if (cached == 0) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
-            n < 1)
-            n = 1;
-        cached = n;
+    struct Entry {
+        int threads;
+        size_t smem;
+        int blocks;
+    };
+    constexpr int kSlots = 16;
+    static Entry cache[kSlots] = {};
+    static int used = 0;
+    static std::mutex lock;
+    std::lock_guard<std::mutex> guard(lock);
+    for (int i = 0; i < used; ++i)
+        if (cache[i].threads == threads && cache[i].smem == smem) return cache[i].blocks;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1;
     }
-    return cached;
+    cache[used < kSlots ? used++ : kSlots - 1] = Entry{threads, smem, n};
+    return n;
 }
 
 // Blocks of a kernel resident on the whole device at once.
