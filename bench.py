@@ -113,6 +113,22 @@ def profiled_traffic(stage, workload):
     return None
 
 
+def roofline_entry(kernel, achieved, peak, peak_src, ms, traffic):
+    """The line's roofline object: algorithmic bytes per launch over the
+    kernel's measured time against the measured copy peak; with the
+    kernel's DRAM traffic per launch (ncu) known, also that traffic over the
+    same time (what the kernel really moves, e.g. a two-level dispatch's
+    staging writes, which the algorithmic bytes do not credit)."""
+    out = {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
+           "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+           "peak_kind": f"{peak_src} copy bandwidth"}
+    if traffic:
+        moved = traffic / (ms * 1e-3) / 1e9
+        out["traffic_gbs"] = round(moved, 2)
+        out["traffic_frac"] = round(moved / peak, 4)
+    return out
+
+
 def max_over_ranks(value, world, device):
     """The largest value over all ranks (each rank passes its own)."""
     if world <= 1:
@@ -853,11 +869,9 @@ class StepBench:
                             "combine": round(t_combine, 5),
                             # combines alone, back to back (layouts from the warm-up)
                             "combine_alone": round(raw["C"], 5)}),
-            "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": round(achieved, 2),
-                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": profiled_traffic(dom_kernel, wl.name if wl.T == inputs.WORKLOADS[wl.name].T
-                                                     else "none"),
-                         "peak_kind": f"{peak_src} copy bandwidth"},
+            "roofline": roofline_entry(dom_kernel, achieved, peak, peak_src, dom_ms,
+                                       profiled_traffic(dom_kernel, wl.name if wl.T == inputs.WORKLOADS[wl.name].T
+                                                        else "none")),
             "clocks": raw["clocks"],
             "step_bytes": step_bytes,
         }

@@ -429,8 +429,12 @@ moe_status_t moe_dispatch_fp8(const moe_config_t *cfg, const moe_layout_t *layou
 /* Two-level dispatch with an fp8 payload (MOE_FLAG_TWO_LEVEL required):
  * each x row is quantized once, into the staging row of every node it
  * touches (codes and scale, as moe_dispatch() stages bf16 rows), and the
- * node expansion then copies codes and scales to the receive rows.  Results
- * equal moe_dispatch_fp8() on the same layout bit for bit.
+ * node expansion then copies codes and scales to the receive rows.  With
+ * H % 16 == 0, H <= 8192, N + k <= 32 and 16-byte aligned x and code
+ * buffers one kernel does both phases (each staging row read back from L2
+ * right after it is written); MOE_FLAG_TWO_LEVEL_SPLIT or other shapes take
+ * a quantizer and two expansion kernels.  Results equal moe_dispatch_fp8()
+ * on the same layout bit for bit.
  *   staging_q      device uint8 [moe_node_staging_rows()][H]
  *   staging_scale  device fp32 [moe_node_staging_rows()]
  *   recv_q, recv_scale  as for moe_dispatch_fp8() */
