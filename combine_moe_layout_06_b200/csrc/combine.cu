@@ -19,6 +19,12 @@
 // while the current chunk's rows are in flight.  The chunk of up to KB
 // expert rows is loaded before any FMA, so KB*VPL streaming loads per lane
 // are in flight at once.
+//
+// Large grids (many resident waves of items) take the paired form: lane l
+// owns vectors 2l and 2l+1 of the chunk and moves both with one 32-byte load
+// or store (sm_100's 256-bit global accesses), which halves the load
+// instructions per byte in flight.  The arithmetic is the same; only which
+// lane holds which element changes.
 #include "moe_kernels.h"
 
 namespace moe {
@@ -41,6 +47,13 @@ constexpr int kThreads = kWarpsPerCta * 32;
 // items per warp in each wave of a large combine (see persistent_grid)
 #ifndef MOE_COMBINE_IPW
 #define MOE_COMBINE_IPW 4
+#endif
+// Resident waves from which the paired (32-byte) form is used; 0 = never.
+// Measured on B200: it shortens the 16-wave combines (DeepSeek-V3-shaped
+// 325 -> 315 us alone, long-context 211 -> 204 us) and lengthens the 1-wave
+// OLMoE-shaped one (24.1 -> 26.0 us); qwen3's 4-wave step was no faster.
+#ifndef MOE_COMBINE_PAIR_WAVES
+#define MOE_COMBINE_PAIR_WAVES 8
 #endif
 
 struct CombArgs {
@@ -100,8 +113,23 @@ __device__ __forceinline__ void load_route(const CombArgs& a, int64_t t, int lan
     }
 }
 
-template <typename V, int VPL, int KB, bool EP = false>
+// 32 contiguous bytes (two 16-byte vectors) in one access; p 32-byte aligned.
+__device__ __forceinline__ void ld_stream_pair(const uint4* p, uint4& u, uint4& v) {
+    asm volatile("ld.global.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w), "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+}
+__device__ __forceinline__ void st_pair(uint4* p, const uint4& u, const uint4& v) {
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(u.x), "r"(u.y),
+                 "r"(u.z), "r"(u.w), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// PAIR (V = uint4, VPL = 2, rv even, expert rows and y 32-byte aligned):
+// lane l holds vectors 2l, 2l+1 of the chunk instead of l, l+32.
+template <typename V, int VPL, int KB, bool EP = false, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
+    static_assert(!PAIR || (sizeof(V) == 16 && VPL == 2 && !EP), "paired form: 16-byte vectors, 2 per lane");
     constexpr int EPV = VecInfo<V>::kElems;
     constexpr int CHUNK = 32 * VPL;
     if (!a.late_trigger) pdl_trigger();
@@ -151,9 +179,13 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
                     if (ok[q]) {
                         const V* row = EP ? reinterpret_cast<const V*>(rj) + base
                                           : eo + (int64_t)sj * a.rv + base;
+                        if constexpr (PAIR) {
+                            if (base + 2 * lane < a.rv) ld_stream_pair(row + 2 * lane, v[q][0], v[q][1]);
+                        } else {
 #pragma unroll
-                        for (int i = 0; i < VPL; ++i)
-                            if (base + i * 32 + lane < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
+                            for (int i = 0; i < VPL; ++i)
+                                if (base + i * 32 + lane < a.rv) v[q][i] = ld_stream(row + i * 32 + lane);
+                        }
                     }
                 }
 #pragma unroll
@@ -161,7 +193,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
                     if (!ok[q]) continue;
 #pragma unroll
                     for (int i = 0; i < VPL; ++i) {
-                        if (base + i * 32 + lane < a.rv) {
+                        if (PAIR ? base + 2 * lane < a.rv : base + i * 32 + lane < a.rv) {
                             float f[EPV];
                             unpack_bf16<V>(v[q][i], f);
 #pragma unroll
@@ -171,9 +203,13 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
                 }
             }
             V* yrow = y + t * a.rv + base;
+            if constexpr (PAIR) {
+                if (base + 2 * lane < a.rv) st_pair(yrow + 2 * lane, pack_bf16<V>(acc[0]), pack_bf16<V>(acc[1]));
+            } else {
 #pragma unroll
-            for (int i = 0; i < VPL; ++i)
-                if (base + i * 32 + lane < a.rv) yrow[i * 32 + lane] = pack_bf16<V>(acc[i]);
+                for (int i = 0; i < VPL; ++i)
+                    if (base + i * 32 + lane < a.rv) yrow[i * 32 + lane] = pack_bf16<V>(acc[i]);
+            }
             if (last_chunk) {
                 s = s_next;
                 wl = w_next;
@@ -189,13 +225,27 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombArgs a) {
     warp_report(a.err, errbits);
 }
 
+template <auto Kern>
+cudaError_t launch_combine_grid(CombArgs a, int64_t items, cudaStream_t stream) {
+    const int grid = persistent_grid<Kern>(items, kThreads, 0, MOE_COMBINE_IPW);
+    a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<Kern>(kThreads)) ? 1 : 0;
+    return launch_pdl(Kern, dim3(grid), dim3(kThreads), 0, stream, a);
+}
+
 template <typename V, int VPL, int KB, bool EP>
 cudaError_t launch_combine_v(CombArgs a, cudaStream_t stream) {
     constexpr auto kern = combine_kernel<V, VPL, KB, EP>;
     const int64_t cpr = (a.rv + 32 * VPL - 1) / (32 * VPL);
-    const int grid = persistent_grid<kern>(a.T * cpr, kThreads, 0, MOE_COMBINE_IPW);
-    a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<kern>(kThreads)) ? 1 : 0;
-    return launch_pdl(kern, dim3(grid), dim3(kThreads), 0, stream, a);
+    const int64_t items = a.T * cpr;
+    if constexpr (!EP && VPL == 2 && sizeof(V) == 16) {
+        constexpr auto paired = combine_kernel<V, VPL, KB, EP, true>;
+        const uintptr_t align = reinterpret_cast<uintptr_t>(a.eo) | reinterpret_cast<uintptr_t>(a.y);
+        const int64_t wave_items = (int64_t)resident_blocks<paired>(kThreads) * kWarpsPerCta * MOE_COMBINE_IPW;
+        if (MOE_COMBINE_PAIR_WAVES > 0 && a.rv % 2 == 0 && align % 32 == 0 &&
+            items >= (int64_t)MOE_COMBINE_PAIR_WAVES * wave_items)
+            return launch_combine_grid<paired>(a, items, stream);
+    }
+    return launch_combine_grid<kern>(a, items, stream);
 }
 
 template <typename V, int VPL, bool EP = false>

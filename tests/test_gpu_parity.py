@@ -376,6 +376,26 @@ def test_workload_combine(oracle_mod, name):
     assert capi.moe_get_error(lay.struct) == capi.MOE_OK
 
 
+@pytest.mark.parametrize("H", [1040, 1520, 1032])
+def test_combine_many_waves_ragged_chunks(oracle_mod, H):
+    """Combines of at least 8 resident waves of (token, 1 KB chunk) items take
+    the 32-byte-per-lane form when the row has an even number of 16-byte
+    vectors: rows ending 2 (H = 1040) and 62 (H = 1520) vectors into their
+    last chunk.  An odd vector count (H = 1032) keeps the 16-byte form at the
+    same size.  Bit for bit against the oracle."""
+    T, E, k, R = 50001, 32, 4, 4
+    _, topk, w = _small_inputs(T, 8, E, k, seed=H)
+    ref = oracle_mod.layout(topk, E, R)
+    eo = inputs.random_bf16_bits((T * k, H), seed=H + 1)
+    cfg = M.cfg_of(T, H, E, k, R)
+    lay, _ = M.gpu_layout(cfg, topk)
+    y = M.bits(M.gpu_combine(cfg, lay, M.to_dev(eo), w))
+    y_ref = oracle_mod.combine(eo, w, ref["slot"])
+    M.assert_combine_close(y, y_ref)
+    assert np.array_equal(y, y_ref)
+    assert capi.moe_get_error(lay.struct) == capi.MOE_OK
+
+
 # ---------------------------------------------------------------- decoupled
 
 @pytest.mark.parametrize("name", NAMES)
