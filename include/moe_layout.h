@@ -249,7 +249,11 @@ moe_status_t moe_layout_dispatch(const moe_config_t *cfg, const int32_t *topk_id
  * token's owner; the order and precision are this library's choice).
  *   expert_out    device bf16 [T*k][H], receive-buffer layout
  *   topk_weights  device fp32 [T][k], used as given
- *   y             device bf16 [T][H] */
+ *   y             device bf16 [T][H]
+ * Large combines (at least 8 resident waves of (token, 1 KB row chunk) work
+ * items) whose rows are a multiple of 32 bytes, with expert_out and y 32-byte
+ * aligned, move 32 bytes per lane per access (sm_100's 256-bit loads and
+ * stores); the results are the same bit for bit either way. */
 moe_status_t moe_combine(const moe_config_t *cfg, const moe_layout_t *layout,
                          const void *expert_out, const float *topk_weights,
                          void *y, void *stream);
