@@ -249,8 +249,44 @@ __device__ __forceinline__ float ld_l2(const float* p) {
     return v;
 }
 
-template <int NG, int W>
+// 32 contiguous bytes per lane in one access (sm_100's 256-bit loads and
+// stores); p 32-byte aligned.
+__device__ __forceinline__ void ld_stream_pair(const uint4* p, uint4& u, uint4& v) {
+    asm volatile("ld.global.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w), "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+}
+__device__ __forceinline__ void ld_l2_pair(const uint4* p, uint4& u, uint4& v) {
+    asm volatile("ld.global.cg.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w), "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+}
+__device__ __forceinline__ void st_pair(uint4* p, const uint4& u, const uint4& v) {
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(u.x), "r"(u.y),
+                 "r"(u.z), "r"(u.w), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void st_stream_pair(uint4* p, const uint4& u, const uint4& v) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(u.x), "r"(u.y),
+                 "r"(u.z), "r"(u.w), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// PAIR (G even; x, staging and receive codes 32-byte aligned): lane l owns
+// the 16-value groups 2l + 64p and 2l + 64p + 1 (p < NG/2) instead of l + 32i,
+// so its two groups' codes are 32 contiguous bytes and every load, store and
+// read-back is one 32-byte access: half the load/store-queue entries of the
+// 16-byte form.
+template <int NG, int W, bool PAIR = false>
 __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeArgs a) {
+    static_assert(!PAIR || NG % 2 == 0, "paired groups");
+    constexpr int kStep = PAIR ? 2 : 1;  // groups handled per access
+    constexpr int kNext = PAIR ? 1 : 0;  // offset of the second group of an access
+    // lane's i-th 16-value group
+    auto grp = [](int i) -> int64_t {
+        const int l = threadIdx.x & 31;
+        return PAIR ? 2 * l + 64 * (i >> 1) + (i & 1) : l + 32 * i;
+    };
     if (!a.late_trigger) pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -296,11 +332,15 @@ __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeA
         uint4 raw[NG][2];
 #pragma unroll
         for (int i = 0; i < NG; ++i) {
-            const int64_t g = lane + 32 * i;
+            const int64_t g = grp(i);
             raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
             if (g < G) {
-                raw[i][0] = ld_stream(src + 2 * g);
-                raw[i][1] = ld_stream(src + 2 * g + 1);
+                if (PAIR) {
+                    ld_stream_pair(src + 2 * g, raw[i][0], raw[i][1]);
+                } else {
+                    raw[i][0] = ld_stream(src + 2 * g);
+                    raw[i][1] = ld_stream(src + 2 * g + 1);
+                }
             }
         }
         // amax as quantize_rows16_kernel finds it (NaNs have no magnitude)
@@ -326,8 +366,7 @@ __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeA
         // 1. codes and scale into the staging row of every node touched
         if (srow >= 0) a.staging_s[srow] = scale;
         const unsigned smask = __ballot_sync(kFullMask, srow >= 0);  // bit 31 - n: node n
-#pragma unroll
-        for (int i = 0; i < NG; ++i) {
+        auto quantize = [&](int i) {
             uint2 c[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -337,14 +376,22 @@ __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeA
                 for (int e = 0; e < 8; ++e) f[e] = f[e] * inv;
                 c[h] = to_e4m3x8(f);
             }
-            const uint4 code = make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
-            const int64_t g = lane + 32 * i;
+            return make_uint4(c[0].x, c[0].y, c[1].x, c[1].y);
+        };
+#pragma unroll
+        for (int i = 0; i < NG; i += kStep) {
+            const uint4 code = quantize(i);
+            const uint4 code2 = PAIR ? quantize(i + kNext) : code;
+            const int64_t g = grp(i);
             unsigned m = smask;
             while (m) {
                 const int j = __ffs(m) - 1;
                 m &= m - 1;
                 const int64_t d = __shfl_sync(kFullMask, srow, j);
-                if (g < G) a.staging_q[d * G + g] = code;
+                if (g < G) {
+                    if (PAIR) st_pair(a.staging_q + d * G + g, code, code2);
+                    else a.staging_q[d * G + g] = code;
+                }
             }
         }
         __syncwarp();  // the staging scales are seen by the lanes that read them back
@@ -359,9 +406,13 @@ __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeA
             if ((cols >> lane) & 1u) a.recv_s[sl] = ld_l2(a.staging_s + row_n);
             uint4 back[NG];
 #pragma unroll
-            for (int i = 0; i < NG; ++i) {
-                const int64_t g = lane + 32 * i;
-                back[i] = g < G ? ld_l2(a.staging_q + row_n * G + g) : make_uint4(0, 0, 0, 0);
+            for (int i = 0; i < NG; i += kStep) {
+                const int64_t g = grp(i);
+                back[i] = back[i + kNext] = make_uint4(0, 0, 0, 0);
+                if (g < G) {
+                    if (PAIR) ld_l2_pair(a.staging_q + row_n * G + g, back[i], back[i + kNext]);
+                    else back[i] = ld_l2(a.staging_q + row_n * G + g);
+                }
             }
             unsigned cm = cols;
             while (cm) {
@@ -369,9 +420,12 @@ __global__ void __launch_bounds__(W * 32) quantize_node_dispatch_kernel(Fp8NodeA
                 cm &= cm - 1;
                 const int64_t d = __shfl_sync(kFullMask, (int64_t)sl, q);
 #pragma unroll
-                for (int i = 0; i < NG; ++i) {
-                    const int64_t g = lane + 32 * i;
-                    if (g < G) st_stream(a.recv_q + d * G + g, back[i]);
+                for (int i = 0; i < NG; i += kStep) {
+                    const int64_t g = grp(i);
+                    if (g < G) {
+                        if (PAIR) st_stream_pair(a.recv_q + d * G + g, back[i], back[i + kNext]);
+                        else st_stream(a.recv_q + d * G + g, back[i]);
+                    }
                 }
             }
         }
@@ -644,12 +698,24 @@ cudaError_t launch_quantize_fp8(const void* src, int64_t rows, int64_t hidden, c
 }
 
 namespace {
-template <int NG, int W>
-cudaError_t launch_node_q(Fp8NodeArgs a, cudaStream_t stream) {
-    constexpr auto kern = quantize_node_dispatch_kernel<NG, W>;
+template <int NG, int W, bool PAIR>
+cudaError_t launch_node_q_form(Fp8NodeArgs a, cudaStream_t stream) {
+    constexpr auto kern = quantize_node_dispatch_kernel<NG, W, PAIR>;
     const int grid = persistent_grid<kern>(a.T, W * 32);
     a.late_trigger = pdl_trigger_at_end(grid, resident_blocks<kern>(W * 32)) ? 1 : 0;
     return launch_pdl(kern, dim3(grid), dim3(W * 32), 0, stream, a);
+}
+// The paired (32-byte) form where the groups pair up and the buffers allow
+// it (compile-time switch MOE_FP8_NODE_PAIR; 0 = never).
+#ifndef MOE_FP8_NODE_PAIR
+#define MOE_FP8_NODE_PAIR 1
+#endif
+template <int NG, int W>
+cudaError_t launch_node_q(Fp8NodeArgs a, cudaStream_t stream) {
+    const uintptr_t align = reinterpret_cast<uintptr_t>(a.src) | reinterpret_cast<uintptr_t>(a.staging_q) |
+                            reinterpret_cast<uintptr_t>(a.recv_q);
+    if (MOE_FP8_NODE_PAIR && a.G % 2 == 0 && align % 32 == 0) return launch_node_q_form<NG, W, true>(a, stream);
+    return launch_node_q_form<NG, W, false>(a, stream);
 }
 }  // namespace
 

@@ -131,6 +131,8 @@ def test_fp8_workload_olmoe(oracle_mod):
 @pytest.mark.parametrize("T,H,E,k,R,N", [
     (33, 136, 13, 4, 5, 5),         # H % 16 != 0: the split form whatever the flag
     (257, 2048, 64, 8, 4, 2),
+    (129, 1056, 32, 8, 8, 2),       # 66 groups: 32-byte accesses, a ragged last block of 64
+    (97, 1040, 32, 6, 4, 2),        # 65 groups (odd): the 16-byte form
     (600, 7168, 32, 8, 8, 4),       # 14 groups of 16 values per lane
     (300, 8192, 64, 16, 16, 16),    # N + k = 32, the one-kernel limit
 ])
