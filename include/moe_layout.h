@@ -215,8 +215,9 @@ moe_status_t moe_layout(const moe_config_t *cfg, const int32_t *topk_idx,
  * MOE_FLAG_TWO_LEVEL_SPLIT or MOE_FLAG_COPY_VECTOR, or where the one kernel
  * does not apply, a pack kernel writes the staging rows and an expansion
  * kernel reads them back.  Measured on B200 on the DeepSeek-V3-shaped
- * workload, the one-kernel form's step (layout, dispatch, combine) is 764 us
- * against 808 us for the two kernels. */
+ * workload in the same build, the one-kernel form's step (layout, dispatch,
+ * combine) took 764 us against 808 us for the two kernels; with later
+ * kernels the one-kernel step is about 719 us. */
 moe_status_t moe_dispatch(const moe_config_t *cfg, const moe_layout_t *layout,
                           const void *x, void *recv, void *node_staging,
                           void *stream);
