@@ -222,9 +222,11 @@ def test_rank_partial_combine_single_rank_equals_column_order(oracle_mod):
 
 
 def test_rank_partial_combine_order_is_rank_order(oracle_mod):
-    """fp32 addition is not associative: a token whose expert on rank 1 carries
-    -2^20 and whose experts on rank 0 carry 2^20 and 2^-9 must give the
-    rank-order result (2^20 + 2^-9 rounds to 2^20 before the -2^20 is added)."""
+    """Per-rank partials first, then their sum, not one column-order sum
+    (fp32 addition is not associative): a token whose expert on rank 1
+    carries -2^20 and whose experts on rank 0 carry 2^20 and 2^-9 gives 0
+    (rank 0's partial 2^20 + 2^-9 rounds to 2^20 before the -2^20 is added),
+    where the column-order sum gives 2^-9."""
     E, R = 4, 2                      # ranks own experts {0,1} and {2,3}
     topk = np.array([[2, 0, 1]], np.int32)
     lay = oracle_mod.layout(topk, E, R)
@@ -237,3 +239,23 @@ def test_rank_partial_combine_order_is_rank_order(oracle_mod):
     y_col = _bits_to_f64(oracle_mod.combine(eo, w, lay["slot"]))
     assert y_rs[0, 0] == 0.0          # (2^20 + 2^-9) - 2^20 in fp32 = 0
     assert y_col[0, 0] == 2.0 ** -9   # -2^20 + 2^20 + 2^-9 in column order
+
+
+def test_rank_partial_combine_adds_ranks_first_to_last(oracle_mod):
+    """Three ranks of one expert each, partials p0 = 1 + 2^-8 (weight 1 + 2^-8
+    on 1.0), p1 = p2 = 2^-24.  In rank order each 2^-24 is half an fp32 ulp of
+    the running total and rounds away (ties to even), leaving 1 + 2^-8, a bf16
+    tie that rounds to 1.0 (0x3F80).  Last rank first would add 2^-24 + 2^-24
+    = 2^-23 exactly, then 1 + 2^-8 + 2^-23, which rounds up to 0x3F81.  With
+    two ranks the order could not show: a single add commutes."""
+    E, R = 3, 3
+    topk = np.array([[0, 1, 2]], np.int32)
+    lay = oracle_mod.layout(topk, E, R)
+    assert list(lay["rank_offsets"]) == [0, 1, 2, 3]
+    vals = {0: 1.0, 1: 2.0 ** -24, 2: 2.0 ** -24}
+    eo = np.zeros((3, 1), np.uint16)
+    for j, e in enumerate(topk[0]):
+        eo[lay["slot"][0, j], 0] = oracle_mod.f32_to_bf16(np.float32(vals[int(e)])).item()
+    w = np.array([[1.0 + 2.0 ** -8, 1.0, 1.0]], np.float32)
+    y = oracle_mod.combine_rank_partials(eo, w, lay["slot"], lay["rank_offsets"])
+    assert y[0, 0] == 0x3F80

@@ -6,6 +6,7 @@ direction), builds it, and runs the oracle pin tests against that build in a
 subprocess.  The pins pass on the real oracle (the other test files), so a
 mutant passing them would mean the pins cannot see that mistake.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -75,28 +76,78 @@ MUTANTS = {
     "widening_drops_low_bit": (
         "    uint32_t u = ((uint32_t)h) << 16;",
         "    uint32_t u = ((uint32_t)(h & 0xFFFEu)) << 16;"),
+    "fp8_amax_of_signed_values": (
+        "float v = fabsf(oracle_bf16_to_f32(src[r * H + h]));",
+        "float v = oracle_bf16_to_f32(src[r * H + h]);"),
+    "e4m3_saturates_to_nan_code": (
+        "        return (uint8_t)(sign | 0x7E);",
+        "        return (uint8_t)(sign | 0x7F);"),
+    "e4m3_subnormal_scale_off": (
+        "v = ldexpf((float)man, -9);",
+        "v = ldexpf((float)man, -10);"),
+    "expert_offsets_inclusive": (
+        "        expert_offsets[e] = (int32_t)run;\n        run += expert_counts[e];",
+        "        run += expert_counts[e];\n        expert_offsets[e] = (int32_t)run;"),
+    "rank_offsets_from_expert_index": (
+        "    if (first == NULL)\n        return ORC_INVALID_ARG;\n    oracle_partition(E, R, first);\n"
+        "    for (int32_t r = 0; r <= R; ++r)\n        rank_offsets[r] = expert_offsets[first[r]];",
+        "    if (first == NULL)\n        return ORC_INVALID_ARG;\n    oracle_partition(E, R, first);\n"
+        "    for (int32_t r = 0; r <= R; ++r)\n        rank_offsets[r] = first[r];"),
+    "validation_accepts_expert_E": (
+        "            if (e < 0 || e >= E)\n                return ORC_EXPERT_OOB;",
+        "            if (e < 0 || e > E)\n                return ORC_EXPERT_OOB;"),
+    "node_cursor_counts_every_token": (
+        "                if (touched) {\n                    node_slot[t * N + n] = ncursor[n];\n                    ncursor[n] += 1;\n                } else {\n                    node_slot[t * N + n] = -1;\n                }",
+        "                node_slot[t * N + n] = touched ? ncursor[n] : -1;\n                ncursor[n] += 1;"),
+    "rank_partials_rounded_before_sum": (
+        "                total = total + part;",
+        "                total = total + oracle_bf16_to_f32(oracle_f32_to_bf16(part));"),
+    "rank_partials_reverse_rank_order": (
+        "            for (int32_t r = 0; r < R; ++r) {\n                float part = 0.0f;",
+        "            for (int32_t r = R - 1; r >= 0; --r) {\n                float part = 0.0f;"),
+    "fp8_dispatch_inverse_scale": (
+        "            recv_scale[dst] = st;",
+        "            recv_scale[dst] = 1.0f / st;"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+PIN_FILES = ["test_oracle_partition.py", "test_oracle_layout.py", "test_oracle_dispatch_combine.py",
+             "test_oracle_fp8.py", "test_oracle_ep.py", "test_oracle_properties.py"]
+
+
+def _run_mutant(name, workdir):
+    """Build the oracle with one planted mistake and run the pins on it;
+    returns (returncode of the pin run, the end of its output)."""
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation anchor for {name} must occur once"
-    mutant_c = tmp_path / "mutant.c"
-    mutant_c.write_text(src.replace(old, new))
-    lib = tmp_path / "libmutant.so"
+    if src.count(old) != 1:
+        return None, f"mutation anchor for {name} must occur once"
+    mutant_c = os.path.join(workdir, "mutant.c")
+    with open(mutant_c, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(workdir, "libmutant.so")
     subprocess.run(["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-shared", "-fPIC",
-                    "-o", str(lib), str(mutant_c), "-lm"], check=True)
-    env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
+                    "-o", lib, mutant_c, "-lm"], check=True)
+    env = dict(os.environ, MOE_ORACLE_LIB=lib)
     cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-           "-k", "not full_workloads",
-           os.path.join(ROOT, "tests", "test_oracle_partition.py"),
-           os.path.join(ROOT, "tests", "test_oracle_layout.py"),
-           os.path.join(ROOT, "tests", "test_oracle_dispatch_combine.py"),
-           os.path.join(ROOT, "tests", "test_oracle_fp8.py"),
-           os.path.join(ROOT, "tests", "test_oracle_ep.py"),
-           os.path.join(ROOT, "tests", "test_oracle_properties.py")]
+           "-k", "not full_workloads", *[os.path.join(ROOT, "tests", p) for p in PIN_FILES]]
     res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert res.returncode == 1, (
-        f"mutant {name} passed every pin:\n{res.stdout[-2000:]}\n{res.stderr[-2000:]}")
+    return res.returncode, res.stdout[-2000:] + res.stderr[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Every mutant's pin run, run concurrently (each is its own build and
+    process, so they share nothing)."""
+    names = sorted(MUTANTS)
+    dirs = {n: str(tmp_path_factory.mktemp(n)) for n in names}
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
+        futures = {n: ex.submit(_run_mutant, n, dirs[n]) for n in names}
+        return {n: f.result() for n, f in futures.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, mutant_runs):
+    rc, out = mutant_runs[name]
+    assert rc is not None, out
+    assert rc == 1, f"mutant {name} passed every pin:\n{out}"
